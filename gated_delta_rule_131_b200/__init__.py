@@ -1,0 +1,135 @@
+"""gdn2 -- Gated Delta Rule-2 kernels for NVIDIA B200 (sm_100a).
+
+Thin Python binding of the C ABI in ``include/gdn2.h``: argument marshalling
+only.  Every step of the computation runs in the CUDA library
+``_build/libgdn2.so``; PyTorch provides device memory and streams.  There is
+no CPU fallback: if the library is missing or no GPU is present the calls
+raise.
+
+Entry points (same names as the C ABI):
+
+* :func:`chunk_fwd` -- chunkwise parallel forward over whole sequences
+  (``gdn2_chunk_fwd``);
+* :func:`decode_step` -- one recurrent step for a batch of single tokens
+  (``gdn2_decode_step``).
+"""
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_build", "libgdn2.so")
+
+GDN2_OK, GDN2_ERR_INVALID_ARG, GDN2_ERR_UNSUPPORTED, GDN2_ERR_CUDA, GDN2_ERR_TIMEOUT = range(5)
+GDN2_F32, GDN2_BF16 = 0, 1
+_DTYPES = {torch.float32: GDN2_F32, torch.bfloat16: GDN2_BF16}
+
+_lib = None
+
+
+class Gdn2Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lib().gdn2_status_string(status).decode()}")
+
+
+def lib():
+    """The loaded ctypes library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"gdn2 CUDA library not built ({LIB_PATH} missing); "
+                               "run `python -m gated_delta_rule_131_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, ci = ctypes.c_void_p, ctypes.c_int
+        L.gdn2_chunk_fwd.argtypes = [vp] * 9 + [ci] * 6 + [vp, ci, vp]
+        L.gdn2_chunk_fwd.restype = ci
+        L.gdn2_decode_step.argtypes = [vp] * 8 + [ci] * 5 + [vp]
+        L.gdn2_decode_step.restype = ci
+        L.gdn2_status_string.argtypes = [ci]
+        L.gdn2_status_string.restype = ctypes.c_char_p
+        L.gdn2_launch_count.argtypes = []
+        L.gdn2_launch_count.restype = ctypes.c_uint64
+        _lib = L
+    return _lib
+
+
+def launch_count() -> int:
+    """Kernel launches issued by the library so far in this process."""
+    return int(lib().gdn2_launch_count())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_tensors(*ts):
+    dev = None
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("gdn2: all tensors must be CUDA tensors")
+        if not t.is_contiguous():
+            raise ValueError("gdn2: all tensors must be contiguous")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError("gdn2: tensors on different devices")
+
+
+def chunk_fwd(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, chunk=64, o=None, S_T=None,
+              output_final_state=True, stream=None):
+    """Chunkwise forward.  Returns ``(o, S_T)`` (``S_T`` None if not requested).
+
+    Dense: q, k, alpha, b ``[B, T, H, d_k]``; v, w ``[B, T, H, d_v]``.
+    Packed (``cu_seqlens`` int32 ``[N+1]`` on the device): ``[T_total, H, d]``.
+    ``S0`` / ``S_T``: ``[N, H, d_k, d_v]`` float32.
+    """
+    if cu_seqlens is None:
+        B, T, H, dk = q.shape
+    else:
+        if cu_seqlens.dtype != torch.int32:
+            raise ValueError("gdn2: cu_seqlens must be int32")
+        B = cu_seqlens.numel() - 1
+        T, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype not in _DTYPES or any(x.dtype != q.dtype for x in (k, v, alpha, b, w)):
+        raise ValueError("gdn2: q, k, v, alpha, b, w must share dtype float32 or bfloat16")
+    if o is None:
+        o = torch.empty(q.shape[:-1] + (dv,), dtype=q.dtype, device=q.device)
+    if S_T is None and output_final_state:
+        S_T = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    if S0 is not None and S0.dtype != torch.float32:
+        raise ValueError("gdn2: S0 must be float32")
+    _check_tensors(q, k, v, alpha, b, w, S0, o, S_T, cu_seqlens)
+    st = lib().gdn2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0),
+                              _ptr(o), _ptr(S_T), B, T, H, dk, dv, chunk, _ptr(cu_seqlens),
+                              _DTYPES[q.dtype], _stream(stream))
+    if st != GDN2_OK:
+        raise Gdn2Error(st, "gdn2_chunk_fwd")
+    return o, S_T
+
+
+def decode_step(q, k, v, alpha, b, w, S, o=None, stream=None):
+    """One decode step: updates ``S`` ``[B, H, d_k, d_v]`` in place, returns ``o`` ``[B, H, d_v]``."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype not in _DTYPES or any(x.dtype != q.dtype for x in (k, v, alpha, b, w)):
+        raise ValueError("gdn2: q, k, v, alpha, b, w must share dtype float32 or bfloat16")
+    if S.dtype != torch.float32:
+        raise ValueError("gdn2: S must be float32")
+    if o is None:
+        o = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
+    _check_tensors(q, k, v, alpha, b, w, S, o)
+    st = lib().gdn2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S),
+                                _ptr(o), B, H, dk, dv, _DTYPES[q.dtype], _stream(stream))
+    if st != GDN2_OK:
+        raise Gdn2Error(st, "gdn2_decode_step")
+    return o

@@ -1,0 +1,61 @@
+// Shared device helpers of the gdn2 CUDA library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn2 {
+
+// Arguments of one gdn2_chunk_fwd call, already validated by the API layer.
+struct ChunkArgs {
+  const void *q, *k, *v, *alpha, *b, *w;
+  const float *S0;
+  void *o;
+  float *ST;
+  const int32_t *cu;  // device offsets [B+1] or nullptr
+  int B, T, H, dk, dv;
+};
+
+// Arguments of one gdn2_decode_step call.
+struct DecodeArgs {
+  const void *q, *k, *v, *alpha, *b, *w;
+  float *S;
+  void *o;
+  int B, H, dk, dv;
+};
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ float warp_allreduce_sum(float x) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+  return x;
+}
+
+// Token span of sequence n: dense batches use n*T .. n*T+T-1, packed ones cu[n] .. cu[n+1]-1.
+__device__ __forceinline__ void seq_span(const ChunkArgs &a, int n, int64_t &bos, int &len) {
+  if (a.cu) {
+    bos = a.cu[n];
+    len = a.cu[n + 1] - a.cu[n];
+  } else {
+    bos = (int64_t)n * a.T;
+    len = a.T;
+  }
+}
+
+// Host side: every kernel launch of the library is counted here.
+void note_launch();
+
+// Launchers (return the CUDA error of the launch).
+cudaError_t launch_chunk_simt(const ChunkArgs &a, bool bf16, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs &a, bool bf16, cudaStream_t stream);
+
+}  // namespace gdn2

@@ -1,0 +1,123 @@
+/*
+ * gdn2.h -- C ABI of the Gated Delta Rule-2 kernels for NVIDIA B200 (sm_100a).
+ *
+ * The operation (for one sequence and one head; state S is d_k x d_v, row =
+ * key channel, column = value channel; a_t = b_t (.) k_t, u_t = w_t (.) v_t):
+ *
+ *     S_t = Diag(alpha_t) S_{t-1}                         decay on the key axis, first
+ *         + k_t ( u_t - (Diag(alpha_t) S_{t-1})^T a_t )^T erase gated per key channel by b_t,
+ *                                                         write gated per value channel by w_t
+ *     o_t = S_t^T q_t                                     readout of the edited state
+ *
+ * Defined by the pages on "Gated DeltaNet-2: Decoupling Erase and Write in
+ * Linear Attention" (arXiv 2605.22791):
+ *   - "NVIDIA AIがGated DeltaNet-2を発表" (ai.warp-studio.com), section
+ *     "Gated DeltaNet-2の核心": b_t per key channel, w_t per value channel,
+ *     both sigmoid projections, decay before the active edit; KDA is the case
+ *     b_t = w_t = one scalar, Gated DeltaNet additionally a scalar decay;
+ *   - "[논문] 게이트형 DeltaNet-2" (euno.news), section "방법론", steps 1-4:
+ *     linear-attention read, the two gates, KDA-style per-channel decay,
+ *     chunkwise WY update for parallel training;
+ *   - "Gated DeltaNet-2: Separando Borrado y Escritura en la Atención Lineal"
+ *     (needhelp.icu), "Innovaciones Técnicas", item 1: the chunkwise algorithm
+ *     folds the per-channel decay into asymmetric erase factors.
+ * The pages print no equation; the erase is read as k_t (b_t (.) k_t)^T, the
+ * readout as S_t^T q_t with no 1/sqrt(d_k) scale.
+ *
+ * Conventions shared by every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, 16-byte
+ *     aligned, densely packed row-major.  The library keeps no state between
+ *     calls and allocates no device memory.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and never synchronise.  A validation failure returns before any
+ *     launch and writes nothing.  A launch failure returns GDN2_ERR_CUDA.  No
+ *     C++ exception crosses this interface.
+ *   - q, k, v, alpha, b, w and o share one element type `dtype` (fp32 or bf16);
+ *     states are always fp32.  alpha holds decay values in (0, 1] (the log is
+ *     never taken by the caller); b and w hold gate values (already sigmoid-ed);
+ *     q and k are used as given (the token mixer normalises them before).
+ *   - Supported head sizes: d_k in {64, 128}, d_v in {64, 128, 256}; anything
+ *     else returns GDN2_ERR_UNSUPPORTED.
+ */
+#ifndef GDN2_H
+#define GDN2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GDN2_API __attribute__((visibility("default")))
+#else
+#define GDN2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GDN2_OK = 0,
+  GDN2_ERR_INVALID_ARG = 1, /* null / misaligned pointer, negative or overflowing size */
+  GDN2_ERR_UNSUPPORTED = 2, /* valid but not implemented: head size, chunk size, dtype */
+  GDN2_ERR_CUDA = 3,        /* a CUDA launch or attribute call failed                 */
+  GDN2_ERR_TIMEOUT = 4      /* reserved: a bounded device-side wait gave up            */
+} gdn2_status;
+
+typedef enum { GDN2_F32 = 0, GDN2_BF16 = 1 } gdn2_dtype;
+
+/* Same type as cudaStream_t, declared here so the header needs no CUDA include. */
+typedef struct CUstream_st *gdn2_stream_t;
+
+/*
+ * gdn2_chunk_fwd -- chunkwise parallel forward (prefill / training forward).
+ *
+ * Computes o_t for every token and the final state of every sequence, using
+ * the chunkwise WY form: inside a chunk of `chunk` tokens the per-channel decay
+ * is folded into the erase factors and the chunk's erase interactions form one
+ * unit-lower-triangular system; the state is carried across chunks in fp32.
+ * The result equals the token-by-token recurrence up to rounding.
+ *
+ * Layout, dense batch (cu_seqlens == NULL): B sequences of T tokens each;
+ *   q, k, alpha, b : [B, T, H, d_k]     v, w, o : [B, T, H, d_v]
+ * Layout, packed varlen (cu_seqlens != NULL): B sequences packed end to end,
+ *   T = total tokens = cu_seqlens[B]; cu_seqlens is a DEVICE int32 array of
+ *   B+1 non-decreasing offsets starting at 0 (not read on the host; a
+ *   violation of this precondition is undefined);
+ *   q, k, alpha, b : [T, H, d_k]        v, w, o : [T, H, d_v]
+ * States: S0, S_T : [B, H, d_k, d_v] fp32 (d_v contiguous).
+ *   S0 == NULL means a zero initial state; S_T == NULL skips the final state;
+ *   S_T may alias S0 (the state is read before it is overwritten).
+ * chunk: 64 (the only supported chunk length).
+ * T == 0 (or an empty sequence) is valid: its S_T equals its S0; when the
+ * batch holds no token at all, the token pointers (q .. w, o) may be NULL.
+ * Returns GDN2_OK, or an error status with nothing launched.
+ */
+GDN2_API gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *alpha,
+                           const void *b, const void *w, const float *S0, void *o, float *S_T,
+                           int B, int T, int H, int d_k, int d_v, int chunk,
+                           const int32_t *cu_seqlens, gdn2_dtype dtype, gdn2_stream_t stream);
+
+/*
+ * gdn2_decode_step -- one recurrent step for a batch of single tokens.
+ *
+ * For every (batch entry, head): S <- the edited state after one token; o <- S^T q.
+ * The state is read once and written once (memory-bound).
+ *   q, k, alpha, b : [B, H, d_k]     v, w, o : [B, H, d_v]
+ *   S              : [B, H, d_k, d_v] fp32, updated in place.
+ * o must not overlap S or the inputs.
+ */
+GDN2_API gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v, const void *alpha,
+                             const void *b, const void *w, float *S, void *o, int B, int H,
+                             int d_k, int d_v, gdn2_dtype dtype, gdn2_stream_t stream);
+
+/* Human-readable name of a status; never NULL. */
+GDN2_API const char *gdn2_status_string(gdn2_status status);
+
+/* Number of kernel launches this library has issued in this process (all calls, all threads). */
+GDN2_API uint64_t gdn2_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN2_H */
