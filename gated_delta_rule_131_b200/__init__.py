@@ -49,6 +49,8 @@ def lib():
         L.gdn2_decode_step.restype = ci
         L.gdn2_status_string.argtypes = [ci]
         L.gdn2_status_string.restype = ctypes.c_char_p
+        L.gdn2_device_status.argtypes = [ci]
+        L.gdn2_device_status.restype = ci
         L.gdn2_launch_count.argtypes = []
         L.gdn2_launch_count.restype = ctypes.c_uint64
         _lib = L
@@ -58,6 +60,11 @@ def lib():
 def launch_count() -> int:
     """Kernel launches issued by the library so far in this process."""
     return int(lib().gdn2_launch_count())
+
+
+def device_status(reset=False) -> int:
+    """Sticky device-side status (GDN2_OK or GDN2_ERR_TIMEOUT); synchronises with the device."""
+    return int(lib().gdn2_device_status(1 if reset else 0))
 
 
 def _ptr(t):

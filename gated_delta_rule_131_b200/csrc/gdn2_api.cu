@@ -46,6 +46,12 @@ const char *gdn2_status_string(gdn2_status s) {
 
 uint64_t gdn2_launch_count(void) { return gdn2::g_launches.load(std::memory_order_relaxed); }
 
+gdn2_status gdn2_device_status(int reset) {
+  int st = 0;
+  if (gdn2::read_device_status(&st, reset != 0) != cudaSuccess) return GDN2_ERR_CUDA;
+  return st == 0 ? GDN2_OK : GDN2_ERR_TIMEOUT;
+}
+
 gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *alpha,
                            const void *b, const void *w, const float *S0, void *o, float *S_T,
                            int B, int T, int H, int d_k, int d_v, int chunk,
@@ -66,7 +72,11 @@ gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v, const vo
   if (B == 0) return GDN2_OK;
 
   gdn2::ChunkArgs a{q, k, v, alpha, b, w, S0, o, S_T, cu_seqlens, B, T, H, d_k, d_v};
-  const cudaError_t err = gdn2::launch_chunk_simt(a, dtype == GDN2_BF16, (cudaStream_t)stream);
+  const bool bf16 = dtype == GDN2_BF16;
+  // bf16 with d_k = 128 runs on the tensor cores; fp32 (whose accuracy bf16 operands cannot
+  // keep) and d_k = 64 run the SIMT kernel
+  const cudaError_t err = gdn2::chunk_tc_supported(a, bf16) ? gdn2::launch_chunk_tc(a, (cudaStream_t)stream)
+                                                            : gdn2::launch_chunk_simt(a, bf16, (cudaStream_t)stream);
   return err == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
 }
 

@@ -113,6 +113,16 @@ GDN2_API gdn2_status gdn2_decode_step(const void *q, const void *k, const void *
 /* Human-readable name of a status; never NULL. */
 GDN2_API const char *gdn2_status_string(gdn2_status status);
 
+/*
+ * gdn2_device_status -- the sticky device-side status of the tensor-core kernels.
+ * Their waits on asynchronous copies and tensor-core completions are bounded
+ * (2 s); a wait that gives up makes the kernel skip the rest of its work, free
+ * its tensor memory and record GDN2_ERR_TIMEOUT here.  Synchronises with the
+ * device (it copies one int).  reset != 0 clears the word after reading it.
+ * Returns GDN2_OK, GDN2_ERR_TIMEOUT, or GDN2_ERR_CUDA if the copy failed.
+ */
+GDN2_API gdn2_status gdn2_device_status(int reset);
+
 /* Number of kernel launches this library has issued in this process (all calls, all threads). */
 GDN2_API uint64_t gdn2_launch_count(void);
 
