@@ -9,10 +9,11 @@
 //   [L; P]    = [A_m; Q_m] K_m^T                   L strictly, P inclusively lower
 //   T         = (I + L)^-1                         fp32 blocked forward substitution
 //   Delta     = T U - T A_m (e^m S)                U = w (.) v
-//   O         = Q S + P Delta = [P T] U + (Q_m - [P T] A_m) (e^m S)
+//   O         = Q S + P Delta = Q_m (e^m S) + P Delta
 //   S_next    = e^{g_C} S + e^{g_C - m} K_m^T Delta
-// so one tensor-core pass per chunk forms, in TMEM,
-//   D_a = [T U; P T U] + [-T A_m; Q_m - P T A_m] (e^m S) = [Delta; O].
+// so, in TMEM, D_a = [T U; 0] + [-T A_m; Q_m] (e^m S) = [Delta; Q S], then
+// D_a += [P; P] Delta leaves O in its lower half (the upper half, Delta, has
+// been read out by then).
 // The decay-absorbed asymmetric erase factors follow the block formulation of
 // "Gated DeltaNet-2: Separando Borrado y Escritura en la Atención Lineal"
 // (needhelp.icu), "Innovaciones Técnicas", item 1; the update itself is the
@@ -20,14 +21,17 @@
 // "Gated DeltaNet-2の核心" (decay first, key-side erase gate b, value-side write
 // gate w, o_t = S_t^T q_t).
 //
-// One CTA per (sequence, head, 64 value columns); 256 threads; 2 CTAs per SM.
+// One CTA per (sequence, head, 64 value columns); 256 threads.
 // Shared memory holds every operand in the 128-byte-swizzled layout that TMA
 // writes and tcgen05.mma reads, so the raw q, k, b tiles are turned into the
 // factor operands in place.  The state slice lives in fp32 registers (thread =
 // key channel x 32 value columns); TMEM holds the MMA accumulators:
-//   cols [0, 64)    L|P, then P T, then K_m^T Delta
-//   cols [64, 192)  [T; P T] A_m
+//   cols [0, 64)    L|P, then K_m^T Delta
+//   cols [64, 192)  [T; 0] A_m
 //   cols [192, 256) D_a = [Delta; O]
+// T is formed in fp32: the four 16x16 diagonal blocks by right-looking
+// substitution, then merged into 32x32 and 64x64 inverses with
+// [[A,0],[C,B]]^-1 = [[A^-1,0],[-B^-1 C A^-1, B^-1]].
 // Precondition of the factorisation: per key channel, the decay accumulated
 // over any 32 consecutive tokens of a chunk stays above about e^-80 (the fp32
 // range); every workload here is far inside it.
@@ -55,18 +59,23 @@ using namespace ptx;
 
 constexpr int C = 64, DK = 128, NV = 64, NT = 256;
 
-// shared-memory map (bytes from a 1024-aligned base)
-constexpr uint32_t XA_BLK = 16384;            // [A_m ; Q_m] 128 rows x 64 ch, two channel blocks
-constexpr uint32_t KT_BLK = 8192;             // K_m 64 rows x 64 ch, two channel blocks
+// shared-memory map (bytes from a 1024-aligned base); every MMA operand tile is 1024-aligned
+constexpr uint32_t XA_BLK = 16384;                 // [A_m | -T A_m ; Q_m] 128 rows x 64 ch, two channel blocks
+constexpr uint32_t KT_BLK = 8192;                  // K_m 64 rows x 64 ch, two channel blocks
 constexpr uint32_t OFF_XA = 0;
 constexpr uint32_t OFF_KT = OFF_XA + 2 * XA_BLK;   // 32768
-constexpr uint32_t OFF_AL = OFF_KT + 2 * KT_BLK;   // 49152: alpha tiles, then T (fp32 64x64)
-constexpr uint32_t OFF_U = OFF_AL + 16384;         // 65536: v tile -> U
-constexpr uint32_t OFF_W = OFF_U + 8192;           // 73728: w tile    } L (fp32 64x64) spans
-constexpr uint32_t OFF_DL = OFF_W + 8192;          // 81920: Delta     }   both slots
-constexpr uint32_t OFF_TP = OFF_DL + 8192;         // 90112: [T ; P | P T] 128 x 64, later e^m S
-constexpr uint32_t OFF_SC = OFF_TP + 16384;        // 106496: decay products and per-channel scalars
-constexpr uint32_t OFF_BAR = OFF_SC + 4 * 128 * 4 + 3 * 128 * 4;  // 110080
+constexpr uint32_t OFF_AL = OFF_KT + 2 * KT_BLK;   // 49152: alpha tiles (two blocks)
+constexpr uint32_t OFF_U = OFF_AL + 16384;         // 65536: v tile -> U = w (.) v
+constexpr uint32_t OFF_W = OFF_U + 8192;           // 73728: w tile
+constexpr uint32_t OFF_DL = OFF_W + 8192;          // 81920: Delta, bf16 64 x 64
+constexpr uint32_t OFF_TZ = OFF_DL + 8192;         // 90112: [T ; 0] bf16 128 x 64
+constexpr uint32_t OFF_PP = OFF_TZ + 16384;        // 106496: [P ; P] bf16 128 x 64
+constexpr uint32_t OFF_SM = OFF_PP + 16384;        // 122880: e^m S, bf16 128 x 64
+constexpr int LDF = 68;                            // row stride of the fp32 64 x 64 scratch
+constexpr uint32_t OFF_LS = OFF_SM + 16384;        // 139264: L (fp32), upper blocks reused as scratch
+constexpr uint32_t OFF_TS = OFF_LS + 64 * LDF * 4; // 156672: T (fp32)
+constexpr uint32_t OFF_SC = OFF_TS + 64 * LDF * 4; // 174080: decay products and per-channel scalars
+constexpr uint32_t OFF_BAR = OFF_SC + 16 * 128 * 4 + 3 * 128 * 4;
 constexpr uint32_t SMEM_USED = OFF_BAR + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for aligning the base
 constexpr uint32_t TMA_BYTES = 10 * 8192;          // q, k, b, alpha (2 boxes each), v, w
@@ -78,12 +87,12 @@ constexpr uint32_t ID_KM64 = idesc_bf16(128, 64, false, true);   // K-major A, M
 constexpr uint32_t ID_KM128 = idesc_bf16(128, 128, false, true); // same, N = 128
 constexpr uint32_t ID_MNMN = idesc_bf16(128, 64, true, true);    // K_m^T Delta
 
-// fp32 64x64 scratch with the column index XOR-swizzled by the row, so that a warp
-// writing one column across 32 rows hits 32 different banks
-__device__ __forceinline__ float &f64x64(float *base, int r, int c) { return base[r * 64 + (c ^ (r & 31))]; }
-
 __device__ __forceinline__ uint4 ld_s128(const uint8_t *p) { return *reinterpret_cast<const uint4 *>(p); }
 __device__ __forceinline__ void st_s128(uint8_t *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
+__device__ __forceinline__ uint4 pack8(const float *e) {
+  return make_uint4(f2_to_bf2(e[0], e[1]), f2_to_bf2(e[2], e[3]), f2_to_bf2(e[4], e[5]), f2_to_bf2(e[6], e[7]));
+}
+__device__ __forceinline__ float fast_rcp(float x) { return __fdividef(1.f, x); }
 
 // Every thread waits; the CTA then agrees on the outcome (so control flow stays uniform).
 __device__ __forceinline__ bool cta_wait(uint32_t bar, uint32_t parity) {
@@ -91,22 +100,46 @@ __device__ __forceinline__ bool cta_wait(uint32_t bar, uint32_t parity) {
   return !__syncthreads_or(!ok);
 }
 
-template <typename Tout>
-__device__ __forceinline__ void store_row32(Tout *dst, const float (&v)[32]);
-template <>
-__device__ __forceinline__ void store_row32<__nv_bfloat16>(__nv_bfloat16 *dst, const float (&v)[32]) {
+__device__ __forceinline__ void store_row32_bf16(__nv_bfloat16 *dst, const float (&v)[32]) {
 #pragma unroll
-  for (int x = 0; x < 4; ++x) {
-    uint4 u;
-    u.x = f2_to_bf2(v[8 * x + 0], v[8 * x + 1]);
-    u.y = f2_to_bf2(v[8 * x + 2], v[8 * x + 3]);
-    u.z = f2_to_bf2(v[8 * x + 4], v[8 * x + 5]);
-    u.w = f2_to_bf2(v[8 * x + 6], v[8 * x + 7]);
-    reinterpret_cast<uint4 *>(dst)[x] = u;
-  }
+  for (int x = 0; x < 4; ++x) reinterpret_cast<uint4 *>(dst)[x] = pack8(&v[8 * x]);
 }
 
-__global__ void __launch_bounds__(NT, 2)
+__device__ __forceinline__ void unpack8(uint4 u, float *e) {
+  float2 t = bf2_to_f2(u.x); e[0] = t.x; e[1] = t.y;
+  t = bf2_to_f2(u.y); e[2] = t.x; e[3] = t.y;
+  t = bf2_to_f2(u.z); e[4] = t.x; e[5] = t.y;
+  t = bf2_to_f2(u.w); e[6] = t.x; e[7] = t.y;
+}
+
+// Decay-absorbed operands of one token row for 8 key channels, in place:
+// A_m = b k f, Q_m = q f, K_m = k fi with f = e^{g_r - m}, fi = 1/f; rows >= Cc are zeroed.
+__device__ __forceinline__ void row_factors(uint8_t *sm, int r, int cb, int x8, int Cc, const float *f, const float *fi) {
+  uint8_t *pa = sm + OFF_XA + cb * XA_BLK + sw128(r, 8 * x8);
+  uint8_t *pq = pa + 8192;
+  uint8_t *pk = sm + OFF_KT + cb * KT_BLK + sw128(r, 8 * x8);
+  uint4 wa = make_uint4(0u, 0u, 0u, 0u), wq = wa, wk = wa;
+  if (r < Cc) {
+    float bb[8], qv[8], kv[8], ea[8], eq[8], ek[8];
+    unpack8(ld_s128(pa), bb);
+    unpack8(ld_s128(pq), qv);
+    unpack8(ld_s128(pk), kv);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      ea[t] = bb[t] * kv[t] * f[t];
+      eq[t] = qv[t] * f[t];
+      ek[t] = kv[t] * fi[t];
+    }
+    wa = pack8(ea);
+    wq = pack8(eq);
+    wk = pack8(ek);
+  }
+  st_s128(pa, wa);
+  st_s128(pq, wq);
+  st_s128(pk, wk);
+}
+
+__global__ void __launch_bounds__(NT, 1)
     chunk_fwd_tc_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ CUtensorMap tm_al, const __grid_constant__ CUtensorMap tm_v,
@@ -114,14 +147,14 @@ __global__ void __launch_bounds__(NT, 2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(sm);
-  float *pp = reinterpret_cast<float *>(sm + OFF_SC);  // [4][128] decay product of each 16-token quarter
-  float *s_em = pp + 512;                              // e^m       (decay from chunk start to token 31)
+  float *pp = reinterpret_cast<float *>(sm + OFF_SC);  // [16][128] decay product of each 4-token group
+  float *s_em = pp + 16 * 128;                         // e^m       (decay from chunk start to token 31)
   float *s_egcm = s_em + 128;                          // e^{g_C-m} (decay over tokens 32..end)
   float *s_egc = s_egcm + 128;                         // e^{g_C}   (decay over the whole chunk)
   const uint32_t bar_ld = sb + OFF_BAR, bar_mma = sb + OFF_BAR + 8;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 16);
-  float *Ls = reinterpret_cast<float *>(sm + OFF_W);
-  float *Ts = reinterpret_cast<float *>(sm + OFF_AL);
+  float *Ls = reinterpret_cast<float *>(sm + OFF_LS);
+  float *Ts = reinterpret_cast<float *>(sm + OFF_TS);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, quad = warp & 3, half = warp >> 2;
   const int tiles = a.dv / NV;
@@ -145,6 +178,10 @@ __global__ void __launch_bounds__(NT, 2)
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
+  // zero rows 64..127 of [T ; 0] once, and the never-written upper blocks of T
+  for (int e = tid; e < 8192 / 16; e += NT) st_s128(sm + OFF_TZ + 8192 + 16 * e, make_uint4(0u, 0u, 0u, 0u));
+  for (int e = tid; e < 64 * LDF; e += NT) Ts[e] = 0.f;
+  fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -190,67 +227,75 @@ __global__ void __launch_bounds__(NT, 2)
     ph_ld ^= 1;
 
     // ---------------------------------------------------------------- B: decay factors, operands
-    const int cp = tid & 63, qq = tid >> 6;  // channel pair (2cp, 2cp+1), token quarter qq
-    const int cb = (2 * cp) >> 6, cc = (2 * cp) & 63;
     {
-      float p0 = 1.f, p1 = 1.f;
-#pragma unroll 4
-      for (int rr = 0; rr < 16; ++rr) {
-        const int r = 16 * qq + rr;
+      // thread = 8 key channels (chunk x8 of channel block cb) x 4 tokens (group G = rows 4G..4G+3);
+      // warps 0-3 hold tokens 0..31 (walk back to token 31), warps 4-7 tokens 32..63 (walk forward)
+      const int ch8 = tid & 15, G = tid >> 4, cb = ch8 >> 3, x8 = ch8 & 7;
+      float al[4][8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = 4 * G + i;
         if (r < Cc) {
-          const float2 al = bf2_to_f2(*reinterpret_cast<const uint32_t *>(sm + OFF_AL + cb * 8192 + sw128(r, cc)));
-          p0 *= al.x;
-          p1 *= al.y;
+          unpack8(ld_s128(sm + OFF_AL + cb * 8192 + sw128(r, 8 * x8)), al[i]);
+        } else {
+#pragma unroll
+          for (int t = 0; t < 8; ++t) al[i][t] = 1.f;
         }
       }
-      pp[qq * 128 + 2 * cp] = p0;
-      pp[qq * 128 + 2 * cp + 1] = p1;
-    }
-    __syncthreads();
-    if (tid < 128) {
-      const float em = pp[tid] * pp[128 + tid], egcm = pp[256 + tid] * pp[384 + tid];
-      s_em[tid] = em;
-      s_egcm[tid] = egcm;
-      s_egc[tid] = em * egcm;
-    }
-    {
-      // f_r = e^{g_r - m}: tokens 0..31 walk backwards from token 31, tokens 32..63 forwards
-      float2 run;
-      if (qq == 0) run = make_float2(pp[128 + 2 * cp], pp[128 + 2 * cp + 1]);
-      else if (qq == 3) run = make_float2(pp[256 + 2 * cp], pp[256 + 2 * cp + 1]);
-      else run = make_float2(1.f, 1.f);
-#pragma unroll 2
-      for (int s = 0; s < 16; ++s) {
-        const int r = (qq < 2) ? (16 * qq + 15 - s) : (16 * qq + s);
-        const uint32_t oa = OFF_XA + cb * XA_BLK + sw128(r, cc);
-        const uint32_t oq = oa + 8192;
-        const uint32_t ok_ = OFF_KT + cb * KT_BLK + sw128(r, cc);
-        float2 al = make_float2(1.f, 1.f);
-        if (r < Cc) al = bf2_to_f2(*reinterpret_cast<const uint32_t *>(sm + OFF_AL + cb * 8192 + sw128(r, cc)));
-        float2 f, fi;
-        if (qq < 2) {
-          fi = run;
-          f = make_float2(__frcp_rn(run.x), __frcp_rn(run.y));
-          run.x *= al.x;
-          run.y *= al.y;
-        } else {
-          run.x *= al.x;
-          run.y *= al.y;
-          f = run;
-          fi = make_float2(__frcp_rn(run.x), __frcp_rn(run.y));
+      float gp[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) gp[t] = al[0][t] * al[1][t] * al[2][t] * al[3][t];
+      float *scan = pp;  // [16 groups][128 channels]: product of alpha over each 4-token group
+      *reinterpret_cast<float4 *>(&scan[G * 128 + 8 * ch8]) = make_float4(gp[0], gp[1], gp[2], gp[3]);
+      *reinterpret_cast<float4 *>(&scan[G * 128 + 8 * ch8 + 4]) = make_float4(gp[4], gp[5], gp[6], gp[7]);
+      __syncthreads();
+      if (tid < 128) {
+        float em = 1.f, egcm = 1.f;
+        for (int g = 0; g < 8; ++g) em *= scan[g * 128 + tid];
+        for (int g = 8; g < 16; ++g) egcm *= scan[g * 128 + tid];
+        s_em[tid] = em;
+        s_egcm[tid] = egcm;
+        s_egc[tid] = em * egcm;
+      }
+      float run[8];  // product of alpha strictly between this group and token 31 (inclusive of 31)
+#pragma unroll
+      for (int t = 0; t < 8; ++t) run[t] = 1.f;
+      if (G < 8) {
+        for (int g = G + 1; g < 8; ++g) {
+          const float4 p0 = *reinterpret_cast<const float4 *>(&scan[g * 128 + 8 * ch8]);
+          const float4 p1 = *reinterpret_cast<const float4 *>(&scan[g * 128 + 8 * ch8 + 4]);
+          run[0] *= p0.x; run[1] *= p0.y; run[2] *= p0.z; run[3] *= p0.w;
+          run[4] *= p1.x; run[5] *= p1.y; run[6] *= p1.z; run[7] *= p1.w;
         }
-        uint32_t wa = 0u, wq = 0u, wk = 0u;
-        if (r < Cc) {
-          const float2 bb = bf2_to_f2(*reinterpret_cast<const uint32_t *>(sm + oa));
-          const float2 qv = bf2_to_f2(*reinterpret_cast<const uint32_t *>(sm + oq));
-          const float2 kv = bf2_to_f2(*reinterpret_cast<const uint32_t *>(sm + ok_));
-          wa = f2_to_bf2(bb.x * kv.x * f.x, bb.y * kv.y * f.y);
-          wq = f2_to_bf2(qv.x * f.x, qv.y * f.y);
-          wk = f2_to_bf2(kv.x * fi.x, kv.y * fi.y);
+#pragma unroll
+        for (int i = 3; i >= 0; --i) {  // run = prod_{r < s <= 31} alpha_s
+          float f[8], fi[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            fi[t] = run[t];
+            f[t] = fast_rcp(run[t]);
+            run[t] *= al[i][t];
+          }
+          row_factors(sm, 4 * G + i, cb, x8, Cc, f, fi);
         }
-        *reinterpret_cast<uint32_t *>(sm + oa) = wa;
-        *reinterpret_cast<uint32_t *>(sm + oq) = wq;
-        *reinterpret_cast<uint32_t *>(sm + ok_) = wk;
+      } else {
+        for (int g = 8; g < G; ++g) {
+          const float4 p0 = *reinterpret_cast<const float4 *>(&scan[g * 128 + 8 * ch8]);
+          const float4 p1 = *reinterpret_cast<const float4 *>(&scan[g * 128 + 8 * ch8 + 4]);
+          run[0] *= p0.x; run[1] *= p0.y; run[2] *= p0.z; run[3] *= p0.w;
+          run[4] *= p1.x; run[5] *= p1.y; run[6] *= p1.z; run[7] *= p1.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {  // run = prod_{32 <= s <= r} alpha_s
+          float f[8], fi[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            run[t] *= al[i][t];
+            f[t] = run[t];
+            fi[t] = fast_rcp(run[t]);
+          }
+          row_factors(sm, 4 * G + i, cb, x8, Cc, f, fi);
+        }
       }
     }
     {  // U = w (.) v for the 64 value columns of this CTA
@@ -292,18 +337,20 @@ __global__ void __launch_bounds__(NT, 2)
     tc_fence_after();
 
     // ---------------------------------------------------------------- C: T = (I + L)^-1
-    {
+    {  // L (strict lower) -> fp32 scratch; P (inclusive lower) -> both halves of [P ; P]
       float v[32];
       tmem_ld32(tl + 0 + 32 * half, v);
       tmem_wait_ld();
       const int row = 32 * quad + lane;
       if (row < 64) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int i = 32 * half + j;
-          f64x64(Ls, row, i) = (i < row) ? v[j] : 0.f;
+        for (int x = 0; x < 8; ++x) {
+          const int i = 32 * half + 4 * x;
+          *reinterpret_cast<float4 *>(&Ls[row * LDF + i]) =
+              make_float4(i < row ? v[4 * x] : 0.f, i + 1 < row ? v[4 * x + 1] : 0.f, i + 2 < row ? v[4 * x + 2] : 0.f,
+                          i + 3 < row ? v[4 * x + 3] : 0.f);
         }
-      } else {  // P (inclusive lower) -> rows 64..127 of the TP tile, bf16
+      } else {
         const int r = row - 64;
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
@@ -311,101 +358,113 @@ __global__ void __launch_bounds__(NT, 2)
           float e[8];
 #pragma unroll
           for (int t = 0; t < 8; ++t) e[t] = (col + t <= r) ? v[8 * x + t] : 0.f;
-          st_s128(sm + OFF_TP + sw128(row, col),
-                  make_uint4(f2_to_bf2(e[0], e[1]), f2_to_bf2(e[2], e[3]), f2_to_bf2(e[4], e[5]), f2_to_bf2(e[6], e[7])));
+          const uint4 u = pack8(e);
+          st_s128(sm + OFF_PP + sw128(r, col), u);
+          st_s128(sm + OFF_PP + sw128(row, col), u);
         }
       }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp < 2) {  // the four 16x16 diagonal blocks: lane = column j of block R
+    if (warp < 2) {  // the four 16x16 diagonal blocks, right-looking; lane = column j of block R
       const int R = 2 * warp + (lane >> 4), j = lane & 15;
+      const float *Lb = Ls + 16 * R * LDF + 16 * R;
       float x[16];
 #pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        float acc = (r == j) ? 1.f : 0.f;
+      for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
-        for (int i = 0; i < r; ++i) acc = fmaf(-f64x64(Ls, 16 * R + r, 16 * R + i), x[i], acc);
-        x[r] = acc;
-      }
+      for (int i = 0; i < 15; ++i)
 #pragma unroll
-      for (int r = 0; r < 16; ++r) f64x64(Ts, 16 * R + r, 16 * R + j) = x[r];
+        for (int r = i + 1; r < 16; ++r) x[r] = fmaf(-Lb[r * LDF + i], x[i], x[r]);
+      float *Tb = Ts + 16 * R * LDF + 16 * R;
+#pragma unroll
+      for (int r = 0; r < 16; ++r) Tb[r * LDF + j] = x[r];
     }
     __syncthreads();
-    for (int R = 1; R < 4; ++R) {  // block row R: T_RI = -T_RR sum_{J=I}^{R-1} L_RJ T_JI
-      for (int e = tid; e < 256 * R; e += NT) {
-        const int I = e >> 8, rr = (e >> 4) & 15, ci = e & 15;
-        float acc = 0.f;
-        for (int J = I; J < R; ++J)
+    {  // T_{R,R-1} for R = 1, 3: Y = L_{R,R-1} T_{R-1,R-1} (parked in the upper block (R-1, R) of L)
+      float acc[2];
 #pragma unroll
-          for (int k = 0; k < 16; ++k)
-            acc = fmaf(f64x64(Ls, 16 * R + rr, 16 * J + k), f64x64(Ts, 16 * J + k, 16 * I + ci), acc);
-        f64x64(Ls, 16 * I + rr, 16 * R + ci) = acc;  // park Y_RI in the unused upper block (I, R)
+      for (int u = 0; u < 2; ++u) {
+        const int R = 1 + 2 * u, r = tid >> 4, c = tid & 15;
+        const float *Lr = Ls + (16 * R + r) * LDF + 16 * (R - 1);
+        const float *Tc = Ts + 16 * (R - 1) * LDF + 16 * (R - 1) + c;
+        float s = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) s = fmaf(Lr[k], Tc[k * LDF], s);
+        acc[u] = s;
       }
-      __syncthreads();
-      for (int e = tid; e < 256 * R; e += NT) {
-        const int I = e >> 8, rr = (e >> 4) & 15, ci = e & 15;
-        float acc = 0.f;
-        for (int k = 0; k <= rr; ++k)
-          acc = fmaf(f64x64(Ts, 16 * R + rr, 16 * R + k), f64x64(Ls, 16 * I + k, 16 * R + ci), acc);
-        f64x64(Ts, 16 * R + rr, 16 * I + ci) = -acc;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int R = 1 + 2 * u, r = tid >> 4, c = tid & 15;
+        Ls[(16 * (R - 1) + r) * LDF + 16 * R + c] = acc[u];
       }
-      __syncthreads();
     }
-    {  // T -> rows 0..63 of the TP tile, bf16, zero above the diagonal
+    __syncthreads();
+    {  // T_{R,R-1} = -T_RR Y
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int R = 1 + 2 * u, r = tid >> 4, c = tid & 15;
+        const float *Tr = Ts + (16 * R + r) * LDF + 16 * R;
+        const float *Yc = Ls + 16 * (R - 1) * LDF + 16 * R + c;
+        float s = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) s = fmaf(Tr[k], Yc[k * LDF], s);
+        Ts[(16 * R + r) * LDF + 16 * (R - 1) + c] = -s;
+      }
+    }
+    __syncthreads();
+    {  // lower-left 32x32 block: Y = L[32:64, 0:32] T[0:32, 0:32] (parked in L[0:32, 32:64])
+      const int r = tid >> 3, c4 = 4 * (tid & 7);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      const float *Lr = Ls + (32 + r) * LDF;
+#pragma unroll 8
+      for (int k = 0; k < 32; ++k) {
+        const float l = Lr[k];
+        const float4 t = *reinterpret_cast<const float4 *>(&Ts[k * LDF + c4]);
+        acc.x = fmaf(l, t.x, acc.x); acc.y = fmaf(l, t.y, acc.y);
+        acc.z = fmaf(l, t.z, acc.z); acc.w = fmaf(l, t.w, acc.w);
+      }
+      *reinterpret_cast<float4 *>(&Ls[r * LDF + 32 + c4]) = acc;  // disjoint from what this stage reads
+    }
+    __syncthreads();
+    {  // T[32:64, 0:32] = -T[32:64, 32:64] Y
+      const int r = tid >> 3, c4 = 4 * (tid & 7);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      const float *Tr = Ts + (32 + r) * LDF + 32;
+#pragma unroll 8
+      for (int k = 0; k < 32; ++k) {
+        const float t = Tr[k];
+        const float4 y = *reinterpret_cast<const float4 *>(&Ls[k * LDF + 32 + c4]);
+        acc.x = fmaf(t, y.x, acc.x); acc.y = fmaf(t, y.y, acc.y);
+        acc.z = fmaf(t, y.z, acc.z); acc.w = fmaf(t, y.w, acc.w);
+      }
+      *reinterpret_cast<float4 *>(&Ts[(32 + r) * LDF + c4]) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+    }
+    __syncthreads();
+    {  // T -> rows 0..63 of [T ; 0], bf16
       const int r = tid >> 2;
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
         const int col = 16 * (tid & 3) + 8 * x;
-        float e[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) e[t] = (col + t <= r) ? f64x64(Ts, r, col + t) : 0.f;
-        st_s128(sm + OFF_TP + sw128(r, col),
-                make_uint4(f2_to_bf2(e[0], e[1]), f2_to_bf2(e[2], e[3]), f2_to_bf2(e[4], e[5]), f2_to_bf2(e[6], e[7])));
+        const float4 t0 = *reinterpret_cast<const float4 *>(&Ts[r * LDF + col]);
+        const float4 t1 = *reinterpret_cast<const float4 *>(&Ts[r * LDF + col + 4]);
+        const float e[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+        st_s128(sm + OFF_TZ + sw128(r, col), pack8(e));
       }
     }
     fence_proxy_async();
     __syncthreads();
 
-    // ---------------------------------------------------------------- M2: rows 64..127 <- P T
+    // ---------------------------------------------------------------- M3, M4: [T; 0] [A_m | U]
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        mma_bf16(tmem + 0, sdesc_sw128(sb + OFF_TP + 32 * k, 16, 1024), sdesc_sw128(sb + OFF_TP + 2048 * k, 16384, 1024),
-                 ID_KM64, k > 0 ? 1u : 0u);
-      mma_commit(bar_mma);
-    }
-    if (!(ok = cta_wait(bar_mma, ph_mma))) break;
-    ph_mma ^= 1;
-    tc_fence_after();
-    if (quad >= 2) {
-      float v[32];
-      tmem_ld32(tl + 0 + 32 * half, v);
-      tmem_wait_ld();
-      const int row = 32 * quad + lane;
-#pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        const int col = 32 * half + 8 * x;
-        st_s128(sm + OFF_TP + sw128(row, col),
-                make_uint4(f2_to_bf2(v[8 * x], v[8 * x + 1]), f2_to_bf2(v[8 * x + 2], v[8 * x + 3]),
-                           f2_to_bf2(v[8 * x + 4], v[8 * x + 5]), f2_to_bf2(v[8 * x + 6], v[8 * x + 7])));
-      }
-    }
-    tc_fence_before();
-    fence_proxy_async();
-    __syncthreads();
-
-    // ---------------------------------------------------------------- M3, M4: [T; P T] [A_m | U]
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        mma_bf16(tmem + 64, sdesc_sw128(sb + OFF_TP + 32 * k, 16, 1024),
+        mma_bf16(tmem + 64, sdesc_sw128(sb + OFF_TZ + 32 * k, 16, 1024),
                  sdesc_sw128(sb + OFF_XA + 2048 * k, XA_BLK, 1024), ID_KM128, k > 0 ? 1u : 0u);
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        mma_bf16(tmem + 192, sdesc_sw128(sb + OFF_TP + 32 * k, 16, 1024), sdesc_sw128(sb + OFF_U + 2048 * k, 8192, 1024),
+        mma_bf16(tmem + 192, sdesc_sw128(sb + OFF_TZ + 32 * k, 16, 1024), sdesc_sw128(sb + OFF_U + 2048 * k, 8192, 1024),
                  ID_KM64, k > 0 ? 1u : 0u);
       mma_commit(bar_mma);
     }
@@ -413,96 +472,81 @@ __global__ void __launch_bounds__(NT, 2)
     ph_mma ^= 1;
     tc_fence_after();
 
-    // ---------------------------------------------------------------- E: [-T A_m; Q_m - P T A_m] in place; e^m S
+    // ---------------------------------------------------------------- E: -T A_m in place of A_m; e^m S
     {
-      const int row = 32 * quad + lane;
+      if (quad < 2) {
+        const int row = 32 * quad + lane;
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        float v[32];
-        tmem_ld32(tl + 64 + 64 * half + 32 * part, v);
-        tmem_wait_ld();
-        uint8_t *base = sm + OFF_XA + half * XA_BLK;
+        for (int part = 0; part < 2; ++part) {
+          float v[32];
+          tmem_ld32(tl + 64 + 64 * half + 32 * part, v);
+          tmem_wait_ld();
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const int col = 32 * part + 8 * x;
-          uint8_t *p = base + sw128(row, col);
-          uint4 u;
-          if (row < 64) {
-            u = make_uint4(f2_to_bf2(-v[8 * x], -v[8 * x + 1]), f2_to_bf2(-v[8 * x + 2], -v[8 * x + 3]),
-                           f2_to_bf2(-v[8 * x + 4], -v[8 * x + 5]), f2_to_bf2(-v[8 * x + 6], -v[8 * x + 7]));
-          } else {
-            const uint4 qm = ld_s128(p);
-            const float2 q0 = bf2_to_f2(qm.x), q1 = bf2_to_f2(qm.y), q2 = bf2_to_f2(qm.z), q3 = bf2_to_f2(qm.w);
-            u = make_uint4(f2_to_bf2(q0.x - v[8 * x], q0.y - v[8 * x + 1]), f2_to_bf2(q1.x - v[8 * x + 2], q1.y - v[8 * x + 3]),
-                           f2_to_bf2(q2.x - v[8 * x + 4], q2.y - v[8 * x + 5]),
-                           f2_to_bf2(q3.x - v[8 * x + 6], q3.y - v[8 * x + 7]));
+          for (int x = 0; x < 4; ++x) {
+            float e[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) e[t] = -v[8 * x + t];
+            st_s128(sm + OFF_XA + half * XA_BLK + sw128(row, 32 * part + 8 * x), pack8(e));
           }
-          st_s128(p, u);
         }
       }
       const float em = s_em[c_me];
 #pragma unroll
       for (int x = 0; x < 4; ++x) {
-        const int col = 32 * half + 8 * x;
-        st_s128(sm + OFF_TP + sw128(c_me, col),
-                make_uint4(f2_to_bf2(em * S[8 * x], em * S[8 * x + 1]), f2_to_bf2(em * S[8 * x + 2], em * S[8 * x + 3]),
-                           f2_to_bf2(em * S[8 * x + 4], em * S[8 * x + 5]), f2_to_bf2(em * S[8 * x + 6], em * S[8 * x + 7])));
+        float e[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) e[t] = em * S[8 * x + t];
+        st_s128(sm + OFF_SM + sw128(c_me, 32 * half + 8 * x), pack8(e));
       }
     }
     tc_fence_before();
     fence_proxy_async();
     __syncthreads();
 
-    // ---------------------------------------------------------------- M5: D_a += [-T A_m; Q_m - P T A_m] (e^m S)
+    // ---------------------------------------------------------------- M5: D_a += [-T A_m; Q_m] (e^m S)
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
       for (int k = 0; k < DK / 16; ++k)
         mma_bf16(tmem + 192, sdesc_sw128(sb + OFF_XA + (k >> 2) * XA_BLK + (k & 3) * 32, 16, 1024),
-                 sdesc_sw128(sb + OFF_TP + 2048 * k, 16384, 1024), ID_KM64, 1u);
+                 sdesc_sw128(sb + OFF_SM + 2048 * k, 16384, 1024), ID_KM64, 1u);
       mma_commit(bar_mma);
     }
     if (!(ok = cta_wait(bar_mma, ph_mma))) break;
     ph_mma ^= 1;
     tc_fence_after();
 
-    // ---------------------------------------------------------------- F: Delta -> smem, O -> global
-    {
+    // ---------------------------------------------------------------- F: Delta -> smem
+    if (quad < 2) {
       float v[32];
       tmem_ld32(tl + 192 + 32 * half, v);
       tmem_wait_ld();
       const int row = 32 * quad + lane;
-      if (row < 64) {
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const int col = 32 * half + 8 * x;
-          st_s128(sm + OFF_DL + sw128(row, col),
-                  make_uint4(f2_to_bf2(v[8 * x], v[8 * x + 1]), f2_to_bf2(v[8 * x + 2], v[8 * x + 3]),
-                             f2_to_bf2(v[8 * x + 4], v[8 * x + 5]), f2_to_bf2(v[8 * x + 6], v[8 * x + 7])));
-        }
-      } else if (row - 64 < Cc) {
-        __nv_bfloat16 *dst = o + ((size_t)(tok0 + row - 64) * a.H + h) * (size_t)a.dv + j0 + 32 * half;
-        store_row32(dst, v);
-      }
+      for (int x = 0; x < 4; ++x) st_s128(sm + OFF_DL + sw128(row, 32 * half + 8 * x), pack8(&v[8 * x]));
     }
     tc_fence_before();
     fence_proxy_async();
     __syncthreads();
 
-    // ---------------------------------------------------------------- M6: K_m^T Delta
+    // ---------------------------------------------------------------- M6, M7: K_m^T Delta; D_a += [P; P] Delta
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
       for (int k = 0; k < 4; ++k)
         mma_bf16(tmem + 0, sdesc_sw128(sb + OFF_KT + 2048 * k, KT_BLK, 1024), sdesc_sw128(sb + OFF_DL + 2048 * k, 8192, 1024),
                  ID_MNMN, k > 0 ? 1u : 0u);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        mma_bf16(tmem + 192, sdesc_sw128(sb + OFF_PP + 32 * k, 16, 1024), sdesc_sw128(sb + OFF_DL + 2048 * k, 8192, 1024),
+                 ID_KM64, 1u);
       mma_commit(bar_mma);
     }
     if (!(ok = cta_wait(bar_mma, ph_mma))) break;
     ph_mma ^= 1;
     tc_fence_after();
 
-    // ---------------------------------------------------------------- G: state update
+    // ---------------------------------------------------------------- G: state update, O -> global
     {
       float v[32];
       tmem_ld32(tl + 0 + 32 * half, v);
@@ -510,6 +554,12 @@ __global__ void __launch_bounds__(NT, 2)
       const float g1 = s_egc[c_me], g2 = s_egcm[c_me];
 #pragma unroll
       for (int j = 0; j < 32; ++j) S[j] = fmaf(g2, v[j], g1 * S[j]);
+      if (quad >= 2) {  // warp-uniform: tcgen05.ld is a warp-collective instruction
+        const int r = 32 * quad + lane - 64;
+        tmem_ld32(tl + 192 + 32 * half, v);
+        tmem_wait_ld();
+        if (r < Cc) store_row32_bf16(o + ((size_t)(tok0 + r) * a.H + h) * (size_t)a.dv + j0 + 32 * half, v);
+      }
     }
     tc_fence_before();
     __syncthreads();
