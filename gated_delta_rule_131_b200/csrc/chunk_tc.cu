@@ -57,29 +57,33 @@ namespace {
 
 using namespace ptx;
 
-constexpr int C = 64, DK = 128, NV = 64, NT = 256;
+constexpr int C = 64, DK = 128, NV = 64;
+constexpr int NT = 384;           // warps 0-3: state side; warps 4-11: key side
+constexpr int NSTATE = 128, NKEY = 256;
+constexpr int BAR_STATE = 1, BAR_KEY = 2;  // named barriers of the two warp groups
 
 // shared-memory map (bytes from a 1024-aligned base); every MMA operand tile is 1024-aligned
-constexpr uint32_t XA_BLK = 16384;                 // [A_m | -T A_m ; Q_m] 128 rows x 64 ch, two channel blocks
-constexpr uint32_t KT_BLK = 8192;                  // K_m 64 rows x 64 ch, two channel blocks
-constexpr uint32_t OFF_XA = 0;
-constexpr uint32_t OFF_KT = OFF_XA + 2 * XA_BLK;   // 32768
-constexpr uint32_t OFF_AL = OFF_KT + 2 * KT_BLK;   // 49152: alpha tiles (two blocks)
-constexpr uint32_t OFF_U = OFF_AL + 16384;         // 65536: v tile -> U = w (.) v
-constexpr uint32_t OFF_W = OFF_U + 8192;           // 73728: w tile
-constexpr uint32_t OFF_DL = OFF_W + 8192;          // 81920: Delta, bf16 64 x 64
-constexpr uint32_t OFF_TZ = OFF_DL + 8192;         // 90112: [T ; 0] bf16 128 x 64
-constexpr uint32_t OFF_PP = OFF_TZ + 16384;        // 106496: [P ; P] bf16 128 x 64
-constexpr uint32_t OFF_SM = OFF_PP + 16384;        // 122880: e^m S, bf16 128 x 64
+constexpr uint32_t XA_BLK = 16384;                 // [A_m | -T A_m ; Q_m] 128 rows x 64 ch (one channel block)
+constexpr uint32_t XA_BUF = 2 * XA_BLK;            // two channel blocks per chunk buffer
+constexpr uint32_t KT_BLK = 8192;                  // K_m 64 rows x 64 ch
+constexpr uint32_t KT_BUF = 2 * KT_BLK;
+constexpr uint32_t OFF_XA = 0;                     // 2 chunk buffers
+constexpr uint32_t OFF_KT = OFF_XA + 2 * XA_BUF;   // 65536: 2 chunk buffers
+constexpr uint32_t OFF_U = OFF_KT + 2 * KT_BUF;    // 98304: 2 chunk buffers of v -> U = w (.) v
+constexpr uint32_t OFF_AL = OFF_U + 2 * 8192;      // 114688: alpha tiles (two channel blocks)
+constexpr uint32_t OFF_W = OFF_AL + 16384;         // 131072: w tile
+constexpr uint32_t OFF_TZP = OFF_W + 8192;         // 139264: [T ; 0 ; P0 ; P1], 64 rows each
+constexpr uint32_t OFF_SM = OFF_TZP + 32768;       // 172032: e^m S (128 x 64); its first 8 KB later holds Delta
 constexpr int LDF = 68;                            // row stride of the fp32 64 x 64 scratch
-constexpr uint32_t OFF_LS = OFF_SM + 16384;        // 139264: L (fp32), upper blocks reused as scratch
-constexpr uint32_t OFF_TS = OFF_LS + 64 * LDF * 4; // 156672: T (fp32)
-constexpr uint32_t OFF_SC = OFF_TS + 64 * LDF * 4; // 174080: decay products and per-channel scalars
-constexpr uint32_t OFF_BAR = OFF_SC + 16 * 128 * 4 + 3 * 128 * 4;
-constexpr uint32_t SMEM_USED = OFF_BAR + 64;
+constexpr uint32_t OFF_LS = OFF_SM + 16384;        // 188416: L (fp32); first 8 KB = decay-product scan
+constexpr uint32_t OFF_TS = OFF_LS + 64 * LDF * 4; // 205824: T (fp32)
+constexpr uint32_t OFF_SC = OFF_TS + 64 * LDF * 4; // 223232: per-channel scalars, 2 chunk buffers
+constexpr uint32_t OFF_BAR = OFF_SC + 2 * 3 * 128 * 4;  // 226304
+constexpr uint32_t SMEM_USED = OFF_BAR + 128;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for aligning the base
 constexpr uint32_t TMA_BYTES = 10 * 8192;          // q, k, b, alpha (2 boxes each), v, w
-constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_LP = 0, TM_DX = 64, TM_DA = 192, TM_DB = 320;  // D_a: two 64-column buffers
 constexpr uint64_t WAIT_NS = 2000000000ull;        // bounded waits: 2 s
 
 constexpr uint32_t ID_LP = idesc_bf16(128, 64, false, false);    // [A_m;Q_m] K_m^T
@@ -87,37 +91,60 @@ constexpr uint32_t ID_KM64 = idesc_bf16(128, 64, false, true);   // K-major A, M
 constexpr uint32_t ID_KM128 = idesc_bf16(128, 128, false, true); // same, N = 128
 constexpr uint32_t ID_MNMN = idesc_bf16(128, 64, true, true);    // K_m^T Delta
 
+// mbarriers (8 bytes each) at OFF_BAR
+enum { B_FULL0 = 0, B_FULL1, B_KMMA, B_SMMA, B_READY0, B_READY1, B_STDONE0, B_STDONE1, B_DAFREE0, B_DAFREE1, B_COUNT };
+
 __device__ __forceinline__ uint4 ld_s128(const uint8_t *p) { return *reinterpret_cast<const uint4 *>(p); }
 __device__ __forceinline__ void st_s128(uint8_t *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
 __device__ __forceinline__ uint4 pack8(const float *e) {
   return make_uint4(f2_to_bf2(e[0], e[1]), f2_to_bf2(e[2], e[3]), f2_to_bf2(e[4], e[5]), f2_to_bf2(e[6], e[7]));
 }
-__device__ __forceinline__ float fast_rcp(float x) { return __fdividef(1.f, x); }
-
-// Every thread waits; the CTA then agrees on the outcome (so control flow stays uniform).
-__device__ __forceinline__ bool cta_wait(uint32_t bar, uint32_t parity) {
-  const bool ok = mbar_wait_bounded(bar, parity, WAIT_NS);
-  return !__syncthreads_or(!ok);
-}
-
-__device__ __forceinline__ void store_row32_bf16(__nv_bfloat16 *dst, const float (&v)[32]) {
-#pragma unroll
-  for (int x = 0; x < 4; ++x) reinterpret_cast<uint4 *>(dst)[x] = pack8(&v[8 * x]);
-}
-
 __device__ __forceinline__ void unpack8(uint4 u, float *e) {
   float2 t = bf2_to_f2(u.x); e[0] = t.x; e[1] = t.y;
   t = bf2_to_f2(u.y); e[2] = t.x; e[3] = t.y;
   t = bf2_to_f2(u.z); e[4] = t.x; e[5] = t.y;
   t = bf2_to_f2(u.w); e[6] = t.x; e[7] = t.y;
 }
+__device__ __forceinline__ float fast_rcp(float x) { return __fdividef(1.f, x); }
+
+__device__ __forceinline__ void group_sync(int id, int count) {
+  asm volatile("barrier.cta.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Barrier of one warp group that also ORs a predicate over its threads.
+__device__ __forceinline__ bool group_or(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// Every thread of a warp group waits (bounded); the group agrees on the outcome; `fail` lets the
+// caller fold in an earlier failure of one thread.
+__device__ __forceinline__ bool group_wait(int id, int count, uint32_t bar, uint32_t parity, bool fail = false) {
+  const bool ok = mbar_wait_bounded(bar, parity, WAIT_NS);
+  return !group_or(id, count, fail || !ok);
+}
+
+__device__ __forceinline__ void store_row32_bf16(__nv_bfloat16 *dst, const float *v) {
+#pragma unroll
+  for (int x = 0; x < 4; ++x) reinterpret_cast<uint4 *>(dst)[x] = pack8(&v[8 * x]);
+}
 
 // Decay-absorbed operands of one token row for 8 key channels, in place:
 // A_m = b k f, Q_m = q f, K_m = k fi with f = e^{g_r - m}, fi = 1/f; rows >= Cc are zeroed.
-__device__ __forceinline__ void row_factors(uint8_t *sm, int r, int cb, int x8, int Cc, const float *f, const float *fi) {
-  uint8_t *pa = sm + OFF_XA + cb * XA_BLK + sw128(r, 8 * x8);
+__device__ __forceinline__ void row_factors(uint8_t *xa, uint8_t *kt, int r, int cb, int x8, int Cc, const float *f,
+                                            const float *fi) {
+  uint8_t *pa = xa + cb * XA_BLK + sw128(r, 8 * x8);
   uint8_t *pq = pa + 8192;
-  uint8_t *pk = sm + OFF_KT + cb * KT_BLK + sw128(r, 8 * x8);
+  uint8_t *pk = kt + cb * KT_BLK + sw128(r, 8 * x8);
   uint4 wa = make_uint4(0u, 0u, 0u, 0u), wq = wa, wk = wa;
   if (r < Cc) {
     float bb[8], qv[8], kv[8], ea[8], eq[8], ek[8];
@@ -139,98 +166,65 @@ __device__ __forceinline__ void row_factors(uint8_t *sm, int r, int cb, int x8, 
   st_s128(pk, wk);
 }
 
-__global__ void __launch_bounds__(NT, 1)
-    chunk_fwd_tc_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap tm_q,
-                        const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_b,
-                        const __grid_constant__ CUtensorMap tm_al, const __grid_constant__ CUtensorMap tm_v,
-                        const __grid_constant__ CUtensorMap tm_w) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t sb = smem_u32(sm);
-  float *pp = reinterpret_cast<float *>(sm + OFF_SC);  // [16][128] decay product of each 4-token group
-  float *s_em = pp + 16 * 128;                         // e^m       (decay from chunk start to token 31)
-  float *s_egcm = s_em + 128;                          // e^{g_C-m} (decay over tokens 32..end)
-  float *s_egc = s_egcm + 128;                         // e^{g_C}   (decay over the whole chunk)
-  const uint32_t bar_ld = sb + OFF_BAR, bar_mma = sb + OFF_BAR + 8;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 16);
+struct Ctx {
+  uint8_t *sm;
+  uint32_t sb, tmem;
+  int H, dv, h, j0, nchunks, len;
+  int64_t bos;
+};
+
+__device__ __forceinline__ uint32_t bar_addr(const Ctx &x, int i) { return x.sb + OFF_BAR + 8 * i; }
+
+// Issue the TMA loads of chunk `c` into chunk buffer c & 1 (one thread).
+__device__ __forceinline__ void issue_chunk_loads(const Ctx &x, int c, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
+                                                  const CUtensorMap *tm_b, const CUtensorMap *tm_al,
+                                                  const CUtensorMap *tm_v, const CUtensorMap *tm_w) {
+  const int b = c & 1;
+  const int tok0 = (int)(x.bos + (int64_t)c * C);
+  const uint32_t full = bar_addr(x, B_FULL0 + b);
+  fence_proxy_async();
+  mbar_expect_tx(full, TMA_BYTES);
+#pragma unroll
+  for (int blk = 0; blk < 2; ++blk) {
+    tma_load_3d(x.sb + OFF_XA + b * XA_BUF + blk * XA_BLK, tm_b, 64 * blk, x.h, tok0, full);         // b -> rows 0..63
+    tma_load_3d(x.sb + OFF_XA + b * XA_BUF + blk * XA_BLK + 8192, tm_q, 64 * blk, x.h, tok0, full);  // q -> rows 64..127
+    tma_load_3d(x.sb + OFF_KT + b * KT_BUF + blk * KT_BLK, tm_k, 64 * blk, x.h, tok0, full);
+    tma_load_3d(x.sb + OFF_AL + blk * 8192, tm_al, 64 * blk, x.h, tok0, full);
+  }
+  tma_load_3d(x.sb + OFF_U + b * 8192, tm_v, x.j0, x.h, tok0, full);
+  tma_load_3d(x.sb + OFF_W, tm_w, x.j0, x.h, tok0, full);
+}
+
+// ==================================================================== key side (warps 4-11)
+// For each chunk: decay factors, L|P, T, [T; 0][A_m | U]; hands the chunk to the state side.
+__device__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_b,
+                         const CUtensorMap *tm_al, const CUtensorMap *tm_v, const CUtensorMap *tm_w) {
+  uint8_t *sm = x.sm;
+  const int kt = threadIdx.x - NSTATE, kwarp = kt >> 5, lane = kt & 31, quad = kwarp & 3, khalf = kwarp >> 2;
+  const uint32_t tl = x.tmem + ((uint32_t)(32 * quad) << 16);
   float *Ls = reinterpret_cast<float *>(sm + OFF_LS);
   float *Ts = reinterpret_cast<float *>(sm + OFF_TS);
+  float *scan = Ls;  // [16 groups][128 channels] during the factor phase
+  uint32_t kphase = 0;
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, quad = warp & 3, half = warp >> 2;
-  const int tiles = a.dv / NV;
-  const int tile = blockIdx.x % tiles;
-  const int h = (blockIdx.x / tiles) % a.H;
-  const int n = blockIdx.x / (tiles * a.H);
-  const int j0 = tile * NV;
-  int64_t bos;
-  int len;
-  seq_span(a, n, bos, len);
-  __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o);
+  if (kt == 0 && x.nchunks > 0) issue_chunk_loads(x, 0, tm_q, tm_k, tm_b, tm_al, tm_v, tm_w);
 
-  if (tid == 0) {
-    mbar_init(bar_ld, 1);
-    mbar_init(bar_mma, 1);
-    fence_mbar_init();
-    prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_b);
-    prefetch_tmap(&tm_al); prefetch_tmap(&tm_v); prefetch_tmap(&tm_w);
-  }
-  if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
-  }
-  // zero rows 64..127 of [T ; 0] once, and the never-written upper blocks of T
-  for (int e = tid; e < 8192 / 16; e += NT) st_s128(sm + OFF_TZ + 8192 + 16 * e, make_uint4(0u, 0u, 0u, 0u));
-  for (int e = tid; e < 64 * LDF; e += NT) Ts[e] = 0.f;
-  fence_proxy_async();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16);  // this warp's TMEM lane quadrant
+  for (int c = 0; c < x.nchunks; ++c) {
+    const int b = c & 1;
+    const int Cc = min(C, x.len - c * C);
+    uint8_t *xa = sm + OFF_XA + b * XA_BUF;
+    uint8_t *ktile = sm + OFF_KT + b * KT_BUF;
+    float *s_em = reinterpret_cast<float *>(sm + OFF_SC) + b * 384;
+    float *s_egcm = s_em + 128, *s_egc = s_em + 256;
 
-  // state slice: key channel c_me, value columns j0 + 32*half .. +31
-  const int c_me = 32 * quad + lane;
-  const size_t s_off = (((size_t)n * a.H + h) * DK + c_me) * (size_t)a.dv + j0 + 32 * half;
-  float S[32];
-  if (a.S0) {
-#pragma unroll
-    for (int x = 0; x < 8; ++x) {
-      const float4 t = reinterpret_cast<const float4 *>(a.S0 + s_off)[x];
-      S[4 * x] = t.x; S[4 * x + 1] = t.y; S[4 * x + 2] = t.z; S[4 * x + 3] = t.w;
-    }
-  } else {
-#pragma unroll
-    for (int x = 0; x < 32; ++x) S[x] = 0.f;
-  }
+    // ------------------------------------------------------------ data of chunk c has landed
+    if (!group_wait(BAR_KEY, NKEY, bar_addr(x, B_FULL0 + b), (c >> 1) & 1)) return false;
 
-  uint32_t ph_ld = 0, ph_mma = 0;
-  bool ok = true;
-  for (int c0 = 0; c0 < len; c0 += C) {
-    const int Cc = min(C, len - c0);
-    const int tok0 = (int)(bos + c0);
-
-    // ---------------------------------------------------------------- A: TMA loads of the chunk
-    if (tid == 0) {
-      fence_proxy_async();
-      mbar_expect_tx(bar_ld, TMA_BYTES);
-#pragma unroll
-      for (int blk = 0; blk < 2; ++blk) {
-        tma_load_3d(sb + OFF_XA + blk * XA_BLK, &tm_b, 64 * blk, h, tok0, bar_ld);         // b -> rows 0..63
-        tma_load_3d(sb + OFF_XA + blk * XA_BLK + 8192, &tm_q, 64 * blk, h, tok0, bar_ld);  // q -> rows 64..127
-        tma_load_3d(sb + OFF_KT + blk * KT_BLK, &tm_k, 64 * blk, h, tok0, bar_ld);
-        tma_load_3d(sb + OFF_AL + blk * 8192, &tm_al, 64 * blk, h, tok0, bar_ld);
-      }
-      tma_load_3d(sb + OFF_U, &tm_v, j0, h, tok0, bar_ld);
-      tma_load_3d(sb + OFF_W, &tm_w, j0, h, tok0, bar_ld);
-    }
-    if (!(ok = cta_wait(bar_ld, ph_ld))) break;
-    ph_ld ^= 1;
-
-    // ---------------------------------------------------------------- B: decay factors, operands
+    // ------------------------------------------------------------ decay factors, operands in place
     {
       // thread = 8 key channels (chunk x8 of channel block cb) x 4 tokens (group G = rows 4G..4G+3);
-      // warps 0-3 hold tokens 0..31 (walk back to token 31), warps 4-7 tokens 32..63 (walk forward)
-      const int ch8 = tid & 15, G = tid >> 4, cb = ch8 >> 3, x8 = ch8 & 7;
+      // warps 0-3 of the group hold tokens 0..31 (walk back to token 31), warps 4-7 tokens 32..63
+      const int ch8 = kt & 15, G = kt >> 4, cb = ch8 >> 3, x8 = ch8 & 7;
       float al[4][8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -245,28 +239,28 @@ __global__ void __launch_bounds__(NT, 1)
       float gp[8];
 #pragma unroll
       for (int t = 0; t < 8; ++t) gp[t] = al[0][t] * al[1][t] * al[2][t] * al[3][t];
-      float *scan = pp;  // [16 groups][128 channels]: product of alpha over each 4-token group
       *reinterpret_cast<float4 *>(&scan[G * 128 + 8 * ch8]) = make_float4(gp[0], gp[1], gp[2], gp[3]);
       *reinterpret_cast<float4 *>(&scan[G * 128 + 8 * ch8 + 4]) = make_float4(gp[4], gp[5], gp[6], gp[7]);
-      __syncthreads();
-      if (tid < 128) {
+      group_sync(BAR_KEY, NKEY);
+      if (kt < 128) {
         float em = 1.f, egcm = 1.f;
-        for (int g = 0; g < 8; ++g) em *= scan[g * 128 + tid];
-        for (int g = 8; g < 16; ++g) egcm *= scan[g * 128 + tid];
-        s_em[tid] = em;
-        s_egcm[tid] = egcm;
-        s_egc[tid] = em * egcm;
+        for (int g = 0; g < 8; ++g) em *= scan[g * 128 + kt];
+        for (int g = 8; g < 16; ++g) egcm *= scan[g * 128 + kt];
+        s_em[kt] = em;
+        s_egcm[kt] = egcm;
+        s_egc[kt] = em * egcm;
       }
-      float run[8];  // product of alpha strictly between this group and token 31 (inclusive of 31)
+      float run[8];
 #pragma unroll
       for (int t = 0; t < 8; ++t) run[t] = 1.f;
+      const int g0 = (G < 8) ? G + 1 : 8, g1 = (G < 8) ? 8 : G;
+      for (int g = g0; g < g1; ++g) {
+        const float4 p0 = *reinterpret_cast<const float4 *>(&scan[g * 128 + 8 * ch8]);
+        const float4 p1 = *reinterpret_cast<const float4 *>(&scan[g * 128 + 8 * ch8 + 4]);
+        run[0] *= p0.x; run[1] *= p0.y; run[2] *= p0.z; run[3] *= p0.w;
+        run[4] *= p1.x; run[5] *= p1.y; run[6] *= p1.z; run[7] *= p1.w;
+      }
       if (G < 8) {
-        for (int g = G + 1; g < 8; ++g) {
-          const float4 p0 = *reinterpret_cast<const float4 *>(&scan[g * 128 + 8 * ch8]);
-          const float4 p1 = *reinterpret_cast<const float4 *>(&scan[g * 128 + 8 * ch8 + 4]);
-          run[0] *= p0.x; run[1] *= p0.y; run[2] *= p0.z; run[3] *= p0.w;
-          run[4] *= p1.x; run[5] *= p1.y; run[6] *= p1.z; run[7] *= p1.w;
-        }
 #pragma unroll
         for (int i = 3; i >= 0; --i) {  // run = prod_{r < s <= 31} alpha_s
           float f[8], fi[8];
@@ -276,15 +270,9 @@ __global__ void __launch_bounds__(NT, 1)
             f[t] = fast_rcp(run[t]);
             run[t] *= al[i][t];
           }
-          row_factors(sm, 4 * G + i, cb, x8, Cc, f, fi);
+          row_factors(xa, ktile, 4 * G + i, cb, x8, Cc, f, fi);
         }
       } else {
-        for (int g = 8; g < G; ++g) {
-          const float4 p0 = *reinterpret_cast<const float4 *>(&scan[g * 128 + 8 * ch8]);
-          const float4 p1 = *reinterpret_cast<const float4 *>(&scan[g * 128 + 8 * ch8 + 4]);
-          run[0] *= p0.x; run[1] *= p0.y; run[2] *= p0.z; run[3] *= p0.w;
-          run[4] *= p1.x; run[5] *= p1.y; run[6] *= p1.z; run[7] *= p1.w;
-        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {  // run = prod_{32 <= s <= r} alpha_s
           float f[8], fi[8];
@@ -294,100 +282,101 @@ __global__ void __launch_bounds__(NT, 1)
             f[t] = run[t];
             fi[t] = fast_rcp(run[t]);
           }
-          row_factors(sm, 4 * G + i, cb, x8, Cc, f, fi);
+          row_factors(xa, ktile, 4 * G + i, cb, x8, Cc, f, fi);
         }
       }
     }
     {  // U = w (.) v for the 64 value columns of this CTA
-      const int r = tid >> 2;
+      const int r = kt >> 2;
+      uint8_t *ub = sm + OFF_U + b * 8192;
 #pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        const int col = 16 * (tid & 3) + 8 * x;
-        uint8_t *pu = sm + OFF_U + sw128(r, col);
-        const uint4 vv = ld_s128(pu), ww = ld_s128(sm + OFF_W + sw128(r, col));
-        uint4 uu = make_uint4(0u, 0u, 0u, 0u);
-        if (r < Cc) {
-          float2 a0 = bf2_to_f2(vv.x), b0 = bf2_to_f2(ww.x), a1 = bf2_to_f2(vv.y), b1 = bf2_to_f2(ww.y);
-          float2 a2 = bf2_to_f2(vv.z), b2 = bf2_to_f2(ww.z), a3 = bf2_to_f2(vv.w), b3 = bf2_to_f2(ww.w);
-          uu.x = f2_to_bf2(a0.x * b0.x, a0.y * b0.y);
-          uu.y = f2_to_bf2(a1.x * b1.x, a1.y * b1.y);
-          uu.z = f2_to_bf2(a2.x * b2.x, a2.y * b2.y);
-          uu.w = f2_to_bf2(a3.x * b3.x, a3.y * b3.y);
-        }
-        st_s128(pu, uu);
+      for (int y = 0; y < 2; ++y) {
+        const int col = 16 * (kt & 3) + 8 * y;
+        uint8_t *pu = ub + sw128(r, col);
+        float vv[8], ww[8], uu[8];
+        unpack8(ld_s128(pu), vv);
+        unpack8(ld_s128(sm + OFF_W + sw128(r, col)), ww);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) uu[t] = (r < Cc) ? vv[t] * ww[t] : 0.f;
+        st_s128(pu, pack8(uu));
       }
     }
     fence_proxy_async();
-    __syncthreads();
+    group_sync(BAR_KEY, NKEY);
 
-    // ---------------------------------------------------------------- M1: [L; P] = [A_m; Q_m] K_m^T
-    if (tid == 0) {
+    // ------------------------------------------------------------ prefetch chunk c+1; M1: [L; P] = [A_m; Q_m] K_m^T
+    bool fail = false;
+    if (kt == 0) {
+      if (c + 1 < x.nchunks) {
+        // buffer (c+1)&1 was last used by chunk c-1: wait until the state side's MMAs on it finished
+        if (c >= 1) fail = !mbar_wait_bounded(bar_addr(x, B_STDONE0 + ((c + 1) & 1)), ((c - 1) >> 1) & 1, WAIT_NS);
+        if (!fail) issue_chunk_loads(x, c + 1, tm_q, tm_k, tm_b, tm_al, tm_v, tm_w);
+      }
       tc_fence_after();
 #pragma unroll
       for (int k = 0; k < DK / 16; ++k) {
         const uint32_t koff = (uint32_t)(k & 3) * 32u;
-        const uint64_t ad = sdesc_sw128(sb + OFF_XA + (k >> 2) * XA_BLK + koff, 16, 1024);
-        const uint64_t bd = sdesc_sw128(sb + OFF_KT + (k >> 2) * KT_BLK + koff, 16, 1024);
-        mma_bf16(tmem + 0, ad, bd, ID_LP, k > 0 ? 1u : 0u);
+        const uint64_t ad = sdesc_sw128(x.sb + OFF_XA + b * XA_BUF + (k >> 2) * XA_BLK + koff, 16, 1024);
+        const uint64_t bd = sdesc_sw128(x.sb + OFF_KT + b * KT_BUF + (k >> 2) * KT_BLK + koff, 16, 1024);
+        mma_bf16(x.tmem + TM_LP, ad, bd, ID_LP, k > 0 ? 1u : 0u);
       }
-      mma_commit(bar_mma);
+      mma_commit(bar_addr(x, B_KMMA));
     }
-    if (!(ok = cta_wait(bar_mma, ph_mma))) break;
-    ph_mma ^= 1;
+    if (!group_wait(BAR_KEY, NKEY, bar_addr(x, B_KMMA), kphase, fail)) return false;
+    kphase ^= 1;
     tc_fence_after();
 
-    // ---------------------------------------------------------------- C: T = (I + L)^-1
-    {  // L (strict lower) -> fp32 scratch; P (inclusive lower) -> both halves of [P ; P]
+    // ------------------------------------------------------------ T = (I + L)^-1
+    uint8_t *pt = sm + OFF_TZP + 16384 + b * 8192;  // P of this chunk (64 x 64 bf16)
+    {  // L (strict lower) -> fp32 scratch; P (inclusive lower) -> its bf16 tile
       float v[32];
-      tmem_ld32(tl + 0 + 32 * half, v);
+      tmem_ld32(tl + TM_LP + 32 * khalf, v);
       tmem_wait_ld();
       const int row = 32 * quad + lane;
       if (row < 64) {
 #pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          const int i = 32 * half + 4 * x;
+        for (int y = 0; y < 8; ++y) {
+          const int i = 32 * khalf + 4 * y;
           *reinterpret_cast<float4 *>(&Ls[row * LDF + i]) =
-              make_float4(i < row ? v[4 * x] : 0.f, i + 1 < row ? v[4 * x + 1] : 0.f, i + 2 < row ? v[4 * x + 2] : 0.f,
-                          i + 3 < row ? v[4 * x + 3] : 0.f);
+              make_float4(i < row ? v[4 * y] : 0.f, i + 1 < row ? v[4 * y + 1] : 0.f, i + 2 < row ? v[4 * y + 2] : 0.f,
+                          i + 3 < row ? v[4 * y + 3] : 0.f);
         }
       } else {
         const int r = row - 64;
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const int col = 32 * half + 8 * x;
+        for (int y = 0; y < 4; ++y) {
+          const int col = 32 * khalf + 8 * y;
           float e[8];
 #pragma unroll
-          for (int t = 0; t < 8; ++t) e[t] = (col + t <= r) ? v[8 * x + t] : 0.f;
-          const uint4 u = pack8(e);
-          st_s128(sm + OFF_PP + sw128(r, col), u);
-          st_s128(sm + OFF_PP + sw128(row, col), u);
+          for (int t = 0; t < 8; ++t) e[t] = (col + t <= r) ? v[8 * y + t] : 0.f;
+          st_s128(pt + sw128(r, col), pack8(e));
         }
       }
     }
     tc_fence_before();
-    __syncthreads();
-    if (warp < 2) {  // the four 16x16 diagonal blocks, right-looking; lane = column j of block R
-      const int R = 2 * warp + (lane >> 4), j = lane & 15;
+    group_sync(BAR_KEY, NKEY);
+    if (kwarp < 2) {  // the four 16x16 diagonal blocks, right-looking; lane = column j of block R
+      const int R = 2 * kwarp + (lane >> 4), j = lane & 15;
       const float *Lb = Ls + 16 * R * LDF + 16 * R;
-      float x[16];
+      float xv[16];
 #pragma unroll
-      for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
+      for (int r = 0; r < 16; ++r) xv[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
       for (int i = 0; i < 15; ++i)
 #pragma unroll
-        for (int r = i + 1; r < 16; ++r) x[r] = fmaf(-Lb[r * LDF + i], x[i], x[r]);
+        for (int r = i + 1; r < 16; ++r) xv[r] = fmaf(-Lb[r * LDF + i], xv[i], xv[r]);
       float *Tb = Ts + 16 * R * LDF + 16 * R;
 #pragma unroll
-      for (int r = 0; r < 16; ++r) Tb[r * LDF + j] = x[r];
+      for (int r = 0; r < 16; ++r) Tb[r * LDF + j] = xv[r];
     }
-    __syncthreads();
+    group_sync(BAR_KEY, NKEY);
     {  // T_{R,R-1} for R = 1, 3: Y = L_{R,R-1} T_{R-1,R-1} (parked in the upper block (R-1, R) of L)
       float acc[2];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int R = 1 + 2 * u, r = tid >> 4, c = tid & 15;
+        const int R = 1 + 2 * u, r = kt >> 4, cl = kt & 15;
         const float *Lr = Ls + (16 * R + r) * LDF + 16 * (R - 1);
-        const float *Tc = Ts + 16 * (R - 1) * LDF + 16 * (R - 1) + c;
+        const float *Tc = Ts + 16 * (R - 1) * LDF + 16 * (R - 1) + cl;
         float s = 0.f;
 #pragma unroll
         for (int k = 0; k < 16; ++k) s = fmaf(Lr[k], Tc[k * LDF], s);
@@ -395,26 +384,26 @@ __global__ void __launch_bounds__(NT, 1)
       }
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int R = 1 + 2 * u, r = tid >> 4, c = tid & 15;
-        Ls[(16 * (R - 1) + r) * LDF + 16 * R + c] = acc[u];
+        const int R = 1 + 2 * u, r = kt >> 4, cl = kt & 15;
+        Ls[(16 * (R - 1) + r) * LDF + 16 * R + cl] = acc[u];
       }
     }
-    __syncthreads();
+    group_sync(BAR_KEY, NKEY);
     {  // T_{R,R-1} = -T_RR Y
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int R = 1 + 2 * u, r = tid >> 4, c = tid & 15;
+        const int R = 1 + 2 * u, r = kt >> 4, cl = kt & 15;
         const float *Tr = Ts + (16 * R + r) * LDF + 16 * R;
-        const float *Yc = Ls + 16 * (R - 1) * LDF + 16 * R + c;
+        const float *Yc = Ls + 16 * (R - 1) * LDF + 16 * R + cl;
         float s = 0.f;
 #pragma unroll
         for (int k = 0; k < 16; ++k) s = fmaf(Tr[k], Yc[k * LDF], s);
-        Ts[(16 * R + r) * LDF + 16 * (R - 1) + c] = -s;
+        Ts[(16 * R + r) * LDF + 16 * (R - 1) + cl] = -s;
       }
     }
-    __syncthreads();
+    group_sync(BAR_KEY, NKEY);
     {  // lower-left 32x32 block: Y = L[32:64, 0:32] T[0:32, 0:32] (parked in L[0:32, 32:64])
-      const int r = tid >> 3, c4 = 4 * (tid & 7);
+      const int r = kt >> 3, c4 = 4 * (kt & 7);
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       const float *Lr = Ls + (32 + r) * LDF;
 #pragma unroll 8
@@ -426,9 +415,9 @@ __global__ void __launch_bounds__(NT, 1)
       }
       *reinterpret_cast<float4 *>(&Ls[r * LDF + 32 + c4]) = acc;  // disjoint from what this stage reads
     }
-    __syncthreads();
+    group_sync(BAR_KEY, NKEY);
     {  // T[32:64, 0:32] = -T[32:64, 32:64] Y
-      const int r = tid >> 3, c4 = 4 * (tid & 7);
+      const int r = kt >> 3, c4 = 4 * (kt & 7);
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       const float *Tr = Ts + (32 + r) * LDF + 32;
 #pragma unroll 8
@@ -440,142 +429,250 @@ __global__ void __launch_bounds__(NT, 1)
       }
       *reinterpret_cast<float4 *>(&Ts[(32 + r) * LDF + c4]) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
     }
-    __syncthreads();
+    group_sync(BAR_KEY, NKEY);
     {  // T -> rows 0..63 of [T ; 0], bf16
-      const int r = tid >> 2;
+      const int r = kt >> 2;
 #pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        const int col = 16 * (tid & 3) + 8 * x;
+      for (int y = 0; y < 2; ++y) {
+        const int col = 16 * (kt & 3) + 8 * y;
         const float4 t0 = *reinterpret_cast<const float4 *>(&Ts[r * LDF + col]);
         const float4 t1 = *reinterpret_cast<const float4 *>(&Ts[r * LDF + col + 4]);
         const float e[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-        st_s128(sm + OFF_TZ + sw128(r, col), pack8(e));
+        st_s128(sm + OFF_TZP + sw128(r, col), pack8(e));
       }
     }
     fence_proxy_async();
-    __syncthreads();
+    group_sync(BAR_KEY, NKEY);
 
-    // ---------------------------------------------------------------- M3, M4: [T; 0] [A_m | U]
-    if (tid == 0) {
+    // ------------------------------------------------------------ M3, M4: [T; 0] [A_m | U]
+    fail = false;
+    if (kt == 0) {
+      // D_a buffer b was last read by the state side for chunk c-2
+      if (c >= 2) fail = !mbar_wait_bounded(bar_addr(x, B_DAFREE0 + b), ((c - 2) >> 1) & 1, WAIT_NS);
       tc_fence_after();
+      if (!fail) {
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        mma_bf16(tmem + 64, sdesc_sw128(sb + OFF_TZ + 32 * k, 16, 1024),
-                 sdesc_sw128(sb + OFF_XA + 2048 * k, XA_BLK, 1024), ID_KM128, k > 0 ? 1u : 0u);
+        for (int k = 0; k < 4; ++k)
+          mma_bf16(x.tmem + TM_DX, sdesc_sw128(x.sb + OFF_TZP + 32 * k, 16, 1024),
+                   sdesc_sw128(x.sb + OFF_XA + b * XA_BUF + 2048 * k, XA_BLK, 1024), ID_KM128, k > 0 ? 1u : 0u);
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        mma_bf16(tmem + 192, sdesc_sw128(sb + OFF_TZ + 32 * k, 16, 1024), sdesc_sw128(sb + OFF_U + 2048 * k, 8192, 1024),
-                 ID_KM64, k > 0 ? 1u : 0u);
-      mma_commit(bar_mma);
+        for (int k = 0; k < 4; ++k)
+          mma_bf16(x.tmem + TM_DA + 64 * b, sdesc_sw128(x.sb + OFF_TZP + 32 * k, 16, 1024),
+                   sdesc_sw128(x.sb + OFF_U + b * 8192 + 2048 * k, 8192, 1024), ID_KM64, k > 0 ? 1u : 0u);
+      }
+      mma_commit(bar_addr(x, B_KMMA));
     }
-    if (!(ok = cta_wait(bar_mma, ph_mma))) break;
-    ph_mma ^= 1;
+    if (!group_wait(BAR_KEY, NKEY, bar_addr(x, B_KMMA), kphase, fail)) return false;
+    kphase ^= 1;
     tc_fence_after();
 
-    // ---------------------------------------------------------------- E: -T A_m in place of A_m; e^m S
-    {
-      if (quad < 2) {
-        const int row = 32 * quad + lane;
+    // ------------------------------------------------------------ -T A_m in place of A_m; hand over
+    if (quad < 2) {  // rows 0..63; warp group half khalf owns channel block khalf
+      const int row = 32 * quad + lane;
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          float v[32];
-          tmem_ld32(tl + 64 + 64 * half + 32 * part, v);
-          tmem_wait_ld();
+      for (int part = 0; part < 2; ++part) {
+        float v[32];
+        tmem_ld32(tl + TM_DX + 64 * khalf + 32 * part, v);
+        tmem_wait_ld();
 #pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            float e[8];
+        for (int y = 0; y < 4; ++y) {
+          float e[8];
 #pragma unroll
-            for (int t = 0; t < 8; ++t) e[t] = -v[8 * x + t];
-            st_s128(sm + OFF_XA + half * XA_BLK + sw128(row, 32 * part + 8 * x), pack8(e));
-          }
+          for (int t = 0; t < 8; ++t) e[t] = -v[8 * y + t];
+          st_s128(xa + khalf * XA_BLK + sw128(row, 32 * part + 8 * y), pack8(e));
         }
-      }
-      const float em = s_em[c_me];
-#pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        float e[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) e[t] = em * S[8 * x + t];
-        st_s128(sm + OFF_SM + sw128(c_me, 32 * half + 8 * x), pack8(e));
       }
     }
     tc_fence_before();
     fence_proxy_async();
-    __syncthreads();
+    group_sync(BAR_KEY, NKEY);
+    if (kt == 0) mbar_arrive(bar_addr(x, B_READY0 + b));
+  }
+  return true;
+}
 
-    // ---------------------------------------------------------------- M5: D_a += [-T A_m; Q_m] (e^m S)
-    if (tid == 0) {
+// ==================================================================== state side (warps 0-3)
+// Holds the fp32 state slice (thread = key channel x 64 value columns) and runs the serial chain.
+__device__ bool state_side(const Ctx &x, float (&S)[64], __nv_bfloat16 *o) {
+  uint8_t *sm = x.sm;
+  const int st = threadIdx.x, warp = st >> 5, lane = st & 31, quad = warp;
+  const uint32_t tl = x.tmem + ((uint32_t)(32 * quad) << 16);
+  const int c_me = st;  // key channel of this thread (TMEM lane of K_m^T Delta)
+  uint32_t sphase = 0;
+
+  for (int c = 0; c < x.nchunks; ++c) {
+    const int b = c & 1;
+    const int Cc = min(C, x.len - c * C);
+    const float *s_em = reinterpret_cast<const float *>(sm + OFF_SC) + b * 384;
+    const int tok0 = (int)(x.bos + (int64_t)c * C);
+
+    if (!group_wait(BAR_STATE, NSTATE, bar_addr(x, B_READY0 + b), (c >> 1) & 1)) return false;
+
+    // ------------------------------------------------------------ e^m S -> shared (bf16)
+    {
+      const float em = s_em[c_me];
+#pragma unroll
+      for (int y = 0; y < 8; ++y) {
+        float e[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) e[t] = em * S[8 * y + t];
+        st_s128(sm + OFF_SM + sw128(c_me, 8 * y), pack8(e));
+      }
+    }
+    fence_proxy_async();
+    group_sync(BAR_STATE, NSTATE);
+
+    // ------------------------------------------------------------ M5: D_a += [-T A_m; Q_m] (e^m S)
+    if (st == 0) {
       tc_fence_after();
 #pragma unroll
       for (int k = 0; k < DK / 16; ++k)
-        mma_bf16(tmem + 192, sdesc_sw128(sb + OFF_XA + (k >> 2) * XA_BLK + (k & 3) * 32, 16, 1024),
-                 sdesc_sw128(sb + OFF_SM + 2048 * k, 16384, 1024), ID_KM64, 1u);
-      mma_commit(bar_mma);
+        mma_bf16(x.tmem + TM_DA + 64 * b,
+                 sdesc_sw128(x.sb + OFF_XA + b * XA_BUF + (k >> 2) * XA_BLK + (k & 3) * 32, 16, 1024),
+                 sdesc_sw128(x.sb + OFF_SM + 2048 * k, 16384, 1024), ID_KM64, 1u);
+      mma_commit(bar_addr(x, B_SMMA));
     }
-    if (!(ok = cta_wait(bar_mma, ph_mma))) break;
-    ph_mma ^= 1;
+    if (!group_wait(BAR_STATE, NSTATE, bar_addr(x, B_SMMA), sphase)) return false;
+    sphase ^= 1;
     tc_fence_after();
 
-    // ---------------------------------------------------------------- F: Delta -> smem
+    // ------------------------------------------------------------ Delta -> shared (bf16)
     if (quad < 2) {
-      float v[32];
-      tmem_ld32(tl + 192 + 32 * half, v);
-      tmem_wait_ld();
       const int row = 32 * quad + lane;
 #pragma unroll
-      for (int x = 0; x < 4; ++x) st_s128(sm + OFF_DL + sw128(row, 32 * half + 8 * x), pack8(&v[8 * x]));
-    }
-    tc_fence_before();
-    fence_proxy_async();
-    __syncthreads();
-
-    // ---------------------------------------------------------------- M6, M7: K_m^T Delta; D_a += [P; P] Delta
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        mma_bf16(tmem + 0, sdesc_sw128(sb + OFF_KT + 2048 * k, KT_BLK, 1024), sdesc_sw128(sb + OFF_DL + 2048 * k, 8192, 1024),
-                 ID_MNMN, k > 0 ? 1u : 0u);
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        mma_bf16(tmem + 192, sdesc_sw128(sb + OFF_PP + 32 * k, 16, 1024), sdesc_sw128(sb + OFF_DL + 2048 * k, 8192, 1024),
-                 ID_KM64, 1u);
-      mma_commit(bar_mma);
-    }
-    if (!(ok = cta_wait(bar_mma, ph_mma))) break;
-    ph_mma ^= 1;
-    tc_fence_after();
-
-    // ---------------------------------------------------------------- G: state update, O -> global
-    {
-      float v[32];
-      tmem_ld32(tl + 0 + 32 * half, v);
-      tmem_wait_ld();
-      const float g1 = s_egc[c_me], g2 = s_egcm[c_me];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) S[j] = fmaf(g2, v[j], g1 * S[j]);
-      if (quad >= 2) {  // warp-uniform: tcgen05.ld is a warp-collective instruction
-        const int r = 32 * quad + lane - 64;
-        tmem_ld32(tl + 192 + 32 * half, v);
+      for (int part = 0; part < 2; ++part) {
+        float v[32];
+        tmem_ld32(tl + TM_DA + 64 * b + 32 * part, v);
         tmem_wait_ld();
-        if (r < Cc) store_row32_bf16(o + ((size_t)(tok0 + r) * a.H + h) * (size_t)a.dv + j0 + 32 * half, v);
+#pragma unroll
+        for (int y = 0; y < 4; ++y) st_s128(sm + OFF_SM + sw128(row, 32 * part + 8 * y), pack8(&v[8 * y]));
       }
     }
     tc_fence_before();
-    __syncthreads();
-  }
+    fence_proxy_async();
+    group_sync(BAR_STATE, NSTATE);
 
-  if (ok && a.ST) {
+    // ------------------------------------------------------------ M6, M7: K_m^T Delta; D_a += [*; P] Delta
+    if (st == 0) {
+      tc_fence_after();
 #pragma unroll
-    for (int x = 0; x < 8; ++x)
-      reinterpret_cast<float4 *>(a.ST + s_off)[x] = make_float4(S[4 * x], S[4 * x + 1], S[4 * x + 2], S[4 * x + 3]);
+      for (int k = 0; k < 4; ++k)
+        mma_bf16(x.tmem + TM_DB, sdesc_sw128(x.sb + OFF_KT + b * KT_BUF + 2048 * k, KT_BLK, 1024),
+                 sdesc_sw128(x.sb + OFF_SM + 2048 * k, 8192, 1024), ID_MNMN, k > 0 ? 1u : 0u);
+      // A rows 64..127 = P of this chunk; rows 0..63 (zeros or the other P tile) only touch the
+      // already consumed Delta half of D_a
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        mma_bf16(x.tmem + TM_DA + 64 * b, sdesc_sw128(x.sb + OFF_TZP + 8192 + b * 8192 + 32 * k, 16, 1024),
+                 sdesc_sw128(x.sb + OFF_SM + 2048 * k, 8192, 1024), ID_KM64, 1u);
+      mma_commit(bar_addr(x, B_SMMA));
+      mma_commit(bar_addr(x, B_STDONE0 + b));
+    }
+    if (!group_wait(BAR_STATE, NSTATE, bar_addr(x, B_SMMA), sphase)) return false;
+    sphase ^= 1;
+    tc_fence_after();
+
+    // ------------------------------------------------------------ state update, O -> global
+    {
+      const float g1 = s_em[256 + c_me], g2 = s_em[128 + c_me];  // e^{g_C}, e^{g_C - m}
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        float v[32];
+        tmem_ld32(tl + TM_DB + 32 * part, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) S[32 * part + j] = fmaf(g2, v[j], g1 * S[32 * part + j]);
+      }
+      if (quad >= 2) {  // warp-uniform: tcgen05.ld is a warp-collective instruction
+        const int r = 32 * quad + lane - 64;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          float v[32];
+          tmem_ld32(tl + TM_DA + 64 * b + 32 * part, v);
+          tmem_wait_ld();
+          if (r < Cc) store_row32_bf16(o + ((size_t)(tok0 + r) * x.H + x.h) * (size_t)x.dv + x.j0 + 32 * part, v);
+        }
+      }
+    }
+    tc_fence_before();
+    group_sync(BAR_STATE, NSTATE);
+    if (st == 0) mbar_arrive(bar_addr(x, B_DAFREE0 + b));
   }
-  if (!ok && tid == 0) atomicExch(&g_device_status, 4);
+  return true;
+}
+
+__global__ void __launch_bounds__(NT, 1)
+    chunk_fwd_tc_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_b,
+                        const __grid_constant__ CUtensorMap tm_al, const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_w) {
+  extern __shared__ uint8_t smem_raw[];
+  Ctx x;
+  x.sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  x.sb = smem_u32(x.sm);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(x.sm + OFF_BAR + 8 * B_COUNT);
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tiles = a.dv / NV;
+  const int tile = blockIdx.x % tiles;
+  x.h = (blockIdx.x / tiles) % a.H;
+  const int n = blockIdx.x / (tiles * a.H);
+  x.j0 = tile * NV;
+  x.H = a.H;
+  x.dv = a.dv;
+  seq_span(a, n, x.bos, x.len);
+  x.nchunks = (x.len + C - 1) / C;
+
+  if (tid == 0) {
+    for (int i = 0; i < B_COUNT; ++i) mbar_init(x.sb + OFF_BAR + 8 * i, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_b);
+    prefetch_tmap(&tm_al); prefetch_tmap(&tm_v); prefetch_tmap(&tm_w);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  // the zero rows of [T ; 0] and the never-written upper blocks of T
+  for (int e = tid; e < 8192 / 16; e += NT) st_s128(x.sm + OFF_TZP + 8192 + 16 * e, make_uint4(0u, 0u, 0u, 0u));
+  float *Ts = reinterpret_cast<float *>(x.sm + OFF_TS);
+  for (int e = tid; e < 64 * LDF; e += NT) Ts[e] = 0.f;
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  x.tmem = *tmem_slot;
+
+  bool ok;
+  if (warp < 4) {
+    // state slice: key channel tid, value columns j0 .. j0+63
+    const size_t s_off = (((size_t)n * a.H + x.h) * DK + tid) * (size_t)a.dv + x.j0;
+    float S[64];
+    if (a.S0) {
+#pragma unroll
+      for (int y = 0; y < 16; ++y) {
+        const float4 t = reinterpret_cast<const float4 *>(a.S0 + s_off)[y];
+        S[4 * y] = t.x; S[4 * y + 1] = t.y; S[4 * y + 2] = t.z; S[4 * y + 3] = t.w;
+      }
+    } else {
+#pragma unroll
+      for (int y = 0; y < 64; ++y) S[y] = 0.f;
+    }
+    ok = state_side(x, S, reinterpret_cast<__nv_bfloat16 *>(a.o));
+    if (ok && a.ST) {
+#pragma unroll
+      for (int y = 0; y < 16; ++y)
+        reinterpret_cast<float4 *>(a.ST + s_off)[y] = make_float4(S[4 * y], S[4 * y + 1], S[4 * y + 2], S[4 * y + 3]);
+    }
+  } else {
+    ok = key_side(x, &tm_q, &tm_k, &tm_b, &tm_al, &tm_v, &tm_w);
+  }
+  if (!ok && (tid == 0 || tid == NSTATE)) atomicExch(&g_device_status, 4);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc(x.tmem, TMEM_COLS);
   }
 }
 
