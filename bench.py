@@ -91,7 +91,7 @@ class ClockSampler:
         0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, device_index, period_s=0.005):
+    def __init__(self, device_index, period_s=0.001):
         self.samples, self.period, self._stop = [], period_s, threading.Event()
         self.ok = False
         self.max_mhz = None
@@ -232,12 +232,16 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--profile-case", choices=["chunk", "decode"],
+                    help="run one warm-up and one measured launch of that kernel on its full workload, for ncu")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     ws, rank, local = init_dist()
     if args.impl == "reference":
         return run_reference(args, ws, rank)
+    if args.profile_case:
+        return profile_case(args.profile_case)
 
     import gated_delta_rule_131_b200 as gdn2
     gdn2.lib()
@@ -328,6 +332,26 @@ def main():
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+    return 0
+
+
+def profile_case(which):
+    """Two launches (warm-up + measured) of one kernel on its full workload; nothing else is timed."""
+    import gated_delta_rule_131_b200 as gdn2
+    dev = torch.device("cuda", 0)
+    if which == "chunk":
+        wl = W.WORKLOADS["layer_1p3b"]
+        d = W.chunk_inputs(wl, device=dev, seed=0)
+        for _ in range(2):
+            gdn2.chunk_fwd(*[d[n] for n in TOK], S0=d["S0"])
+    else:
+        wl = W.WORKLOADS["decode"]
+        S = W.decode_state(wl, device=dev, seed=0)
+        for s in range(2):
+            t = W.decode_token_inputs(wl, s, device=dev, seed=0)
+            gdn2.decode_step(*[t[n] for n in TOK], S=S)
+    torch.cuda.synchronize(dev)
+    print(f"profile case {which}: ok", flush=True)
     return 0
 
 

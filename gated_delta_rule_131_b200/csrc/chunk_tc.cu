@@ -197,7 +197,7 @@ __device__ __forceinline__ void issue_chunk_loads(const Ctx &x, int c, const CUt
 
 // ==================================================================== key side (warps 4-11)
 // For each chunk: decay factors, L|P, T, [T; 0][A_m | U]; hands the chunk to the state side.
-__device__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_b,
+__device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_b,
                          const CUtensorMap *tm_al, const CUtensorMap *tm_v, const CUtensorMap *tm_w) {
   uint8_t *sm = x.sm;
   const int kt = threadIdx.x - NSTATE, kwarp = kt >> 5, lane = kt & 31, quad = kwarp & 3, khalf = kwarp >> 2;
@@ -493,7 +493,7 @@ __device__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, const CUtensorMa
 
 // ==================================================================== state side (warps 0-3)
 // Holds the fp32 state slice (thread = key channel x 64 value columns) and runs the serial chain.
-__device__ bool state_side(const Ctx &x, float (&S)[64], __nv_bfloat16 *o) {
+__device__ __forceinline__ bool state_side(const Ctx &x, float (&S)[64], __nv_bfloat16 *o) {
   uint8_t *sm = x.sm;
   const int st = threadIdx.x, warp = st >> 5, lane = st & 31, quad = warp;
   const uint32_t tl = x.tmem + ((uint32_t)(32 * quad) << 16);
@@ -608,7 +608,8 @@ __global__ void __launch_bounds__(NT, 1)
                         const __grid_constant__ CUtensorMap tm_w) {
   extern __shared__ uint8_t smem_raw[];
   Ctx x;
-  x.sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // align by pointer arithmetic on the shared array, so every derived pointer stays a shared-space pointer
+  x.sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   x.sb = smem_u32(x.sm);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(x.sm + OFF_BAR + 8 * B_COUNT);
 
