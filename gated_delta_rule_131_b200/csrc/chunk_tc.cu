@@ -29,9 +29,10 @@
 //   cols [0, 64)    L|P, then K_m^T Delta
 //   cols [64, 192)  [T; 0] A_m
 //   cols [192, 256) D_a = [Delta; O]
-// T is formed in fp32: the four 16x16 diagonal blocks by right-looking
+// T is formed in fp32 storage: the four 16x16 diagonal blocks by right-looking
 // substitution, then merged into 32x32 and 64x64 inverses with
-// [[A,0],[C,B]]^-1 = [[A^-1,0],[-B^-1 C A^-1, B^-1]].
+// [[A,0],[C,B]]^-1 = [[A^-1,0],[-B^-1 C A^-1, B^-1]]; the merge products run on
+// the warp-level tensor cores with tf32 operands (T is rounded to bf16 after).
 // Precondition of the factorisation: per key channel, the decay accumulated
 // over any 32 consecutive tokens of a chunk stays above about e^-80 (the fp32
 // range); every workload here is far inside it.
@@ -164,6 +165,38 @@ __device__ __forceinline__ void row_factors(uint8_t *xa, uint8_t *kt, int r, int
   st_s128(pa, wa);
   st_s128(pq, wq);
   st_s128(pk, wk);
+}
+
+// D (16 x 8) = A (16 x K) B (K x 8) on the warp-level tensor-core path (mma.sync, tf32 operands
+// rounded from fp32, fp32 accumulate).  A points at element (0, 0) of a row-major fp32 block with
+// row stride LDF, B likewise.  Fragment ownership follows the m16n8k8 tf32 layout: lane = 4 g + t
+// holds D rows g and g + 8, columns 2t and 2t + 1.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+template <int K>
+__device__ __forceinline__ void mma_tf32_16x8(const float *A, const float *B, int lane, float (&d)[4]) {
+  const int g = lane >> 2, t = lane & 3;
+  d[0] = d[1] = d[2] = d[3] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < K; kk += 8) {
+    const uint32_t a0 = to_tf32(A[g * LDF + kk + t]), a1 = to_tf32(A[(g + 8) * LDF + kk + t]);
+    const uint32_t a2 = to_tf32(A[g * LDF + kk + t + 4]), a3 = to_tf32(A[(g + 8) * LDF + kk + t + 4]);
+    const uint32_t b0 = to_tf32(B[(kk + t) * LDF + g]), b1 = to_tf32(B[(kk + t + 4) * LDF + g]);
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+}
+// Store a 16 x 8 tile (times `scale`) into a row-major fp32 block with row stride LDF.
+__device__ __forceinline__ void store_16x8(float *D, int lane, const float (&d)[4], float scale) {
+  const int g = lane >> 2, t = lane & 3;
+  *reinterpret_cast<float2 *>(&D[g * LDF + 2 * t]) = make_float2(scale * d[0], scale * d[1]);
+  *reinterpret_cast<float2 *>(&D[(g + 8) * LDF + 2 * t]) = make_float2(scale * d[2], scale * d[3]);
 }
 
 struct Ctx {
@@ -370,64 +403,33 @@ __device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, 
       for (int r = 0; r < 16; ++r) Tb[r * LDF + j] = xv[r];
     }
     group_sync(BAR_KEY, NKEY);
-    {  // T_{R,R-1} for R = 1, 3: Y = L_{R,R-1} T_{R-1,R-1} (parked in the upper block (R-1, R) of L)
-      float acc[2];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int R = 1 + 2 * u, r = kt >> 4, cl = kt & 15;
-        const float *Lr = Ls + (16 * R + r) * LDF + 16 * (R - 1);
-        const float *Tc = Ts + 16 * (R - 1) * LDF + 16 * (R - 1) + cl;
-        float s = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) s = fmaf(Lr[k], Tc[k * LDF], s);
-        acc[u] = s;
-      }
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int R = 1 + 2 * u, r = kt >> 4, cl = kt & 15;
-        Ls[(16 * (R - 1) + r) * LDF + 16 * R + cl] = acc[u];
-      }
+    // merges on the warp-level tensor cores (tf32): 16x16 blocks, then the 32x32 block
+    if (kwarp < 4) {  // Y_R = L_{R,R-1} T_{R-1,R-1}, R = 1, 3, parked in the upper block (R-1, R) of L
+      const int R = (kwarp < 2) ? 1 : 3, nt = kwarp & 1;
+      float d[4];
+      mma_tf32_16x8<16>(Ls + 16 * R * LDF + 16 * (R - 1), Ts + 16 * (R - 1) * LDF + 16 * (R - 1) + 8 * nt, lane, d);
+      store_16x8(Ls + 16 * (R - 1) * LDF + 16 * R + 8 * nt, lane, d, 1.f);
     }
     group_sync(BAR_KEY, NKEY);
-    {  // T_{R,R-1} = -T_RR Y
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int R = 1 + 2 * u, r = kt >> 4, cl = kt & 15;
-        const float *Tr = Ts + (16 * R + r) * LDF + 16 * R;
-        const float *Yc = Ls + 16 * (R - 1) * LDF + 16 * R + cl;
-        float s = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) s = fmaf(Tr[k], Yc[k * LDF], s);
-        Ts[(16 * R + r) * LDF + 16 * (R - 1) + cl] = -s;
-      }
+    if (kwarp < 4) {  // T_{R,R-1} = -T_RR Y_R
+      const int R = (kwarp < 2) ? 1 : 3, nt = kwarp & 1;
+      float d[4];
+      mma_tf32_16x8<16>(Ts + 16 * R * LDF + 16 * R, Ls + 16 * (R - 1) * LDF + 16 * R + 8 * nt, lane, d);
+      store_16x8(Ts + 16 * R * LDF + 16 * (R - 1) + 8 * nt, lane, d, -1.f);
     }
     group_sync(BAR_KEY, NKEY);
-    {  // lower-left 32x32 block: Y = L[32:64, 0:32] T[0:32, 0:32] (parked in L[0:32, 32:64])
-      const int r = kt >> 3, c4 = 4 * (kt & 7);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      const float *Lr = Ls + (32 + r) * LDF;
-#pragma unroll 8
-      for (int k = 0; k < 32; ++k) {
-        const float l = Lr[k];
-        const float4 t = *reinterpret_cast<const float4 *>(&Ts[k * LDF + c4]);
-        acc.x = fmaf(l, t.x, acc.x); acc.y = fmaf(l, t.y, acc.y);
-        acc.z = fmaf(l, t.z, acc.z); acc.w = fmaf(l, t.w, acc.w);
-      }
-      *reinterpret_cast<float4 *>(&Ls[r * LDF + 32 + c4]) = acc;  // disjoint from what this stage reads
+    {  // lower-left 32x32 block: Y = L[32:64, 0:32] T[0:32, 0:32], parked in L[0:32, 32:64]
+      const int mt = kwarp >> 2, nt = kwarp & 3;
+      float d[4];
+      mma_tf32_16x8<32>(Ls + (32 + 16 * mt) * LDF, Ts + 8 * nt, lane, d);
+      store_16x8(Ls + 16 * mt * LDF + 32 + 8 * nt, lane, d, 1.f);  // disjoint from what this stage reads
     }
     group_sync(BAR_KEY, NKEY);
     {  // T[32:64, 0:32] = -T[32:64, 32:64] Y
-      const int r = kt >> 3, c4 = 4 * (kt & 7);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      const float *Tr = Ts + (32 + r) * LDF + 32;
-#pragma unroll 8
-      for (int k = 0; k < 32; ++k) {
-        const float t = Tr[k];
-        const float4 y = *reinterpret_cast<const float4 *>(&Ls[k * LDF + 32 + c4]);
-        acc.x = fmaf(t, y.x, acc.x); acc.y = fmaf(t, y.y, acc.y);
-        acc.z = fmaf(t, y.z, acc.z); acc.w = fmaf(t, y.w, acc.w);
-      }
-      *reinterpret_cast<float4 *>(&Ts[(32 + r) * LDF + c4]) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+      const int mt = kwarp >> 2, nt = kwarp & 3;
+      float d[4];
+      mma_tf32_16x8<32>(Ts + (32 + 16 * mt) * LDF + 32, Ls + 32 + 8 * nt, lane, d);
+      store_16x8(Ts + (32 + 16 * mt) * LDF + 8 * nt, lane, d, -1.f);
     }
     group_sync(BAR_KEY, NKEY);
     {  // T -> rows 0..63 of [T ; 0], bf16
