@@ -93,7 +93,7 @@ constexpr uint32_t ID_KM128 = idesc_bf16(128, 128, false, true); // same, N = 12
 constexpr uint32_t ID_MNMN = idesc_bf16(128, 64, true, true);    // K_m^T Delta
 
 // mbarriers (8 bytes each) at OFF_BAR
-enum { B_FULL0 = 0, B_FULL1, B_KMMA, B_SMMA, B_READY0, B_READY1, B_STDONE0, B_STDONE1, B_DAFREE0, B_DAFREE1, B_COUNT };
+enum { B_FULL0 = 0, B_FULL1, B_KMMA, B_SMMA, B_READY0, B_READY1, B_KBDONE, B_COUNT };
 
 __device__ __forceinline__ uint4 ld_s128(const uint8_t *p) { return *reinterpret_cast<const uint4 *>(p); }
 __device__ __forceinline__ void st_s128(uint8_t *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
@@ -139,19 +139,16 @@ __device__ __forceinline__ void store_row32_bf16(__nv_bfloat16 *dst, const float
   for (int x = 0; x < 4; ++x) reinterpret_cast<uint4 *>(dst)[x] = pack8(&v[8 * x]);
 }
 
-// Decay-absorbed operands of one token row for 8 key channels, in place:
-// A_m = b k f, Q_m = q f, K_m = k fi with f = e^{g_r - m}, fi = 1/f; rows >= Cc are zeroed.
-__device__ __forceinline__ void row_factors(uint8_t *xa, uint8_t *kt, int r, int cb, int x8, int Cc, const float *f,
-                                            const float *fi) {
-  uint8_t *pa = xa + cb * XA_BLK + sw128(r, 8 * x8);
-  uint8_t *pq = pa + 8192;
-  uint8_t *pk = kt + cb * KT_BLK + sw128(r, 8 * x8);
+// Decay-absorbed operands of one token row for 8 key channels, from the raw bf16 values already in
+// registers: A_m = b k f, Q_m = q f, K_m = k fi with f = e^{g_r - m}, fi = 1/f (zeros when !valid).
+__device__ __forceinline__ void row_factors(uint8_t *pa, uint8_t *pq, uint8_t *pk, uint4 rb, uint4 rq, uint4 rk,
+                                            bool valid, const float *f, const float *fi) {
   uint4 wa = make_uint4(0u, 0u, 0u, 0u), wq = wa, wk = wa;
-  if (r < Cc) {
+  if (valid) {
     float bb[8], qv[8], kv[8], ea[8], eq[8], ek[8];
-    unpack8(ld_s128(pa), bb);
-    unpack8(ld_s128(pq), qv);
-    unpack8(ld_s128(pk), kv);
+    unpack8(rb, bb);
+    unpack8(rq, qv);
+    unpack8(rk, kv);
 #pragma unroll
     for (int t = 0; t < 8; ++t) {
       ea[t] = bb[t] * kv[t] * f[t];
@@ -240,7 +237,6 @@ __device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, 
   float *scan = Ls;  // [16 groups][128 channels] during the factor phase
   uint32_t kphase = 0;
 
-  if (kt == 0 && x.nchunks > 0) issue_chunk_loads(x, 0, tm_q, tm_k, tm_b, tm_al, tm_v, tm_w);
 
   for (int c = 0; c < x.nchunks; ++c) {
     const int b = c & 1;
@@ -256,95 +252,118 @@ __device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, 
     // ------------------------------------------------------------ decay factors, operands in place
     {
       // thread = 8 key channels (chunk x8 of channel block cb) x 4 tokens (group G = rows 4G..4G+3);
-      // warps 0-3 of the group hold tokens 0..31 (walk back to token 31), warps 4-7 tokens 32..63
+      // groups 0-7 hold tokens 0..31 (walk back to token 31), groups 8-15 tokens 32..63 (walk forward).
+      // All raw tiles this thread needs are loaded first, so their latency overlaps the barriers.
       const int ch8 = kt & 15, G = kt >> 4, cb = ch8 >> 3, x8 = ch8 & 7;
-      float al[4][8];
+      uint4 ra[4], rb[4], rq[4], rk[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int r = 4 * G + i;
-        if (r < Cc) {
-          unpack8(ld_s128(sm + OFF_AL + cb * 8192 + sw128(r, 8 * x8)), al[i]);
-        } else {
+        const uint32_t o = sw128(4 * G + i, 8 * x8);
+        ra[i] = ld_s128(sm + OFF_AL + cb * 8192 + o);
+        rb[i] = ld_s128(xa + cb * XA_BLK + o);
+        rq[i] = ld_s128(xa + cb * XA_BLK + 8192 + o);
+        rk[i] = ld_s128(ktile + cb * KT_BLK + o);
+      }
+      const int ur = kt >> 2;  // U = w (.) v: token row ur, value columns 16 (kt & 3) .. +15
+      uint8_t *ub = sm + OFF_U + b * 8192;
+      uint4 rv[2], rw[2];
 #pragma unroll
-          for (int t = 0; t < 8; ++t) al[i][t] = 1.f;
-        }
+      for (int y = 0; y < 2; ++y) {
+        rv[y] = ld_s128(ub + sw128(ur, 16 * (kt & 3) + 8 * y));
+        rw[y] = ld_s128(sm + OFF_W + sw128(ur, 16 * (kt & 3) + 8 * y));
       }
       float gp[8];
 #pragma unroll
-      for (int t = 0; t < 8; ++t) gp[t] = al[0][t] * al[1][t] * al[2][t] * al[3][t];
+      for (int t = 0; t < 8; ++t) gp[t] = 1.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (4 * G + i < Cc) {
+          float al[8];
+          unpack8(ra[i], al);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) gp[t] *= al[t];
+        }
       *reinterpret_cast<float4 *>(&scan[G * 128 + 8 * ch8]) = make_float4(gp[0], gp[1], gp[2], gp[3]);
       *reinterpret_cast<float4 *>(&scan[G * 128 + 8 * ch8 + 4]) = make_float4(gp[4], gp[5], gp[6], gp[7]);
       group_sync(BAR_KEY, NKEY);
-      if (kt < 128) {
-        float em = 1.f, egcm = 1.f;
-        for (int g = 0; g < 8; ++g) em *= scan[g * 128 + kt];
-        for (int g = 8; g < 16; ++g) egcm *= scan[g * 128 + kt];
-        s_em[kt] = em;
-        s_egcm[kt] = egcm;
-        s_egc[kt] = em * egcm;
-      }
-      float run[8];
+      if (kt < 128) {  // per channel: products between each group and token 31, in place of the group products
+        float p[16];
 #pragma unroll
-      for (int t = 0; t < 8; ++t) run[t] = 1.f;
-      const int g0 = (G < 8) ? G + 1 : 8, g1 = (G < 8) ? 8 : G;
-      for (int g = g0; g < g1; ++g) {
-        const float4 p0 = *reinterpret_cast<const float4 *>(&scan[g * 128 + 8 * ch8]);
-        const float4 p1 = *reinterpret_cast<const float4 *>(&scan[g * 128 + 8 * ch8 + 4]);
-        run[0] *= p0.x; run[1] *= p0.y; run[2] *= p0.z; run[3] *= p0.w;
-        run[4] *= p1.x; run[5] *= p1.y; run[6] *= p1.z; run[7] *= p1.w;
+        for (int g = 0; g < 16; ++g) p[g] = scan[g * 128 + kt];
+        float acc = 1.f;
+#pragma unroll
+        for (int g = 7; g >= 0; --g) {
+          scan[g * 128 + kt] = acc;  // prod over groups g+1..7
+          acc *= p[g];
+        }
+        const float em = acc;
+        acc = 1.f;
+#pragma unroll
+        for (int g = 8; g < 16; ++g) {
+          scan[g * 128 + kt] = acc;  // prod over groups 8..g-1
+          acc *= p[g];
+        }
+        s_em[kt] = em;
+        s_egcm[kt] = acc;
+        s_egc[kt] = em * acc;
       }
+      group_sync(BAR_KEY, NKEY);
+      float run[8];
+      {
+        const float4 p0 = *reinterpret_cast<const float4 *>(&scan[G * 128 + 8 * ch8]);
+        const float4 p1 = *reinterpret_cast<const float4 *>(&scan[G * 128 + 8 * ch8 + 4]);
+        run[0] = p0.x; run[1] = p0.y; run[2] = p0.z; run[3] = p0.w;
+        run[4] = p1.x; run[5] = p1.y; run[6] = p1.z; run[7] = p1.w;
+      }
+      uint8_t *pa0 = xa + cb * XA_BLK, *pk0 = ktile + cb * KT_BLK;
       if (G < 8) {
 #pragma unroll
         for (int i = 3; i >= 0; --i) {  // run = prod_{r < s <= 31} alpha_s
-          float f[8], fi[8];
+          const int r = 4 * G + i;
+          float al[8], f[8], fi[8];
+          unpack8(ra[i], al);
 #pragma unroll
           for (int t = 0; t < 8; ++t) {
             fi[t] = run[t];
             f[t] = fast_rcp(run[t]);
-            run[t] *= al[i][t];
+            if (r < Cc) run[t] *= al[t];
           }
-          row_factors(xa, ktile, 4 * G + i, cb, x8, Cc, f, fi);
+          const uint32_t o = sw128(r, 8 * x8);
+          row_factors(pa0 + o, pa0 + 8192 + o, pk0 + o, rb[i], rq[i], rk[i], r < Cc, f, fi);
         }
       } else {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {  // run = prod_{32 <= s <= r} alpha_s
-          float f[8], fi[8];
+          const int r = 4 * G + i;
+          float al[8], f[8], fi[8];
+          unpack8(ra[i], al);
 #pragma unroll
           for (int t = 0; t < 8; ++t) {
-            run[t] *= al[i][t];
+            if (r < Cc) run[t] *= al[t];
             f[t] = run[t];
             fi[t] = fast_rcp(run[t]);
           }
-          row_factors(xa, ktile, 4 * G + i, cb, x8, Cc, f, fi);
+          const uint32_t o = sw128(r, 8 * x8);
+          row_factors(pa0 + o, pa0 + 8192 + o, pk0 + o, rb[i], rq[i], rk[i], r < Cc, f, fi);
         }
       }
-    }
-    {  // U = w (.) v for the 64 value columns of this CTA
-      const int r = kt >> 2;
-      uint8_t *ub = sm + OFF_U + b * 8192;
 #pragma unroll
       for (int y = 0; y < 2; ++y) {
-        const int col = 16 * (kt & 3) + 8 * y;
-        uint8_t *pu = ub + sw128(r, col);
         float vv[8], ww[8], uu[8];
-        unpack8(ld_s128(pu), vv);
-        unpack8(ld_s128(sm + OFF_W + sw128(r, col)), ww);
+        unpack8(rv[y], vv);
+        unpack8(rw[y], ww);
 #pragma unroll
-        for (int t = 0; t < 8; ++t) uu[t] = (r < Cc) ? vv[t] * ww[t] : 0.f;
-        st_s128(pu, pack8(uu));
+        for (int t = 0; t < 8; ++t) uu[t] = (ur < Cc) ? vv[t] * ww[t] : 0.f;
+        st_s128(ub + sw128(ur, 16 * (kt & 3) + 8 * y), pack8(uu));
       }
     }
     fence_proxy_async();
     group_sync(BAR_KEY, NKEY);
 
-    // ------------------------------------------------------------ prefetch chunk c+1; M1: [L; P] = [A_m; Q_m] K_m^T
-    bool fail = false;
+    // ------------------------------------------------------------ M1: [L; P] = [A_m; Q_m] K_m^T
+    // (the alpha and w tiles of chunk c are consumed: the state side may now load chunk c+1)
     if (kt == 0) {
-      if (c + 1 < x.nchunks) {
-        // buffer (c+1)&1 was last used by chunk c-1: wait until the state side's MMAs on it finished
-        if (c >= 1) fail = !mbar_wait_bounded(bar_addr(x, B_STDONE0 + ((c + 1) & 1)), ((c - 1) >> 1) & 1, WAIT_NS);
-        if (!fail) issue_chunk_loads(x, c + 1, tm_q, tm_k, tm_b, tm_al, tm_v, tm_w);
-      }
+      mbar_arrive(bar_addr(x, B_KBDONE));
       tc_fence_after();
 #pragma unroll
       for (int k = 0; k < DK / 16; ++k) {
@@ -355,6 +374,7 @@ __device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, 
       }
       mma_commit(bar_addr(x, B_KMMA));
     }
+    const bool fail = false;
     if (!group_wait(BAR_KEY, NKEY, bar_addr(x, B_KMMA), kphase, fail)) return false;
     kphase ^= 1;
     tc_fence_after();
@@ -447,24 +467,20 @@ __device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, 
     group_sync(BAR_KEY, NKEY);
 
     // ------------------------------------------------------------ M3, M4: [T; 0] [A_m | U]
-    fail = false;
+    // (D_a buffer b is free: the state side finished chunk c-2 before it loaded chunk c)
     if (kt == 0) {
-      // D_a buffer b was last read by the state side for chunk c-2
-      if (c >= 2) fail = !mbar_wait_bounded(bar_addr(x, B_DAFREE0 + b), ((c - 2) >> 1) & 1, WAIT_NS);
       tc_fence_after();
-      if (!fail) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma_bf16(x.tmem + TM_DX, sdesc_sw128(x.sb + OFF_TZP + 32 * k, 16, 1024),
-                   sdesc_sw128(x.sb + OFF_XA + b * XA_BUF + 2048 * k, XA_BLK, 1024), ID_KM128, k > 0 ? 1u : 0u);
+      for (int k = 0; k < 4; ++k)
+        mma_bf16(x.tmem + TM_DX, sdesc_sw128(x.sb + OFF_TZP + 32 * k, 16, 1024),
+                 sdesc_sw128(x.sb + OFF_XA + b * XA_BUF + 2048 * k, XA_BLK, 1024), ID_KM128, k > 0 ? 1u : 0u);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma_bf16(x.tmem + TM_DA + 64 * b, sdesc_sw128(x.sb + OFF_TZP + 32 * k, 16, 1024),
-                   sdesc_sw128(x.sb + OFF_U + b * 8192 + 2048 * k, 8192, 1024), ID_KM64, k > 0 ? 1u : 0u);
-      }
+      for (int k = 0; k < 4; ++k)
+        mma_bf16(x.tmem + TM_DA + 64 * b, sdesc_sw128(x.sb + OFF_TZP + 32 * k, 16, 1024),
+                 sdesc_sw128(x.sb + OFF_U + b * 8192 + 2048 * k, 8192, 1024), ID_KM64, k > 0 ? 1u : 0u);
       mma_commit(bar_addr(x, B_KMMA));
     }
-    if (!group_wait(BAR_KEY, NKEY, bar_addr(x, B_KMMA), kphase, fail)) return false;
+    if (!group_wait(BAR_KEY, NKEY, bar_addr(x, B_KMMA), kphase)) return false;
     kphase ^= 1;
     tc_fence_after();
 
@@ -495,12 +511,18 @@ __device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, 
 
 // ==================================================================== state side (warps 0-3)
 // Holds the fp32 state slice (thread = key channel x 64 value columns) and runs the serial chain.
-__device__ __forceinline__ bool state_side(const Ctx &x, float (&S)[64], __nv_bfloat16 *o) {
+__device__ __forceinline__ bool state_side(const Ctx &x, float (&S)[64], __nv_bfloat16 *o, const CUtensorMap *tm_q,
+                                           const CUtensorMap *tm_k, const CUtensorMap *tm_b, const CUtensorMap *tm_al,
+                                           const CUtensorMap *tm_v, const CUtensorMap *tm_w) {
   uint8_t *sm = x.sm;
   const int st = threadIdx.x, warp = st >> 5, lane = st & 31, quad = warp;
   const uint32_t tl = x.tmem + ((uint32_t)(32 * quad) << 16);
   const int c_me = st;  // key channel of this thread (TMEM lane of K_m^T Delta)
   uint32_t sphase = 0;
+  // The state side's thread 0 is also the load producer.  Chunk c+1 goes into buffer (c+1)&1,
+  // last used by chunk c-1, which this side has finished; it waits only until the key side has
+  // read the single-buffered alpha and w tiles of chunk c.
+  if (st == 0 && x.nchunks > 0) issue_chunk_loads(x, 0, tm_q, tm_k, tm_b, tm_al, tm_v, tm_w);
 
   for (int c = 0; c < x.nchunks; ++c) {
     const int b = c & 1;
@@ -508,7 +530,12 @@ __device__ __forceinline__ bool state_side(const Ctx &x, float (&S)[64], __nv_bf
     const float *s_em = reinterpret_cast<const float *>(sm + OFF_SC) + b * 384;
     const int tok0 = (int)(x.bos + (int64_t)c * C);
 
-    if (!group_wait(BAR_STATE, NSTATE, bar_addr(x, B_READY0 + b), (c >> 1) & 1)) return false;
+    bool fail = false;
+    if (st == 0 && c + 1 < x.nchunks) {
+      fail = !mbar_wait_bounded(bar_addr(x, B_KBDONE), c & 1, WAIT_NS);
+      if (!fail) issue_chunk_loads(x, c + 1, tm_q, tm_k, tm_b, tm_al, tm_v, tm_w);
+    }
+    if (!group_wait(BAR_STATE, NSTATE, bar_addr(x, B_READY0 + b), (c >> 1) & 1, fail)) return false;
 
     // ------------------------------------------------------------ e^m S -> shared (bf16)
     {
@@ -568,7 +595,6 @@ __device__ __forceinline__ bool state_side(const Ctx &x, float (&S)[64], __nv_bf
         mma_bf16(x.tmem + TM_DA + 64 * b, sdesc_sw128(x.sb + OFF_TZP + 8192 + b * 8192 + 32 * k, 16, 1024),
                  sdesc_sw128(x.sb + OFF_SM + 2048 * k, 8192, 1024), ID_KM64, 1u);
       mma_commit(bar_addr(x, B_SMMA));
-      mma_commit(bar_addr(x, B_STDONE0 + b));
     }
     if (!group_wait(BAR_STATE, NSTATE, bar_addr(x, B_SMMA), sphase)) return false;
     sphase ^= 1;
@@ -598,7 +624,6 @@ __device__ __forceinline__ bool state_side(const Ctx &x, float (&S)[64], __nv_bf
     }
     tc_fence_before();
     group_sync(BAR_STATE, NSTATE);
-    if (st == 0) mbar_arrive(bar_addr(x, B_DAFREE0 + b));
   }
   return true;
 }
@@ -661,7 +686,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
       for (int y = 0; y < 64; ++y) S[y] = 0.f;
     }
-    ok = state_side(x, S, reinterpret_cast<__nv_bfloat16 *>(a.o));
+    ok = state_side(x, S, reinterpret_cast<__nv_bfloat16 *>(a.o), &tm_q, &tm_k, &tm_b, &tm_al, &tm_v, &tm_w);
     if (ok && a.ST) {
 #pragma unroll
       for (int y = 0; y < 16; ++y)
