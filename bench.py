@@ -250,8 +250,10 @@ def main():
     wl = W.WORKLOADS["layer_1p3b"]
     tokens = wl.B * wl.T
 
-    # two independent input sets (seeded per rank), 2 x 235 MB > L2, alternated between steps
-    sets = [W.chunk_inputs(wl, device=dev, seed=1000 * rank + i) for i in range(2)]
+    # this rank's shard of a global batch of ws x B sequences (each sequence has its own seeded
+    # generator); two independent input sets, 2 x 235 MB > L2, alternated between steps
+    mine = W.shard(wl.B * ws, ws, rank)
+    sets = [W.chunk_inputs(wl, device=dev, seed=i, indices=mine) for i in range(2)]
     o = torch.empty(wl.B, wl.T, wl.H, wl.dv, device=dev, dtype=torch.bfloat16)
     ST = torch.empty(wl.B, wl.H, wl.dk, wl.dv, device=dev, dtype=torch.float32)
     stream = torch.cuda.current_stream(dev)

@@ -116,15 +116,24 @@ def token_inputs(wl: Workload, length: int, device, seed: int, tag: str, index: 
             dict(q=q, k=k, v=v, alpha=alpha, b=b, w=w).items()}
 
 
-def initial_state(wl: Workload, n_seq: int, device, seed: int, index0: int = 0) -> torch.Tensor:
-    """S0 [n_seq, H, d_k, d_v] fp32; sequence i draws from its own generator."""
-    out = torch.zeros(n_seq, wl.H, wl.dk, wl.dv, device=device, dtype=torch.float32)
+def initial_state(wl: Workload, n_seq: int, device, seed: int, index0: int = 0,
+                  indices: Optional[List[int]] = None) -> torch.Tensor:
+    """S0 [n_seq, H, d_k, d_v] fp32; sequence i (global index) draws from its own generator."""
+    idx = list(range(index0, index0 + n_seq)) if indices is None else list(indices)
+    out = torch.zeros(len(idx), wl.H, wl.dk, wl.dv, device=device, dtype=torch.float32)
     if wl.s0 == "normal":
-        for i in range(n_seq):
-            g = _gen(device, seed, "S0", index0 + i)
-            out[i] = torch.randn(wl.H, wl.dk, wl.dv, device=device, dtype=torch.float32,
+        for j, i in enumerate(idx):
+            g = _gen(device, seed, "S0", i)
+            out[j] = torch.randn(wl.H, wl.dk, wl.dv, device=device, dtype=torch.float32,
                                  generator=g) * 0.02
     return out
+
+
+def shard(n_global: int, world_size: int, rank: int) -> List[int]:
+    """Global sequence indices owned by ``rank``: contiguous blocks, sizes differing by at most one."""
+    per, extra = divmod(n_global, world_size)
+    start = rank * per + min(rank, extra)
+    return list(range(start, start + per + (1 if rank < extra else 0)))
 
 
 def seq_lengths(wl: Workload, seed: int) -> List[int]:
@@ -135,15 +144,20 @@ def seq_lengths(wl: Workload, seed: int) -> List[int]:
     return [int(x) for x in torch.randint(1, wl.T + 1, (wl.B,), generator=g)]
 
 
-def chunk_inputs(wl: Workload, device="cpu", seed: int = 0, lengths: Optional[List[int]] = None) -> dict:
-    """All inputs of a chunk_fwd workload.
+def chunk_inputs(wl: Workload, device="cpu", seed: int = 0, lengths: Optional[List[int]] = None,
+                 indices: Optional[List[int]] = None) -> dict:
+    """All inputs of a chunk_fwd workload (or of the sequences ``indices`` of it, e.g. one rank's shard).
 
     Dense: q, k, alpha, b [B, T, H, d_k]; v, w [B, T, H, d_v]; cu_seqlens None.
     Packed: the same tensors are [T_total, H, d]; cu_seqlens int32 [N+1] on ``device``.
     Also returns S0 [N, H, d_k, d_v] fp32 and the list of lengths.
     """
-    lens = seq_lengths(wl, seed) if lengths is None else list(lengths)
-    per = [token_inputs(wl, L, device, seed, "seq", i) for i, L in enumerate(lens)]
+    all_lens = seq_lengths(wl, seed) if lengths is None else list(lengths)
+    idx = list(range(len(all_lens))) if indices is None else list(indices)
+    if lengths is None and not wl.varlen and indices is not None:
+        all_lens = [wl.T] * (max(idx) + 1 if idx else 0)
+    lens = [all_lens[i] for i in idx]
+    per = [token_inputs(wl, all_lens[i], device, seed, "seq", i) for i in idx]
     names = ("q", "k", "v", "alpha", "b", "w")
     if wl.varlen:
         out = {n: torch.cat([p[n] for p in per], 0) for n in names}
@@ -154,7 +168,7 @@ def chunk_inputs(wl: Workload, device="cpu", seed: int = 0, lengths: Optional[Li
     else:
         out = {n: torch.stack([p[n] for p in per], 0) for n in names}
         out["cu_seqlens"] = None
-    out["S0"] = initial_state(wl, len(lens), device, seed)
+    out["S0"] = initial_state(wl, len(lens), device, seed, indices=idx)
     out["lengths"] = lens
     return out
 
