@@ -73,7 +73,7 @@ constexpr uint32_t OFF_KT = OFF_XA + 2 * XA_BUF;   // 65536: 2 chunk buffers
 constexpr uint32_t OFF_U = OFF_KT + 2 * KT_BUF;    // 98304: 2 chunk buffers of v -> U = w (.) v
 constexpr uint32_t OFF_AL = OFF_U + 2 * 8192;      // 114688: alpha tiles (two channel blocks)
 constexpr uint32_t OFF_W = OFF_AL + 16384;         // 131072: w tile
-constexpr uint32_t OFF_TZP = OFF_W + 8192;         // 139264: [T ; 0 ; P0 ; P1], 64 rows each
+constexpr uint32_t OFF_TZP = OFF_W + 8192;         // 139264: two chunk buffers of [T ; P] (128 x 64 bf16)
 constexpr uint32_t OFF_SM = OFF_TZP + 32768;       // 172032: e^m S (128 x 64); its first 8 KB later holds Delta
 constexpr int LDF = 68;                            // row stride of the fp32 64 x 64 scratch
 constexpr uint32_t OFF_LS = OFF_SM + 16384;        // 188416: L (fp32); first 8 KB = decay-product scan
@@ -84,7 +84,7 @@ constexpr uint32_t SMEM_USED = OFF_BAR + 128;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for aligning the base
 constexpr uint32_t TMA_BYTES = 10 * 8192;          // q, k, b, alpha (2 boxes each), v, w
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TM_LP = 0, TM_DX = 64, TM_DA = 192, TM_DB = 320;  // D_a: two 64-column buffers
+constexpr uint32_t TM_LP = 0, TM_DX = 64, TM_DA = 192, TM_DU = 256, TM_DB = 320;
 constexpr uint64_t WAIT_NS = 2000000000ull;        // bounded waits: 2 s
 
 constexpr uint32_t ID_LP = idesc_bf16(128, 64, false, false);    // [A_m;Q_m] K_m^T
@@ -380,7 +380,8 @@ __device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, 
     tc_fence_after();
 
     // ------------------------------------------------------------ T = (I + L)^-1
-    uint8_t *pt = sm + OFF_TZP + 16384 + b * 8192;  // P of this chunk (64 x 64 bf16)
+    uint8_t *tp = sm + OFF_TZP + b * 16384;  // [T ; P] of this chunk
+    uint8_t *pt = tp + 8192;                 // P (64 x 64 bf16)
     {  // L (strict lower) -> fp32 scratch; P (inclusive lower) -> its bf16 tile
       float v[32];
       tmem_ld32(tl + TM_LP + 32 * khalf, v);
@@ -452,7 +453,7 @@ __device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, 
       store_16x8(Ts + (32 + 16 * mt) * LDF + 8 * nt, lane, d, -1.f);
     }
     group_sync(BAR_KEY, NKEY);
-    {  // T -> rows 0..63 of [T ; 0], bf16
+    {  // T -> rows 0..63 of [T ; P], bf16
       const int r = kt >> 2;
 #pragma unroll
       for (int y = 0; y < 2; ++y) {
@@ -460,50 +461,13 @@ __device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, 
         const float4 t0 = *reinterpret_cast<const float4 *>(&Ts[r * LDF + col]);
         const float4 t1 = *reinterpret_cast<const float4 *>(&Ts[r * LDF + col + 4]);
         const float e[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-        st_s128(sm + OFF_TZP + sw128(r, col), pack8(e));
+        st_s128(tp + sw128(r, col), pack8(e));
       }
     }
     fence_proxy_async();
     group_sync(BAR_KEY, NKEY);
 
-    // ------------------------------------------------------------ M3, M4: [T; 0] [A_m | U]
-    // (D_a buffer b is free: the state side finished chunk c-2 before it loaded chunk c)
-    if (kt == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        mma_bf16(x.tmem + TM_DX, sdesc_sw128(x.sb + OFF_TZP + 32 * k, 16, 1024),
-                 sdesc_sw128(x.sb + OFF_XA + b * XA_BUF + 2048 * k, XA_BLK, 1024), ID_KM128, k > 0 ? 1u : 0u);
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        mma_bf16(x.tmem + TM_DA + 64 * b, sdesc_sw128(x.sb + OFF_TZP + 32 * k, 16, 1024),
-                 sdesc_sw128(x.sb + OFF_U + b * 8192 + 2048 * k, 8192, 1024), ID_KM64, k > 0 ? 1u : 0u);
-      mma_commit(bar_addr(x, B_KMMA));
-    }
-    if (!group_wait(BAR_KEY, NKEY, bar_addr(x, B_KMMA), kphase)) return false;
-    kphase ^= 1;
-    tc_fence_after();
-
-    // ------------------------------------------------------------ -T A_m in place of A_m; hand over
-    if (quad < 2) {  // rows 0..63; warp group half khalf owns channel block khalf
-      const int row = 32 * quad + lane;
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        float v[32];
-        tmem_ld32(tl + TM_DX + 64 * khalf + 32 * part, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int y = 0; y < 4; ++y) {
-          float e[8];
-#pragma unroll
-          for (int t = 0; t < 8; ++t) e[t] = -v[8 * y + t];
-          st_s128(xa + khalf * XA_BLK + sw128(row, 32 * part + 8 * y), pack8(e));
-        }
-      }
-    }
-    tc_fence_before();
-    fence_proxy_async();
-    group_sync(BAR_KEY, NKEY);
+    // ------------------------------------------------------------ hand the chunk to the state side
     if (kt == 0) mbar_arrive(bar_addr(x, B_READY0 + b));
   }
   return true;
@@ -537,8 +501,21 @@ __device__ __forceinline__ bool state_side(const Ctx &x, float (&S)[64], __nv_bf
     }
     if (!group_wait(BAR_STATE, NSTATE, bar_addr(x, B_READY0 + b), (c >> 1) & 1, fail)) return false;
 
-    // ------------------------------------------------------------ e^m S -> shared (bf16)
-    {
+    // ------------------------------------------------------------ M3, M4: [T; P] [A_m | U]; e^m S -> shared
+    const uint32_t tpa = x.sb + OFF_TZP + b * 16384;  // [T ; P] of this chunk
+    if (st == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        mma_bf16(x.tmem + TM_DX, sdesc_sw128(tpa + 32 * k, 16, 1024),
+                 sdesc_sw128(x.sb + OFF_XA + b * XA_BUF + 2048 * k, XA_BLK, 1024), ID_KM128, k > 0 ? 1u : 0u);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        mma_bf16(x.tmem + TM_DU, sdesc_sw128(tpa + 32 * k, 16, 1024), sdesc_sw128(x.sb + OFF_U + b * 8192 + 2048 * k, 8192, 1024),
+                 ID_KM64, k > 0 ? 1u : 0u);
+      mma_commit(bar_addr(x, B_SMMA));
+    }
+    {  // rows 0..63 of the products are T A_m and T U (rows 64..127, P A_m and P U, are not used)
       const float em = s_em[c_me];
 #pragma unroll
       for (int y = 0; y < 8; ++y) {
@@ -548,31 +525,54 @@ __device__ __forceinline__ bool state_side(const Ctx &x, float (&S)[64], __nv_bf
         st_s128(sm + OFF_SM + sw128(c_me, 8 * y), pack8(e));
       }
     }
+    if (!group_wait(BAR_STATE, NSTATE, bar_addr(x, B_SMMA), sphase)) return false;
+    sphase ^= 1;
+    tc_fence_after();
+    if (quad < 2) {  // -T A_m in place of A_m (rows 0..63, both channel blocks)
+      const int row = 32 * quad + lane;
+#pragma unroll
+      for (int part = 0; part < 4; ++part) {
+        float v[32];
+        tmem_ld32(tl + TM_DX + 32 * part, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          float e[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) e[t] = -v[8 * y + t];
+          st_s128(sm + OFF_XA + b * XA_BUF + (part >> 1) * XA_BLK + sw128(row, 32 * (part & 1) + 8 * y), pack8(e));
+        }
+      }
+    }
+    tc_fence_before();
     fence_proxy_async();
     group_sync(BAR_STATE, NSTATE);
 
-    // ------------------------------------------------------------ M5: D_a += [-T A_m; Q_m] (e^m S)
+    // ------------------------------------------------------------ M5: D_a = [-T A_m; Q_m] (e^m S)
     if (st == 0) {
       tc_fence_after();
 #pragma unroll
       for (int k = 0; k < DK / 16; ++k)
-        mma_bf16(x.tmem + TM_DA + 64 * b,
+        mma_bf16(x.tmem + TM_DA,
                  sdesc_sw128(x.sb + OFF_XA + b * XA_BUF + (k >> 2) * XA_BLK + (k & 3) * 32, 16, 1024),
-                 sdesc_sw128(x.sb + OFF_SM + 2048 * k, 16384, 1024), ID_KM64, 1u);
+                 sdesc_sw128(x.sb + OFF_SM + 2048 * k, 16384, 1024), ID_KM64, k > 0 ? 1u : 0u);
       mma_commit(bar_addr(x, B_SMMA));
     }
     if (!group_wait(BAR_STATE, NSTATE, bar_addr(x, B_SMMA), sphase)) return false;
     sphase ^= 1;
     tc_fence_after();
 
-    // ------------------------------------------------------------ Delta -> shared (bf16)
+    // ------------------------------------------------------------ Delta = T U + D_a -> shared (bf16)
     if (quad < 2) {
       const int row = 32 * quad + lane;
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
-        float v[32];
-        tmem_ld32(tl + TM_DA + 64 * b + 32 * part, v);
+        float v[32], u[32];
+        tmem_ld32(tl + TM_DA + 32 * part, v);
+        tmem_ld32(tl + TM_DU + 32 * part, u);
         tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] += u[j];
 #pragma unroll
         for (int y = 0; y < 4; ++y) st_s128(sm + OFF_SM + sw128(row, 32 * part + 8 * y), pack8(&v[8 * y]));
       }
@@ -588,12 +588,12 @@ __device__ __forceinline__ bool state_side(const Ctx &x, float (&S)[64], __nv_bf
       for (int k = 0; k < 4; ++k)
         mma_bf16(x.tmem + TM_DB, sdesc_sw128(x.sb + OFF_KT + b * KT_BUF + 2048 * k, KT_BLK, 1024),
                  sdesc_sw128(x.sb + OFF_SM + 2048 * k, 8192, 1024), ID_MNMN, k > 0 ? 1u : 0u);
-      // A rows 64..127 = P of this chunk; rows 0..63 (zeros or the other P tile) only touch the
-      // already consumed Delta half of D_a
+      // A = [T ; P]: rows 64..127 add P Delta to Q S; rows 0..63 only touch the Delta half of D_a,
+      // which has been read out already
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        mma_bf16(x.tmem + TM_DA + 64 * b, sdesc_sw128(x.sb + OFF_TZP + 8192 + b * 8192 + 32 * k, 16, 1024),
-                 sdesc_sw128(x.sb + OFF_SM + 2048 * k, 8192, 1024), ID_KM64, 1u);
+        mma_bf16(x.tmem + TM_DA, sdesc_sw128(tpa + 32 * k, 16, 1024), sdesc_sw128(x.sb + OFF_SM + 2048 * k, 8192, 1024),
+                 ID_KM64, 1u);
       mma_commit(bar_addr(x, B_SMMA));
     }
     if (!group_wait(BAR_STATE, NSTATE, bar_addr(x, B_SMMA), sphase)) return false;
@@ -616,7 +616,7 @@ __device__ __forceinline__ bool state_side(const Ctx &x, float (&S)[64], __nv_bf
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
           float v[32];
-          tmem_ld32(tl + TM_DA + 64 * b + 32 * part, v);
+          tmem_ld32(tl + TM_DA + 32 * part, v);
           tmem_wait_ld();
           if (r < Cc) store_row32_bf16(o + ((size_t)(tok0 + r) * x.H + x.h) * (size_t)x.dv + x.j0 + 32 * part, v);
         }
@@ -661,8 +661,7 @@ __global__ void __launch_bounds__(NT, 1)
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
-  // the zero rows of [T ; 0] and the never-written upper blocks of T
-  for (int e = tid; e < 8192 / 16; e += NT) st_s128(x.sm + OFF_TZP + 8192 + 16 * e, make_uint4(0u, 0u, 0u, 0u));
+  // the never-written upper blocks of T
   float *Ts = reinterpret_cast<float *>(x.sm + OFF_TS);
   for (int e = tid; e < 64 * LDF; e += NT) Ts[e] = 0.f;
   fence_proxy_async();
