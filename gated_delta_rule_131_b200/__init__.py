@@ -51,6 +51,8 @@ def lib():
         L.gdn2_status_string.restype = ctypes.c_char_p
         L.gdn2_device_status.argtypes = [ci]
         L.gdn2_device_status.restype = ci
+        L.gdn2_selftest_bounded_wait.argtypes = [ci, vp]
+        L.gdn2_selftest_bounded_wait.restype = ci
         L.gdn2_launch_count.argtypes = []
         L.gdn2_launch_count.restype = ctypes.c_uint64
         _lib = L
@@ -65,6 +67,13 @@ def launch_count() -> int:
 def device_status(reset=False) -> int:
     """Sticky device-side status (GDN2_OK or GDN2_ERR_TIMEOUT); synchronises with the device."""
     return int(lib().gdn2_device_status(1 if reset else 0))
+
+
+def selftest_bounded_wait(limit_us=20000, stream=None):
+    """Run the bounded-wait self-test (a wait that nothing completes gives up after limit_us)."""
+    st = lib().gdn2_selftest_bounded_wait(int(limit_us), _stream(stream))
+    if st != GDN2_OK:
+        raise Gdn2Error(st, "gdn2_selftest_bounded_wait")
 
 
 def _ptr(t):

@@ -83,6 +83,7 @@ constexpr uint32_t OFF_BAR = OFF_SC + 2 * 3 * 128 * 4;  // 226304
 constexpr uint32_t SMEM_USED = OFF_BAR + 128;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for aligning the base
 constexpr uint32_t TMA_BYTES = 10 * 8192;          // q, k, b, alpha (2 boxes each), v, w
+constexpr uint32_t TMA_BYTES_HALF = 6 * 8192;     // cluster pair: own channel block of q, k, b, alpha; v, w
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_LP = 0, TM_DX = 64, TM_DA = 192, TM_DU = 256, TM_DB = 320;
 constexpr uint64_t WAIT_NS = 2000000000ull;        // bounded waits: 2 s
@@ -93,7 +94,12 @@ constexpr uint32_t ID_KM128 = idesc_bf16(128, 128, false, true); // same, N = 12
 constexpr uint32_t ID_MNMN = idesc_bf16(128, 64, true, true);    // K_m^T Delta
 
 // mbarriers (8 bytes each) at OFF_BAR
-enum { B_FULL0 = 0, B_FULL1, B_KMMA, B_SMMA, B_READY0, B_READY1, B_KBDONE, B_COUNT };
+enum {
+  B_FULL0 = 0, B_FULL1, B_KMMA, B_SMMA, B_READY0, B_READY1, B_KBDONE,
+  B_HALF0, B_HALF1,    // cluster pair: the peer's channel half of chunk buffer 0 / 1 has landed here
+  B_PFREE0, B_PFREE1,  // cluster pair: the peer's state side finished an even / odd chunk
+  B_COUNT
+};
 
 __device__ __forceinline__ uint4 ld_s128(const uint8_t *p) { return *reinterpret_cast<const uint4 *>(p); }
 __device__ __forceinline__ void st_s128(uint8_t *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
@@ -141,8 +147,9 @@ __device__ __forceinline__ void store_row32_bf16(__nv_bfloat16 *dst, const float
 
 // Decay-absorbed operands of one token row for 8 key channels, from the raw bf16 values already in
 // registers: A_m = b k f, Q_m = q f, K_m = k fi with f = e^{g_r - m}, fi = 1/f (zeros when !valid).
+template <int CL>
 __device__ __forceinline__ void row_factors(uint8_t *pa, uint8_t *pq, uint8_t *pk, uint4 rb, uint4 rq, uint4 rk,
-                                            bool valid, const float *f, const float *fi) {
+                                            bool valid, const float *f, const float *fi, uint32_t peer_delta) {
   uint4 wa = make_uint4(0u, 0u, 0u, 0u), wq = wa, wk = wa;
   if (valid) {
     float bb[8], qv[8], kv[8], ea[8], eq[8], ek[8];
@@ -162,6 +169,11 @@ __device__ __forceinline__ void row_factors(uint8_t *pa, uint8_t *pq, uint8_t *p
   st_s128(pa, wa);
   st_s128(pq, wq);
   st_s128(pk, wk);
+  if (CL == 2) {  // the same bytes at the same offsets in the peer CTA of the cluster
+    st_cluster_128(smem_u32(pa) + peer_delta, wa);
+    st_cluster_128(smem_u32(pq) + peer_delta, wq);
+    st_cluster_128(smem_u32(pk) + peer_delta, wk);
+  }
 }
 
 // D (16 x 8) = A (16 x K) B (K x 8) on the warp-level tensor-core path (mma.sync, tf32 operands
@@ -199,13 +211,16 @@ __device__ __forceinline__ void store_16x8(float *D, int lane, const float (&d)[
 struct Ctx {
   uint8_t *sm;
   uint32_t sb, tmem;
+  uint32_t rank, peer_delta;  // cluster pair: this CTA's rank; peer shared::cluster address minus own
   int H, dv, h, j0, nchunks, len;
   int64_t bos;
 };
 
 __device__ __forceinline__ uint32_t bar_addr(const Ctx &x, int i) { return x.sb + OFF_BAR + 8 * i; }
 
-// Issue the TMA loads of chunk `c` into chunk buffer c & 1 (one thread).
+// Issue the TMA loads of chunk `c` into chunk buffer c & 1 (one thread).  A cluster pair loads
+// only its own channel block of q, k, b, alpha; the peer fills the other block.
+template <int CL>
 __device__ __forceinline__ void issue_chunk_loads(const Ctx &x, int c, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
                                                   const CUtensorMap *tm_b, const CUtensorMap *tm_al,
                                                   const CUtensorMap *tm_v, const CUtensorMap *tm_w) {
@@ -213,9 +228,10 @@ __device__ __forceinline__ void issue_chunk_loads(const Ctx &x, int c, const CUt
   const int tok0 = (int)(x.bos + (int64_t)c * C);
   const uint32_t full = bar_addr(x, B_FULL0 + b);
   fence_proxy_async();
-  mbar_expect_tx(full, TMA_BYTES);
+  mbar_expect_tx(full, CL == 2 ? TMA_BYTES_HALF : TMA_BYTES);
 #pragma unroll
   for (int blk = 0; blk < 2; ++blk) {
+    if (CL == 2 && blk != (int)x.rank) continue;
     tma_load_3d(x.sb + OFF_XA + b * XA_BUF + blk * XA_BLK, tm_b, 64 * blk, x.h, tok0, full);         // b -> rows 0..63
     tma_load_3d(x.sb + OFF_XA + b * XA_BUF + blk * XA_BLK + 8192, tm_q, 64 * blk, x.h, tok0, full);  // q -> rows 64..127
     tma_load_3d(x.sb + OFF_KT + b * KT_BUF + blk * KT_BLK, tm_k, 64 * blk, x.h, tok0, full);
@@ -227,6 +243,7 @@ __device__ __forceinline__ void issue_chunk_loads(const Ctx &x, int c, const CUt
 
 // ==================================================================== key side (warps 4-11)
 // For each chunk: decay factors, L|P, T, [T; 0][A_m | U]; hands the chunk to the state side.
+template <int CL>
 __device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_b,
                          const CUtensorMap *tm_al, const CUtensorMap *tm_v, const CUtensorMap *tm_w) {
   uint8_t *sm = x.sm;
@@ -250,6 +267,7 @@ __device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, 
     if (!group_wait(BAR_KEY, NKEY, bar_addr(x, B_FULL0 + b), (c >> 1) & 1)) return false;
 
     // ------------------------------------------------------------ decay factors, operands in place
+    if (CL == 1)
     {
       // thread = 8 key channels (chunk x8 of channel block cb) x 4 tokens (group G = rows 4G..4G+3);
       // groups 0-7 hold tokens 0..31 (walk back to token 31), groups 8-15 tokens 32..63 (walk forward).
@@ -329,7 +347,7 @@ __device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, 
             if (r < Cc) run[t] *= al[t];
           }
           const uint32_t o = sw128(r, 8 * x8);
-          row_factors(pa0 + o, pa0 + 8192 + o, pk0 + o, rb[i], rq[i], rk[i], r < Cc, f, fi);
+          row_factors<1>(pa0 + o, pa0 + 8192 + o, pk0 + o, rb[i], rq[i], rk[i], r < Cc, f, fi, 0u);
         }
       } else {
 #pragma unroll
@@ -344,7 +362,7 @@ __device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, 
             fi[t] = fast_rcp(run[t]);
           }
           const uint32_t o = sw128(r, 8 * x8);
-          row_factors(pa0 + o, pa0 + 8192 + o, pk0 + o, rb[i], rq[i], rk[i], r < Cc, f, fi);
+          row_factors<1>(pa0 + o, pa0 + 8192 + o, pk0 + o, rb[i], rq[i], rk[i], r < Cc, f, fi, 0u);
         }
       }
 #pragma unroll
@@ -357,13 +375,133 @@ __device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, 
         st_s128(ub + sw128(ur, 16 * (kt & 3) + 8 * y), pack8(uu));
       }
     }
+    else {
+      // Cluster pair: this CTA forms only its own channel block cb (64 channels) and writes every
+      // result both here and into the peer.  thread = 8 channels (chunk x8) x 2 tokens (group G =
+      // rows 2G, 2G+1); groups 0-15 walk back to token 31, groups 16-31 walk forward.
+      const int x8 = kt & 7, G = kt >> 3, cb = (int)x.rank;
+      uint4 ra[2], rb[2], rq[2], rk[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const uint32_t o = sw128(2 * G + i, 8 * x8);
+        ra[i] = ld_s128(sm + OFF_AL + cb * 8192 + o);
+        rb[i] = ld_s128(xa + cb * XA_BLK + o);
+        rq[i] = ld_s128(xa + cb * XA_BLK + 8192 + o);
+        rk[i] = ld_s128(ktile + cb * KT_BLK + o);
+      }
+      const int ur = kt >> 2;  // U = w (.) v: token row ur, value columns 16 (kt & 3) .. +15
+      uint8_t *ub = sm + OFF_U + b * 8192;
+      uint4 rv[2], rw[2];
+#pragma unroll
+      for (int y = 0; y < 2; ++y) {
+        rv[y] = ld_s128(ub + sw128(ur, 16 * (kt & 3) + 8 * y));
+        rw[y] = ld_s128(sm + OFF_W + sw128(ur, 16 * (kt & 3) + 8 * y));
+      }
+      float gp[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) gp[t] = 1.f;
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+        if (2 * G + i < Cc) {
+          float al[8];
+          unpack8(ra[i], al);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) gp[t] *= al[t];
+        }
+      *reinterpret_cast<float4 *>(&scan[G * 64 + 8 * x8]) = make_float4(gp[0], gp[1], gp[2], gp[3]);
+      *reinterpret_cast<float4 *>(&scan[G * 64 + 8 * x8 + 4]) = make_float4(gp[4], gp[5], gp[6], gp[7]);
+      group_sync(BAR_KEY, NKEY);
+      if (kt < 64) {  // per channel: products between each group and token 31, in place of the group products
+        float p[32];
+#pragma unroll
+        for (int g = 0; g < 32; ++g) p[g] = scan[g * 64 + kt];
+        float acc = 1.f;
+#pragma unroll
+        for (int g = 15; g >= 0; --g) {
+          scan[g * 64 + kt] = acc;
+          acc *= p[g];
+        }
+        const float em = acc;
+        acc = 1.f;
+#pragma unroll
+        for (int g = 16; g < 32; ++g) {
+          scan[g * 64 + kt] = acc;
+          acc *= p[g];
+        }
+        const int ch = 64 * cb + kt;
+        s_em[ch] = em;
+        s_egcm[ch] = acc;
+        s_egc[ch] = em * acc;
+        st_cluster_f32(smem_u32(&s_em[ch]) + x.peer_delta, em);
+        st_cluster_f32(smem_u32(&s_egcm[ch]) + x.peer_delta, acc);
+        st_cluster_f32(smem_u32(&s_egc[ch]) + x.peer_delta, em * acc);
+      }
+      group_sync(BAR_KEY, NKEY);
+      float run[8];
+      {
+        const float4 p0 = *reinterpret_cast<const float4 *>(&scan[G * 64 + 8 * x8]);
+        const float4 p1 = *reinterpret_cast<const float4 *>(&scan[G * 64 + 8 * x8 + 4]);
+        run[0] = p0.x; run[1] = p0.y; run[2] = p0.z; run[3] = p0.w;
+        run[4] = p1.x; run[5] = p1.y; run[6] = p1.z; run[7] = p1.w;
+      }
+      uint8_t *pa0 = xa + cb * XA_BLK, *pk0 = ktile + cb * KT_BLK;
+      if (G < 16) {
+#pragma unroll
+        for (int i = 1; i >= 0; --i) {  // run = prod_{r < s <= 31} alpha_s
+          const int r = 2 * G + i;
+          float al[8], f[8], fi[8];
+          unpack8(ra[i], al);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            fi[t] = run[t];
+            f[t] = fast_rcp(run[t]);
+            if (r < Cc) run[t] *= al[t];
+          }
+          const uint32_t o = sw128(r, 8 * x8);
+          row_factors<2>(pa0 + o, pa0 + 8192 + o, pk0 + o, rb[i], rq[i], rk[i], r < Cc, f, fi, x.peer_delta);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {  // run = prod_{32 <= s <= r} alpha_s
+          const int r = 2 * G + i;
+          float al[8], f[8], fi[8];
+          unpack8(ra[i], al);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            if (r < Cc) run[t] *= al[t];
+            f[t] = run[t];
+            fi[t] = fast_rcp(run[t]);
+          }
+          const uint32_t o = sw128(r, 8 * x8);
+          row_factors<2>(pa0 + o, pa0 + 8192 + o, pk0 + o, rb[i], rq[i], rk[i], r < Cc, f, fi, x.peer_delta);
+        }
+      }
+#pragma unroll
+      for (int y = 0; y < 2; ++y) {
+        float vv[8], ww[8], uu[8];
+        unpack8(rv[y], vv);
+        unpack8(rw[y], ww);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) uu[t] = (ur < Cc) ? vv[t] * ww[t] : 0.f;
+        st_s128(ub + sw128(ur, 16 * (kt & 3) + 8 * y), pack8(uu));
+      }
+      // publish this thread's share of the channel half to the peer
+      fence_proxy_async_cluster();
+      mbar_arrive_remote(bar_addr(x, B_HALF0 + b) + x.peer_delta);
+    }
     fence_proxy_async();
     group_sync(BAR_KEY, NKEY);
 
     // ------------------------------------------------------------ M1: [L; P] = [A_m; Q_m] K_m^T
     // (the alpha and w tiles of chunk c are consumed: the state side may now load chunk c+1)
+    bool kfail = false;
     if (kt == 0) {
       mbar_arrive(bar_addr(x, B_KBDONE));
+      if (CL == 2) {
+        // the peer's channel half of this chunk
+        kfail = !mbar_wait_bounded_cluster(bar_addr(x, B_HALF0 + b), (c >> 1) & 1, WAIT_NS);
+        fence_proxy_async();
+      }
       tc_fence_after();
 #pragma unroll
       for (int k = 0; k < DK / 16; ++k) {
@@ -374,7 +512,7 @@ __device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, 
       }
       mma_commit(bar_addr(x, B_KMMA));
     }
-    const bool fail = false;
+    const bool fail = kfail;
     if (!group_wait(BAR_KEY, NKEY, bar_addr(x, B_KMMA), kphase, fail)) return false;
     kphase ^= 1;
     tc_fence_after();
@@ -468,13 +606,16 @@ __device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, 
     group_sync(BAR_KEY, NKEY);
 
     // ------------------------------------------------------------ hand the chunk to the state side
-    if (kt == 0) mbar_arrive(bar_addr(x, B_READY0 + b));
+    if (kt == 0) {
+      mbar_arrive(bar_addr(x, B_READY0 + b));
+    }
   }
   return true;
 }
 
 // ==================================================================== state side (warps 0-3)
 // Holds the fp32 state slice (thread = key channel x 64 value columns) and runs the serial chain.
+template <int CL>
 __device__ __forceinline__ bool state_side(const Ctx &x, float (&S)[64], __nv_bfloat16 *o, const CUtensorMap *tm_q,
                                            const CUtensorMap *tm_k, const CUtensorMap *tm_b, const CUtensorMap *tm_al,
                                            const CUtensorMap *tm_v, const CUtensorMap *tm_w) {
@@ -486,7 +627,9 @@ __device__ __forceinline__ bool state_side(const Ctx &x, float (&S)[64], __nv_bf
   // The state side's thread 0 is also the load producer.  Chunk c+1 goes into buffer (c+1)&1,
   // last used by chunk c-1, which this side has finished; it waits only until the key side has
   // read the single-buffered alpha and w tiles of chunk c.
-  if (st == 0 && x.nchunks > 0) issue_chunk_loads(x, 0, tm_q, tm_k, tm_b, tm_al, tm_v, tm_w);
+  // In a cluster pair the peer also writes into buffer (c+1)&1, so chunk c+1 is loaded only after
+  // the peer's state side has finished chunk c-1 too.
+  if (st == 0 && x.nchunks > 0) issue_chunk_loads<CL>(x, 0, tm_q, tm_k, tm_b, tm_al, tm_v, tm_w);
 
   for (int c = 0; c < x.nchunks; ++c) {
     const int b = c & 1;
@@ -495,9 +638,14 @@ __device__ __forceinline__ bool state_side(const Ctx &x, float (&S)[64], __nv_bf
     const int tok0 = (int)(x.bos + (int64_t)c * C);
 
     bool fail = false;
+    if (st == 0 && CL == 2 && c >= 1) {  // tell the peer that chunk c-1 is done here
+      mbar_arrive_remote(bar_addr(x, B_PFREE0 + ((c - 1) & 1)) + x.peer_delta);
+    }
     if (st == 0 && c + 1 < x.nchunks) {
-      fail = !mbar_wait_bounded(bar_addr(x, B_KBDONE), c & 1, WAIT_NS);
-      if (!fail) issue_chunk_loads(x, c + 1, tm_q, tm_k, tm_b, tm_al, tm_v, tm_w);
+      if (CL == 2 && c >= 1)
+        fail = !mbar_wait_bounded_cluster(bar_addr(x, B_PFREE0 + ((c - 1) & 1)), ((c - 1) >> 1) & 1, WAIT_NS);
+      if (!fail) fail = !mbar_wait_bounded(bar_addr(x, B_KBDONE), c & 1, WAIT_NS);
+      if (!fail) issue_chunk_loads<CL>(x, c + 1, tm_q, tm_k, tm_b, tm_al, tm_v, tm_w);
     }
     if (!group_wait(BAR_STATE, NSTATE, bar_addr(x, B_READY0 + b), (c >> 1) & 1, fail)) return false;
 
@@ -628,6 +776,7 @@ __device__ __forceinline__ bool state_side(const Ctx &x, float (&S)[64], __nv_bf
   return true;
 }
 
+template <int CL>
 __global__ void __launch_bounds__(NT, 1)
     chunk_fwd_tc_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_b,
@@ -651,8 +800,10 @@ __global__ void __launch_bounds__(NT, 1)
   seq_span(a, n, x.bos, x.len);
   x.nchunks = (x.len + C - 1) / C;
 
+  x.rank = (CL == 2) ? cluster_ctarank() : 0u;
+  x.peer_delta = (CL == 2) ? mapa(x.sb, x.rank ^ 1u) - x.sb : 0u;
   if (tid == 0) {
-    for (int i = 0; i < B_COUNT; ++i) mbar_init(x.sb + OFF_BAR + 8 * i, 1);
+    for (int i = 0; i < B_COUNT; ++i) mbar_init(x.sb + OFF_BAR + 8 * i, (i == B_HALF0 || i == B_HALF1) ? NKEY : 1);
     fence_mbar_init();
     prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_b);
     prefetch_tmap(&tm_al); prefetch_tmap(&tm_v); prefetch_tmap(&tm_w);
@@ -669,6 +820,7 @@ __global__ void __launch_bounds__(NT, 1)
   __syncthreads();
   tc_fence_after();
   x.tmem = *tmem_slot;
+  if (CL == 2) cluster_sync();  // both CTAs' barriers are initialised before any remote arrive
 
   bool ok;
   if (warp < 4) {
@@ -685,22 +837,39 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
       for (int y = 0; y < 64; ++y) S[y] = 0.f;
     }
-    ok = state_side(x, S, reinterpret_cast<__nv_bfloat16 *>(a.o), &tm_q, &tm_k, &tm_b, &tm_al, &tm_v, &tm_w);
+    ok = state_side<CL>(x, S, reinterpret_cast<__nv_bfloat16 *>(a.o), &tm_q, &tm_k, &tm_b, &tm_al, &tm_v, &tm_w);
     if (ok && a.ST) {
 #pragma unroll
       for (int y = 0; y < 16; ++y)
         reinterpret_cast<float4 *>(a.ST + s_off)[y] = make_float4(S[4 * y], S[4 * y + 1], S[4 * y + 2], S[4 * y + 3]);
     }
   } else {
-    ok = key_side(x, &tm_q, &tm_k, &tm_b, &tm_al, &tm_v, &tm_w);
+    ok = key_side<CL>(x, &tm_q, &tm_k, &tm_b, &tm_al, &tm_v, &tm_w);
   }
   if (!ok && (tid == 0 || tid == NSTATE)) atomicExch(&g_device_status, 4);
   tc_fence_before();
   __syncthreads();
+  if (CL == 2) cluster_sync();  // no CTA leaves while its peer may still write into it
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(x.tmem, TMEM_COLS);
   }
+}
+
+// Self-test of the bounded-wait path: waits on an mbarrier that nothing ever arrives on, gives up
+// after `limit_ns`, and records GDN2_ERR_TIMEOUT exactly like the chunk kernel does.  No fault, trap
+// or endless loop is involved; the context stays usable afterwards.
+__global__ void bounded_wait_probe_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const bool ok = mbar_wait_bounded(b, 0, limit_ns);
+  const bool any_timeout = __syncthreads_or(!ok);
+  if (any_timeout && threadIdx.x == 0) atomicExch(&g_device_status, 4);
 }
 
 // ------------------------------------------------------------------ host side: tensor maps
@@ -735,6 +904,12 @@ bool make_map(CUtensorMap *m, const void *base, long long tokens, int H, int D) 
 
 }  // namespace
 
+cudaError_t launch_bounded_wait_probe(uint64_t limit_ns, cudaStream_t stream) {
+  note_launch();
+  bounded_wait_probe_kernel<<<1, 32, 0, stream>>>(limit_ns);
+  return cudaGetLastError();
+}
+
 bool chunk_tc_supported(const ChunkArgs &a, bool bf16) { return bf16 && a.dk == DK && a.dv % NV == 0; }
 
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream) {
@@ -749,10 +924,29 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream) {
       !make_map(&mb, a.b, tokens, a.H, DK) || !make_map(&mal, a.alpha, tokens, a.H, DK) ||
       !make_map(&mv, a.v, tokens, a.H, a.dv) || !make_map(&mw, a.w, tokens, a.H, a.dv))
     return cudaErrorInvalidValue;
-  cudaError_t err = cudaFuncSetAttribute(chunk_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  const bool pair = (a.dv / NV) % 2 == 0;  // the two value slices of a head share the factor work
+  cudaError_t err = cudaFuncSetAttribute(pair ? chunk_fwd_tc_kernel<2> : chunk_fwd_tc_kernel<1>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (err != cudaSuccess) return err;
   note_launch();
-  chunk_fwd_tc_kernel<<<(unsigned)blocks, NT, SMEM_BYTES, stream>>>(a, mq, mk, mb, mal, mv, mw);
+  if (!pair) {
+    chunk_fwd_tc_kernel<1><<<(unsigned)blocks, NT, SMEM_BYTES, stream>>>(a, mq, mk, mb, mal, mv, mw);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks, 1, 1);
+  cfg.blockDim = dim3(NT, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, chunk_fwd_tc_kernel<2>, a, mq, mk, mb, mal, mv, mw);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 

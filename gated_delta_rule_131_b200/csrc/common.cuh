@@ -58,6 +58,7 @@ void note_launch();
 cudaError_t launch_chunk_simt(const ChunkArgs &a, bool bf16, cudaStream_t stream);
 bool chunk_tc_supported(const ChunkArgs &a, bool bf16);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream);
+cudaError_t launch_bounded_wait_probe(uint64_t limit_ns, cudaStream_t stream);
 // Reads (and optionally clears) the device-side status word that bounded waits set.
 cudaError_t read_device_status(int *status, bool reset);
 cudaError_t launch_decode(const DecodeArgs &a, bool bf16, cudaStream_t stream);

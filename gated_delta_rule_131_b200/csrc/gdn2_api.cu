@@ -46,6 +46,12 @@ const char *gdn2_status_string(gdn2_status s) {
 
 uint64_t gdn2_launch_count(void) { return gdn2::g_launches.load(std::memory_order_relaxed); }
 
+gdn2_status gdn2_selftest_bounded_wait(int limit_us, gdn2_stream_t stream) {
+  if (limit_us <= 0 || limit_us > 10000000) return GDN2_ERR_INVALID_ARG;
+  const cudaError_t err = gdn2::launch_bounded_wait_probe((uint64_t)limit_us * 1000ull, (cudaStream_t)stream);
+  return err == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+}
+
 gdn2_status gdn2_device_status(int reset) {
   int st = 0;
   if (gdn2::read_device_status(&st, reset != 0) != cudaSuccess) return GDN2_ERR_CUDA;

@@ -123,6 +123,16 @@ GDN2_API const char *gdn2_status_string(gdn2_status status);
  */
 GDN2_API gdn2_status gdn2_device_status(int reset);
 
+/*
+ * gdn2_selftest_bounded_wait -- exercises the failure path of the bounded device-side waits.
+ * Launches one CTA that waits on a barrier nothing arrives on; after `limit_us` microseconds
+ * (1 .. 10,000,000) the wait gives up and records GDN2_ERR_TIMEOUT in the status word that
+ * gdn2_device_status() reads -- the same path the tensor-core kernels take.  Nothing faults and
+ * the context stays usable.  Asynchronous on `stream`.  Returns GDN2_OK, GDN2_ERR_INVALID_ARG
+ * for a limit out of range, or GDN2_ERR_CUDA if the launch failed.
+ */
+GDN2_API gdn2_status gdn2_selftest_bounded_wait(int limit_us, gdn2_stream_t stream);
+
 /* Number of kernel launches this library has issued in this process (all calls, all threads). */
 GDN2_API uint64_t gdn2_launch_count(void);
 

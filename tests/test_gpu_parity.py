@@ -189,3 +189,19 @@ def test_decode_continues_chunk_fwd(g):
     o_ref, S_ref = oracle.recurrent(*[np64(d[n]) for n in TOK], S0=np64(d["S0"]))
     check_bf16(np64(torch.cat(outs, 1)), o_ref, "o")
     check_bf16(np64(S), S_ref, "S")
+
+
+# ------------------------------------------------------------------ failure path of the bounded waits
+
+def test_bounded_wait_timeout_is_reported_and_context_survives(g):
+    """A device wait that nothing completes gives up after its limit and records GDN2_ERR_TIMEOUT;
+    no fault, and the context keeps working (a chunk_fwd afterwards still matches the oracle)."""
+    torch.cuda.synchronize()
+    assert g.device_status(reset=True) == g.GDN2_OK
+    g.selftest_bounded_wait(limit_us=20000)
+    torch.cuda.synchronize()
+    assert g.device_status(reset=True) == g.GDN2_ERR_TIMEOUT
+    assert g.device_status() == g.GDN2_OK
+    wl = W.Workload("after_timeout", B=1, T=100, H=2, dk=128, dv=128)
+    run_case(g, wl, seed=21)
+    assert g.device_status() == g.GDN2_OK
