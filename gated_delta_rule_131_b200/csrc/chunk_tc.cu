@@ -485,9 +485,9 @@ __device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, 
         for (int t = 0; t < 8; ++t) uu[t] = (ur < Cc) ? vv[t] * ww[t] : 0.f;
         st_s128(ub + sw128(ur, 16 * (kt & 3) + 8 * y), pack8(uu));
       }
-      // publish this thread's share of the channel half to the peer
+      // make this thread's DSMEM writes visible to the peer's tensor-core (async) proxy; the key
+      // leader publishes the whole half after the group barrier below
       fence_proxy_async_cluster();
-      mbar_arrive_remote(bar_addr(x, B_HALF0 + b) + x.peer_delta);
     }
     fence_proxy_async();
     group_sync(BAR_KEY, NKEY);
@@ -498,6 +498,9 @@ __device__ __forceinline__ bool key_side(const Ctx &x, const CUtensorMap *tm_q, 
     if (kt == 0) {
       mbar_arrive(bar_addr(x, B_KBDONE));
       if (CL == 2) {
+        // one release at cluster scope covers every key thread's DSMEM writes (ordered before it by
+        // the group barrier)
+        mbar_arrive_remote(bar_addr(x, B_HALF0 + b) + x.peer_delta);
         // the peer's channel half of this chunk
         kfail = !mbar_wait_bounded_cluster(bar_addr(x, B_HALF0 + b), (c >> 1) & 1, WAIT_NS);
         fence_proxy_async();
@@ -803,7 +806,7 @@ __global__ void __launch_bounds__(NT, 1)
   x.rank = (CL == 2) ? cluster_ctarank() : 0u;
   x.peer_delta = (CL == 2) ? mapa(x.sb, x.rank ^ 1u) - x.sb : 0u;
   if (tid == 0) {
-    for (int i = 0; i < B_COUNT; ++i) mbar_init(x.sb + OFF_BAR + 8 * i, (i == B_HALF0 || i == B_HALF1) ? NKEY : 1);
+    for (int i = 0; i < B_COUNT; ++i) mbar_init(x.sb + OFF_BAR + 8 * i, 1);
     fence_mbar_init();
     prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_b);
     prefetch_tmap(&tm_al); prefetch_tmap(&tm_v); prefetch_tmap(&tm_w);
