@@ -54,9 +54,16 @@ def lib():
         L.gdn2_selftest_bounded_wait.argtypes = [ci, vp]
         L.gdn2_selftest_bounded_wait.restype = ci
         L.gdn2_launch_count.argtypes = []
+        L.gdn2_chunk_fwd_workspace_bytes.argtypes = [ci] * 7 + [ci]
+        L.gdn2_chunk_fwd_workspace_bytes.restype = ctypes.c_size_t
         L.gdn2_launch_count.restype = ctypes.c_uint64
         _lib = L
     return _lib
+
+
+def chunk_fwd_workspace_bytes(B, T, H, dk, dv, packed=False, dtype=torch.bfloat16, chunk=64) -> int:
+    """Device bytes ``chunk_fwd`` takes from the library's pool for this shape (0: none)."""
+    return int(lib().gdn2_chunk_fwd_workspace_bytes(B, T, H, dk, dv, chunk, 1 if packed else 0, _DTYPES[dtype]))
 
 
 def launch_count() -> int:

@@ -54,6 +54,10 @@ cudaError_t read_device_status(int *status, bool reset) {
   return err;
 }
 
+cudaError_t device_status_word(int **ptr) {
+  return cudaGetSymbolAddress(reinterpret_cast<void **>(ptr), g_device_status);
+}
+
 namespace {
 
 using namespace ptx;

@@ -1,0 +1,985 @@
+// Chunkwise WY forward of the Gated Delta Rule-2 as two tensor-core kernels
+// (bf16 inputs, d_k = 128, fp32 state and accumulation), split where the
+// dependence on the state begins:
+//
+//   wy_factor_kernel   one CTA per (chunk, head), all chunks at once: the
+//                      decay-absorbed erase factors, [L; P], T = (I + L)^-1, and
+//                      from them the chunk's state transition and output maps,
+//                      stored to a workspace record;
+//   state_pass_kernel  one CTA per (sequence, head, 64 value columns): walks the
+//                      chunks of its sequence in order and carries S in fp32.
+//
+// Per chunk of C = 64 tokens (r, i index tokens, c a key channel, m the running
+// log-decay at token 31 of the chunk, g_r the running log-decay at r):
+//   f_r     = exp(g_r - m)  per key channel (bounded by the decay over 32 tokens either way)
+//   A_m     = (b (.) k) (.) f,  Q_m = q (.) f,  K_m = k (.) 1/f
+//   [L; P]  = [A_m; Q_m] K_m^T              L strictly, P inclusively lower triangular
+//   T       = (I + L)^-1                    fp32 blocked forward substitution
+//   W       = -T A_m
+// With S the state entering the chunk and U = w (.) v, the WY form reads
+//   Delta   = T U + W Diag(e^m) S
+//   O       = Q_m Diag(e^m) S + P Delta
+//   S_next  = Diag(e^{g_C}) S + Diag(e^{g_C - m}) K_m^T Delta,
+// which the state pass evaluates as
+//   S_next  = Diag(e^{g_C}) S + Mt S + Nt U,   O = Qt S + Pt U,   with
+//   Mt = Diag(e^{g_C-m}) K_m^T W Diag(e^m)   (d_k x d_k)   Nt = Diag(e^{g_C-m}) K_m^T T   (d_k x C)
+//   Qt = (Q_m + P W) Diag(e^m)               (C x d_k)     Pt = P T                       (C x C)
+// so its serial chain per chunk is one tensor-core pass over S.  A record holds
+// Mt, Nt, Qt, Pt (bf16) and e^{g_C} (fp32).
+// The decay-absorbed asymmetric erase factors follow the block formulation of
+// "Gated DeltaNet-2: Separando Borrado y Escritura en la Atención Lineal"
+// (needhelp.icu), "Innovaciones Técnicas", item 1; the update itself is the
+// per-token rule of "NVIDIA AIがGated DeltaNet-2を発表" (ai.warp-studio.com),
+// "Gated DeltaNet-2の核心" (decay first, key-side erase gate b, value-side
+// write gate w, o_t = S_t^T q_t).
+//
+// Every operand tile is a 64-column bf16 tile in the 128-byte-swizzled layout
+// that TMA writes and tcgen05.mma reads, in shared memory and in the workspace
+// alike, so records move between the kernels as whole TMA boxes.
+// Precondition of the factorisation: per key channel, the decay accumulated
+// over any 32 consecutive tokens of a chunk stays above about e^-80 (the fp32
+// range); every workload here is far inside it.
+#include <cuda.h>
+
+#include <climits>
+#include <cstring>
+
+#include "common.cuh"
+#include "tc_ptx.cuh"
+
+namespace gdn2 {
+
+namespace {
+
+using namespace ptx;
+
+constexpr int C = 64, DK = 128, NV = 64;
+constexpr int LDF = 68;                      // row stride of the fp32 64 x 64 scratch
+constexpr uint64_t WAIT_NS = 2000000000ull;  // bounded waits: 2 s
+
+constexpr uint32_t XA_BLK = 16384;  // [A_m ; Q_m]: 128 rows x 64 channels (one channel block)
+constexpr uint32_t KT_BLK = 8192;   // K_m: 64 rows x 64 channels
+
+// workspace record of one (chunk, head), every tile K-major for the state pass's A operands:
+// Mt 128 x 128 (two 128-row tiles), Nt 128 x 64, Qt 64 x 128 (two 64-row tiles), Pt 64 x 64, e^{g_C}
+constexpr uint32_t REC_M = 32768, REC_N = 16384, REC_Q = 16384, REC_P = 8192, REC_G = 512;
+
+constexpr uint32_t ID_LP = idesc_bf16(128, 64, false, false);    // [A_m;Q_m] K_m^T
+constexpr uint32_t ID_KM64 = idesc_bf16(128, 64, false, true);   // K-major A, MN-major B, N = 64
+constexpr uint32_t ID_KM128 = idesc_bf16(128, 128, false, true); // same, N = 128
+constexpr uint32_t ID_MN64 = idesc_bf16(128, 64, true, true);    // MN-major A and B, N = 64
+constexpr uint32_t ID_MN128 = idesc_bf16(128, 128, true, true);  // same, N = 128
+
+__device__ __forceinline__ uint4 ld_s128(const uint8_t *p) { return *reinterpret_cast<const uint4 *>(p); }
+__device__ __forceinline__ void st_s128(uint8_t *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
+__device__ __forceinline__ uint4 pack8(const float *e) {
+  return make_uint4(f2_to_bf2(e[0], e[1]), f2_to_bf2(e[2], e[3]), f2_to_bf2(e[4], e[5]), f2_to_bf2(e[6], e[7]));
+}
+__device__ __forceinline__ void unpack8(uint4 u, float *e) {
+  float2 t = bf2_to_f2(u.x); e[0] = t.x; e[1] = t.y;
+  t = bf2_to_f2(u.y); e[2] = t.x; e[3] = t.y;
+  t = bf2_to_f2(u.z); e[4] = t.x; e[5] = t.y;
+  t = bf2_to_f2(u.w); e[6] = t.x; e[7] = t.y;
+}
+__device__ __forceinline__ float fast_rcp(float x) { return __fdividef(1.f, x); }
+
+__device__ __forceinline__ void group_sync(int id, int count) {
+  asm volatile("barrier.cta.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Barrier of one warp group that also ORs a predicate over its threads.
+__device__ __forceinline__ bool group_or(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// Every thread of a warp group waits (bounded); the group agrees on the outcome.
+__device__ __forceinline__ bool group_wait(int id, int count, uint32_t bar, uint32_t parity, bool fail = false) {
+  const bool ok = mbar_wait_bounded(bar, parity, WAIT_NS);
+  return !group_or(id, count, fail || !ok);
+}
+
+// D (16 x 8) = A (16 x K) B (K x 8) on the warp-level tensor-core path (mma.sync, tf32 operands
+// rounded from fp32, fp32 accumulate).  A points at element (0, 0) of a row-major fp32 block with
+// row stride LDF, B likewise.  Lane 4 g + t holds D rows g and g + 8, columns 2t and 2t + 1.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+template <int K>
+__device__ __forceinline__ void mma_tf32_16x8(const float *A, const float *B, int lane, float (&d)[4]) {
+  const int g = lane >> 2, t = lane & 3;
+  d[0] = d[1] = d[2] = d[3] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < K; kk += 8) {
+    const uint32_t a0 = to_tf32(A[g * LDF + kk + t]), a1 = to_tf32(A[(g + 8) * LDF + kk + t]);
+    const uint32_t a2 = to_tf32(A[g * LDF + kk + t + 4]), a3 = to_tf32(A[(g + 8) * LDF + kk + t + 4]);
+    const uint32_t b0 = to_tf32(B[(kk + t) * LDF + g]), b1 = to_tf32(B[(kk + t + 4) * LDF + g]);
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+}
+// Store a 16 x 8 tile (times `scale`) into a row-major fp32 block with row stride LDF.
+__device__ __forceinline__ void store_16x8(float *D, int lane, const float (&d)[4], float scale) {
+  const int g = lane >> 2, t = lane & 3;
+  *reinterpret_cast<float2 *>(&D[g * LDF + 2 * t]) = make_float2(scale * d[0], scale * d[1]);
+  *reinterpret_cast<float2 *>(&D[(g + 8) * LDF + 2 * t]) = make_float2(scale * d[2], scale * d[3]);
+}
+
+// Decay-absorbed operands of one token row for 8 key channels, from the raw bf16 values already in
+// registers: A_m = b k f (rows 0..63 of the [A_m ; Q_m] block), Q_m = q f (rows 64..127), K_m = k fi,
+// with f = e^{g_r - m}, fi = 1/f; zeros when the row is past the sequence.
+__device__ __forceinline__ void row_factors(uint8_t *pa, uint8_t *pk, uint32_t o, uint4 rb, uint4 rq, uint4 rk,
+                                            bool valid, const float *f, const float *fi) {
+  uint4 wa = make_uint4(0u, 0u, 0u, 0u), wq = wa, wk = wa;
+  if (valid) {
+    float bb[8], qv[8], kv[8], ea[8], eq[8], ek[8];
+    unpack8(rb, bb);
+    unpack8(rq, qv);
+    unpack8(rk, kv);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      ea[t] = bb[t] * kv[t] * f[t];
+      eq[t] = qv[t] * f[t];
+      ek[t] = kv[t] * fi[t];
+    }
+    wa = pack8(ea);
+    wq = pack8(eq);
+    wk = pack8(ek);
+  }
+  st_s128(pa + o, wa);
+  st_s128(pa + 8192 + o, wq);
+  st_s128(pk + o, wk);
+}
+
+// Sequence n holding global chunk `gidx`, from the chunk offsets of a packed batch (coff[n] = first
+// global chunk of sequence n; empty sequences own no chunk).  Requires coff[0] <= gidx < coff[N].
+__device__ __forceinline__ int seq_of_chunk(const int32_t *coff, int N, int gidx) {
+  int lo = 0, hi = N;
+  while (lo < hi) {  // largest n with coff[n] <= gidx
+    const int mid = (lo + hi + 1) >> 1;
+    if (coff[mid] <= gidx) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// ==================================================================== kernel 1: WY factors
+namespace wy {
+constexpr int NT = 256;
+// shared memory (two CTAs per SM); regions are reused once their first contents are dead
+constexpr uint32_t OFF_XA = 0;                       // [A_m ; Q_m], two channel blocks -> Qt in rows 0..63
+constexpr uint32_t OFF_KT = OFF_XA + 2 * XA_BLK;     // 32768: K_m, two channel blocks -> Mt tile 0
+constexpr uint32_t OFF_TP = OFF_KT + 2 * KT_BLK;     // 49152: [T ; P] -> Nt; decay-product scan during the factors
+constexpr uint32_t OFF_AL = OFF_TP + 16384;          // 65536: alpha tiles -> L (fp32) -> W (two 64-channel tiles) -> Mt tile 1
+constexpr uint32_t OFF_TS = OFF_AL + 64 * LDF * 4;   // 82944: T (fp32) -> Pt
+constexpr uint32_t OFF_SC = OFF_TS + 64 * LDF * 4;   // 100352: e^m, e^{g_C-m}, e^{g_C}
+constexpr uint32_t OFF_BAR = OFF_SC + 3 * 128 * 4;   // 101888: FULL, MMA
+constexpr uint32_t SMEM_USED = OFF_BAR + 32;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
+constexpr uint32_t TMA_BYTES = 8 * 8192;             // q, k, b, alpha: two channel blocks each
+constexpr uint32_t TMEM_COLS = 256;
+static_assert(2 * (SMEM_BYTES + 1024) <= 232448, "two CTAs per SM");
+static_assert(OFF_AL % 1024 == 0 && OFF_TS % 1024 == 0, "MMA operand tiles are 1024-aligned");
+}  // namespace wy
+
+struct WyParams {
+  int *status;     // device status word: GDN2_ERR_TIMEOUT (4) when a bounded wait gave up
+  int N;           // sequences
+  int nc;          // chunks per sequence of a dense batch
+  int64_t tokens;  // rows of the token tensors
+  const int32_t *coff;  // packed batch: chunk offsets [N+1]; dense: nullptr
+  float *g;             // workspace e^{g_C} [records][128]
+};
+
+__global__ void __launch_bounds__(wy::NT, 2)
+    wy_factor_kernel(const ChunkArgs a, const WyParams p, const __grid_constant__ CUtensorMap tm_q,
+                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_b,
+                     const __grid_constant__ CUtensorMap tm_al, const __grid_constant__ CUtensorMap tm_wm,
+                     const __grid_constant__ CUtensorMap tm_wn, const __grid_constant__ CUtensorMap tm_wq,
+                     const __grid_constant__ CUtensorMap tm_wp) {
+  using namespace wy;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, quad = warp & 3, khalf = warp >> 2;
+
+  const int rec = blockIdx.x;  // global chunk * H + head
+  const int h = rec % a.H, gidx = rec / a.H;
+  int n, c;
+  if (p.coff) {
+    if (gidx >= p.coff[p.N]) return;  // beyond the chunks of the packed batch (uniform per CTA)
+    n = seq_of_chunk(p.coff, p.N, gidx);
+    c = gidx - p.coff[n];
+  } else {
+    n = gidx / p.nc;
+    c = gidx % p.nc;
+  }
+  int64_t bos;
+  int len;
+  seq_span(a, n, bos, len);
+  const int Cc = min(C, len - c * C);
+  const int tok0 = (int)(bos + (int64_t)c * C);
+
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 16);
+  const uint32_t bar_full = sb + OFF_BAR, bar_mma = sb + OFF_BAR + 8;
+  float *Ls = reinterpret_cast<float *>(sm + OFF_AL);
+  float *Ts = reinterpret_cast<float *>(sm + OFF_TS);
+  float *scan = reinterpret_cast<float *>(sm + OFF_TP);  // [16 groups][128 channels]
+  float *s_em = reinterpret_cast<float *>(sm + OFF_SC), *s_egcm = s_em + 128, *s_egc = s_em + 256;
+
+  if (tid == 0) {
+    mbar_init(bar_full, 1);
+    mbar_init(bar_mma, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_b); prefetch_tmap(&tm_al);
+    mbar_expect_tx(bar_full, TMA_BYTES);
+#pragma unroll
+    for (int blk = 0; blk < 2; ++blk) {
+      tma_load_3d(sb + OFF_XA + blk * XA_BLK, &tm_b, 64 * blk, h, tok0, bar_full);         // b -> rows 0..63
+      tma_load_3d(sb + OFF_XA + blk * XA_BLK + 8192, &tm_q, 64 * blk, h, tok0, bar_full);  // q -> rows 64..127
+      tma_load_3d(sb + OFF_KT + blk * KT_BLK, &tm_k, 64 * blk, h, tok0, bar_full);
+      tma_load_3d(sb + OFF_AL + blk * 8192, &tm_al, 64 * blk, h, tok0, bar_full);
+    }
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  // the never-written blocks (0,1) and (2,3) of T, which the 32x32 merges read
+  for (int e = tid; e < 512; e += NT) {
+    const int R = 2 * (e >> 8), r = (e >> 4) & 15, j = e & 15;
+    Ts[(16 * R + r) * LDF + 16 * (R + 1) + j] = 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16);
+  bool ok = true;
+
+  // ------------------------------------------------------------ decay factors, operands in place
+  if (!mbar_wait_bounded(bar_full, 0, WAIT_NS)) ok = false;
+  if (__syncthreads_or(!ok)) goto done;
+  {
+    // thread = 8 key channels (chunk x8 of channel block cb) x 4 tokens (group G = rows 4G..4G+3);
+    // groups 0-7 hold tokens 0..31 (walk back to token 31), groups 8-15 tokens 32..63 (walk forward)
+    const int ch8 = tid & 15, G = tid >> 4, cb = ch8 >> 3, x8 = ch8 & 7;
+    uint4 ra[4], rb[4], rq[4], rk[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t o = sw128(4 * G + i, 8 * x8);
+      ra[i] = ld_s128(sm + OFF_AL + cb * 8192 + o);
+      rb[i] = ld_s128(sm + OFF_XA + cb * XA_BLK + o);
+      rq[i] = ld_s128(sm + OFF_XA + cb * XA_BLK + 8192 + o);
+      rk[i] = ld_s128(sm + OFF_KT + cb * KT_BLK + o);
+    }
+    float gp[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) gp[t] = 1.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (4 * G + i < Cc) {
+        float al[8];
+        unpack8(ra[i], al);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) gp[t] *= al[t];
+      }
+    *reinterpret_cast<float4 *>(&scan[G * 128 + 8 * ch8]) = make_float4(gp[0], gp[1], gp[2], gp[3]);
+    *reinterpret_cast<float4 *>(&scan[G * 128 + 8 * ch8 + 4]) = make_float4(gp[4], gp[5], gp[6], gp[7]);
+    __syncthreads();
+    if (tid < 128) {  // per channel: products between each group and token 31, in place of the group products
+      float pg[16];
+#pragma unroll
+      for (int g = 0; g < 16; ++g) pg[g] = scan[g * 128 + tid];
+      float acc = 1.f;
+#pragma unroll
+      for (int g = 7; g >= 0; --g) {
+        scan[g * 128 + tid] = acc;  // prod over groups g+1..7
+        acc *= pg[g];
+      }
+      const float em = acc;
+      acc = 1.f;
+#pragma unroll
+      for (int g = 8; g < 16; ++g) {
+        scan[g * 128 + tid] = acc;  // prod over groups 8..g-1
+        acc *= pg[g];
+      }
+      s_em[tid] = em;
+      s_egcm[tid] = acc;
+      s_egc[tid] = em * acc;
+    }
+    __syncthreads();
+    float run[8];
+    {
+      const float4 p0 = *reinterpret_cast<const float4 *>(&scan[G * 128 + 8 * ch8]);
+      const float4 p1 = *reinterpret_cast<const float4 *>(&scan[G * 128 + 8 * ch8 + 4]);
+      run[0] = p0.x; run[1] = p0.y; run[2] = p0.z; run[3] = p0.w;
+      run[4] = p1.x; run[5] = p1.y; run[6] = p1.z; run[7] = p1.w;
+    }
+    uint8_t *pa0 = sm + OFF_XA + cb * XA_BLK, *pk0 = sm + OFF_KT + cb * KT_BLK;
+    if (G < 8) {
+#pragma unroll
+      for (int i = 3; i >= 0; --i) {  // run = prod_{r < s <= 31} alpha_s
+        const int r = 4 * G + i;
+        float al[8], f[8], fi[8];
+        unpack8(ra[i], al);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          fi[t] = run[t];
+          f[t] = fast_rcp(run[t]);
+          if (r < Cc) run[t] *= al[t];
+        }
+        row_factors(pa0, pk0, sw128(r, 8 * x8), rb[i], rq[i], rk[i], r < Cc, f, fi);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {  // run = prod_{32 <= s <= r} alpha_s
+        const int r = 4 * G + i;
+        float al[8], f[8], fi[8];
+        unpack8(ra[i], al);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (r < Cc) run[t] *= al[t];
+          f[t] = run[t];
+          fi[t] = fast_rcp(run[t]);
+        }
+        row_factors(pa0, pk0, sw128(r, 8 * x8), rb[i], rq[i], rk[i], r < Cc, f, fi);
+      }
+    }
+  }
+  fence_proxy_async();
+  __syncthreads();
+
+  // ------------------------------------------------------------ M1: [L; P] = [A_m; Q_m] K_m^T (TMEM cols 0..63)
+  if (tid == 0) {
+    tc_fence_after();
+#pragma unroll
+    for (int k = 0; k < DK / 16; ++k) {
+      const uint32_t koff = (uint32_t)(k & 3) * 32u;
+      const uint64_t ad = sdesc_sw128(sb + OFF_XA + (k >> 2) * XA_BLK + koff, 16, 1024);
+      const uint64_t bd = sdesc_sw128(sb + OFF_KT + (k >> 2) * KT_BLK + koff, 16, 1024);
+      mma_bf16(tmem + 0, ad, bd, ID_LP, k > 0 ? 1u : 0u);
+    }
+    mma_commit(bar_mma);
+  }
+  if (!mbar_wait_bounded(bar_mma, 0, WAIT_NS)) ok = false;
+  if (__syncthreads_or(!ok)) goto done;
+  tc_fence_after();
+
+  // ------------------------------------------------------------ T = (I + L)^-1
+  {  // L (strict lower) -> fp32 scratch; P (inclusive lower) -> rows 64..127 of [T ; P]
+    float v[32];
+    tmem_ld32(tl + 32 * khalf, v);
+    tmem_wait_ld();
+    const int row = 32 * quad + lane;
+    if (row < 64) {
+#pragma unroll
+      for (int y = 0; y < 8; ++y) {
+        const int i = 32 * khalf + 4 * y;
+        *reinterpret_cast<float4 *>(&Ls[row * LDF + i]) =
+            make_float4(i < row ? v[4 * y] : 0.f, i + 1 < row ? v[4 * y + 1] : 0.f, i + 2 < row ? v[4 * y + 2] : 0.f,
+                        i + 3 < row ? v[4 * y + 3] : 0.f);
+      }
+    } else {
+      const int r = row - 64;
+#pragma unroll
+      for (int y = 0; y < 4; ++y) {
+        const int col = 32 * khalf + 8 * y;
+        float e[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) e[t] = (col + t <= r) ? v[8 * y + t] : 0.f;
+        st_s128(sm + OFF_TP + 8192 + sw128(r, col), pack8(e));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp < 2) {  // the four 16x16 diagonal blocks, right-looking; lane = column j of block R
+    const int R = 2 * warp + (lane >> 4), j = lane & 15;
+    const float *Lb = Ls + 16 * R * LDF + 16 * R;
+    float xv[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) xv[r] = (r == j) ? 1.f : 0.f;
+#pragma unroll
+    for (int i = 0; i < 15; ++i)
+#pragma unroll
+      for (int r = i + 1; r < 16; ++r) xv[r] = fmaf(-Lb[r * LDF + i], xv[i], xv[r]);
+    float *Tb = Ts + 16 * R * LDF + 16 * R;
+#pragma unroll
+    for (int r = 0; r < 16; ++r) Tb[r * LDF + j] = xv[r];
+  }
+  __syncthreads();
+  // merges on the warp-level tensor cores (tf32), with [[A,0],[C,B]]^-1 = [[A^-1,0],[-B^-1 C A^-1, B^-1]]:
+  // 16x16 blocks first; a warp needs only its own column tile of Y, so a warp barrier suffices
+  if (warp < 4) {
+    const int R = (warp < 2) ? 1 : 3, nt = warp & 1;
+    float d[4];
+    // Y_R = L_{R,R-1} T_{R-1,R-1}, parked in the upper block (R-1, R) of L
+    mma_tf32_16x8<16>(Ls + 16 * R * LDF + 16 * (R - 1), Ts + 16 * (R - 1) * LDF + 16 * (R - 1) + 8 * nt, lane, d);
+    store_16x8(Ls + 16 * (R - 1) * LDF + 16 * R + 8 * nt, lane, d, 1.f);
+    __syncwarp();
+    // T_{R,R-1} = -T_RR Y_R
+    mma_tf32_16x8<16>(Ts + 16 * R * LDF + 16 * R, Ls + 16 * (R - 1) * LDF + 16 * R + 8 * nt, lane, d);
+    store_16x8(Ts + 16 * R * LDF + 16 * (R - 1) + 8 * nt, lane, d, -1.f);
+  }
+  __syncthreads();
+  {  // lower-left 32x32 block: Y = L[32:64, 0:32] T[0:32, 0:32], parked in L[0:32, 32:64]
+    const int mt = warp >> 2, nt = warp & 3;
+    float d[4];
+    mma_tf32_16x8<32>(Ls + (32 + 16 * mt) * LDF, Ts + 8 * nt, lane, d);
+    store_16x8(Ls + 16 * mt * LDF + 32 + 8 * nt, lane, d, 1.f);  // disjoint from what this stage reads
+  }
+  __syncthreads();
+  {  // T[32:64, 0:32] = -T[32:64, 32:64] Y
+    const int mt = warp >> 2, nt = warp & 3;
+    float d[4];
+    mma_tf32_16x8<32>(Ts + (32 + 16 * mt) * LDF + 32, Ls + 32 + 8 * nt, lane, d);
+    store_16x8(Ts + (32 + 16 * mt) * LDF + 8 * nt, lane, d, -1.f);
+  }
+  __syncthreads();
+  {  // T -> rows 0..63 of [T ; P], bf16 (the upper-right 32x32 block is zero)
+    const int r = tid >> 2;
+#pragma unroll
+    for (int y = 0; y < 2; ++y) {
+      const int col = 16 * (tid & 3) + 8 * y;
+      float e[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (r >= 32 || col < 32) {
+        const float4 t0 = *reinterpret_cast<const float4 *>(&Ts[r * LDF + col]);
+        const float4 t1 = *reinterpret_cast<const float4 *>(&Ts[r * LDF + col + 4]);
+        e[0] = t0.x; e[1] = t0.y; e[2] = t0.z; e[3] = t0.w; e[4] = t1.x; e[5] = t1.y; e[6] = t1.z; e[7] = t1.w;
+      }
+      st_s128(sm + OFF_TP + sw128(r, col), pack8(e));
+    }
+  }
+  fence_proxy_async();
+  __syncthreads();
+
+  // ------------------------------------------------------------ round 1: [T; P] [A_m | T] and K_m^T T
+  // TMEM cols 0..127: rows 0..63 T A_m; cols 128..191: rows 64..127 P T; cols 192..255: K_m^T T
+  if (tid == 0) {
+    tc_fence_after();
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint64_t a_tp = sdesc_sw128(sb + OFF_TP + 32 * k, 16, 1024);
+      const uint64_t b_t = sdesc_sw128(sb + OFF_TP + 2048 * k, 8192, 1024);  // T: rows = K, MN-major
+      mma_bf16(tmem + 0, a_tp, sdesc_sw128(sb + OFF_XA + 2048 * k, XA_BLK, 1024), ID_KM128, k > 0 ? 1u : 0u);
+      mma_bf16(tmem + 128, a_tp, b_t, ID_KM64, k > 0 ? 1u : 0u);
+      mma_bf16(tmem + 192, sdesc_sw128(sb + OFF_KT + 2048 * k, KT_BLK, 1024), b_t, ID_MN64, k > 0 ? 1u : 0u);
+    }
+    mma_commit(bar_mma);
+  }
+  if (!mbar_wait_bounded(bar_mma, 1, WAIT_NS)) ok = false;
+  if (__syncthreads_or(!ok)) goto done;
+  tc_fence_after();
+  {
+    const int row = 32 * quad + lane;
+    if (quad < 2) {  // W = -T A_m -> W tile khalf (64 tokens x 64 channels, MN-major B operand)
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        float v[32];
+        tmem_ld32(tl + 64 * khalf + 32 * part, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          float e[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) e[t] = -v[8 * y + t];
+          st_s128(sm + OFF_AL + khalf * 8192 + sw128(row, 32 * part + 8 * y), pack8(e));
+        }
+      }
+    } else {  // Pt = P T -> rows 64..127 of the products; warp group khalf takes 32 columns
+      float v[32];
+      tmem_ld32(tl + 128 + 32 * khalf, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int y = 0; y < 4; ++y) st_s128(sm + OFF_TS + sw128(row - 64, 32 * khalf + 8 * y), pack8(&v[8 * y]));
+    }
+    {  // Nt = Diag(e^{g_C-m}) K_m^T T, key channel `row`, tokens 32 khalf .. +31
+      float v[32];
+      tmem_ld32(tl + 192 + 32 * khalf, v);
+      tmem_wait_ld();
+      const float g2 = s_egcm[row];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] *= g2;
+#pragma unroll
+      for (int y = 0; y < 4; ++y) st_s128(sm + OFF_TP + sw128(row, 32 * khalf + 8 * y), pack8(&v[8 * y]));
+    }
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+
+  // ------------------------------------------------------------ round 2: K_m^T W and [Pt; *] A_m
+  // TMEM cols 0..127: K_m^T W; cols 128..255: rows 0..63 Pt A_m (rows 64..127 read whatever follows Pt)
+  if (tid == 0) {
+    tc_fence_after();
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      mma_bf16(tmem + 0, sdesc_sw128(sb + OFF_KT + 2048 * k, KT_BLK, 1024), sdesc_sw128(sb + OFF_AL + 2048 * k, 8192, 1024),
+               ID_MN128, k > 0 ? 1u : 0u);
+      mma_bf16(tmem + 128, sdesc_sw128(sb + OFF_TS + 32 * k, 16, 1024), sdesc_sw128(sb + OFF_XA + 2048 * k, XA_BLK, 1024),
+               ID_KM128, k > 0 ? 1u : 0u);
+    }
+    mma_commit(bar_mma);
+  }
+  if (!mbar_wait_bounded(bar_mma, 0, WAIT_NS)) ok = false;
+  if (__syncthreads_or(!ok)) goto done;
+  tc_fence_after();
+  {
+    const int row = 32 * quad + lane;
+    {  // Mt = Diag(e^{g_C-m}) K_m^T W Diag(e^m): row = key channel, input channels 64 khalf .. +63
+      const float g2 = s_egcm[row];
+      uint8_t *dst = sm + (khalf ? OFF_AL : OFF_KT);
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        float v[32];
+        tmem_ld32(tl + 64 * khalf + 32 * part, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] *= g2 * s_em[64 * khalf + 32 * part + j];
+#pragma unroll
+        for (int y = 0; y < 4; ++y) st_s128(dst + sw128(row, 32 * part + 8 * y), pack8(&v[8 * y]));
+      }
+    }
+    if (quad < 2) {  // Qt = (Q_m - Pt A_m) Diag(e^m) in place of A_m, channel block khalf
+      uint8_t *blk = sm + OFF_XA + khalf * XA_BLK;
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        float v[32];
+        tmem_ld32(tl + 128 + 64 * khalf + 32 * part, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          const int col = 32 * part + 8 * y;
+          float qm[8], e[8];
+          unpack8(ld_s128(blk + 8192 + sw128(row, col)), qm);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) e[t] = (qm[t] - v[8 * y + t]) * s_em[64 * khalf + col + t];
+          st_s128(blk + sw128(row, col), pack8(e));
+        }
+      }
+    }
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+
+  // ------------------------------------------------------------ the record -> workspace
+  if (tid == 0) {
+    tma_store_2d(&tm_wm, 0, rec * 128, sb + OFF_KT);
+    tma_store_2d(&tm_wm, 64, rec * 128, sb + OFF_AL);
+    tma_store_2d(&tm_wn, 0, rec * 128, sb + OFF_TP);
+    tma_store_2d(&tm_wq, 0, rec * 64, sb + OFF_XA);
+    tma_store_2d(&tm_wq, 64, rec * 64, sb + OFF_XA + XA_BLK);
+    tma_store_2d(&tm_wp, 0, rec * 64, sb + OFF_TS);
+    bulk_store(p.g + (size_t)rec * 128, sb + OFF_SC + 256 * 4, REC_G);
+    bulk_commit();
+    bulk_wait_read();
+  }
+
+done:
+  if (!ok && tid == 0) atomicExch(p.status, 4);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ==================================================================== kernel 2: state pass
+namespace sp {
+constexpr int NT = 224;  // warps 0-3: state (thread = key channel); warp 4: loads; warps 5-6: U = w (.) v
+constexpr int NSTATE = 128;
+constexpr int BAR_STATE = 1;
+// one stage (chunk buffer); every MMA operand tile 1024-aligned
+constexpr uint32_t S_M = 0;                  // Mt: two 128-row tiles (input channel blocks)
+constexpr uint32_t S_N = S_M + REC_M;        // 32768: Nt
+constexpr uint32_t S_Q = S_N + REC_N;        // 49152: Qt: two 64-row tiles (an MMA reads 64 more rows past each)
+constexpr uint32_t S_P = S_Q + REC_Q;        // 65536: Pt
+constexpr uint32_t S_V = S_P + REC_P;        // 73728: v -> U = w (.) v (64 tokens x 64 columns)
+constexpr uint32_t S_W = S_V + 8192;         // 81920: w
+constexpr uint32_t S_G = S_W + 8192;         // 90112: e^{g_C}
+constexpr uint32_t STAGE = S_G + 1024;       // 91136
+constexpr uint32_t OFF_SB = 2 * STAGE;       // 182272: S (bf16), key channel rows x 64 columns; two buffers
+constexpr uint32_t OFF_BAR = OFF_SB + 2 * 16384;  // 215040
+constexpr uint32_t SMEM_USED = OFF_BAR + 128;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
+constexpr uint32_t TX_BYTES = REC_M + REC_N + REC_Q + REC_P + 2 * 8192 + REC_G;
+constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t TM_D1 = 0, TM_D2 = 64;  // D1: Mt S + Nt U; D2: rows 0..63 Qt S + Pt U
+enum { B_FULL0 = 0, B_FULL1, B_UREADY0, B_UREADY1, B_EMPTY0, B_EMPTY1, B_D1, B_D2, B_COUNT };
+static_assert(SMEM_BYTES <= 232448, "one CTA per SM");
+}  // namespace sp
+
+__global__ void __launch_bounds__(sp::NT, 1)
+    state_pass_kernel(const ChunkArgs a, const WyParams p, const __grid_constant__ CUtensorMap tm_wm,
+                      const __grid_constant__ CUtensorMap tm_wn, const __grid_constant__ CUtensorMap tm_wq,
+                      const __grid_constant__ CUtensorMap tm_wp, const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_w) {
+  using namespace sp;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 8 * B_COUNT);
+  auto bar = [&](int i) { return sb + OFF_BAR + 8u * (uint32_t)i; };
+
+  const int tiles = a.dv / NV;
+  const int tile = blockIdx.x % tiles;
+  const int h = (blockIdx.x / tiles) % a.H;
+  const int n = blockIdx.x / (tiles * a.H);
+  const int j0 = tile * NV;
+  int64_t bos;
+  int len;
+  seq_span(a, n, bos, len);
+  const int nch = (len + C - 1) / C;
+  const int coff = p.coff ? p.coff[n] : n * p.nc;  // global chunk of this sequence's chunk 0
+
+  if (tid == 0) {
+    for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), (i == B_UREADY0 || i == B_UREADY1) ? 2u : 1u);
+    fence_mbar_init();
+    prefetch_tmap(&tm_wm); prefetch_tmap(&tm_wn); prefetch_tmap(&tm_wq); prefetch_tmap(&tm_wp);
+    prefetch_tmap(&tm_v); prefetch_tmap(&tm_w);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+
+  if (warp == 4) {
+    // ---------------------------------------------------------- loads (one thread)
+    if (lane == 0) {
+      for (int c = 0; c < nch; ++c) {
+        const int s = c & 1;
+        // stage s last held chunk c-2: wait until the state side is done with it
+        if (c >= 2 && !mbar_wait_bounded(bar(B_EMPTY0 + s), ((c - 2) >> 1) & 1, WAIT_NS)) { ok = false; break; }
+        const uint32_t st = sb + s * STAGE, full = bar(B_FULL0 + s);
+        const int rec = (coff + c) * a.H + h;
+        const int tok0 = (int)(bos + (int64_t)c * C);
+        mbar_expect_tx(full, TX_BYTES);
+        tma_load_2d(st + S_M, &tm_wm, 0, rec * 128, full);
+        tma_load_2d(st + S_M + 16384, &tm_wm, 64, rec * 128, full);
+        tma_load_2d(st + S_N, &tm_wn, 0, rec * 128, full);
+        tma_load_2d(st + S_Q, &tm_wq, 0, rec * 64, full);
+        tma_load_2d(st + S_Q + 8192, &tm_wq, 64, rec * 64, full);
+        tma_load_2d(st + S_P, &tm_wp, 0, rec * 64, full);
+        tma_load_3d(st + S_V, &tm_v, j0, h, tok0, full);
+        tma_load_3d(st + S_W, &tm_w, j0, h, tok0, full);
+        bulk_load(st + S_G, p.g + (size_t)rec * 128, REC_G, full);
+      }
+    }
+  } else if (warp >= 5) {
+    // ---------------------------------------------------------- U = w (.) v, in place of v
+    const int uw = warp - 5;  // rows 32 uw .. 32 uw + 31
+    for (int c = 0; c < nch; ++c) {
+      const int s = c & 1;
+      const int Cc = min(C, len - c * C);
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar(B_FULL0 + s), (c >> 1) & 1, WAIT_NS))) { ok = false; break; }
+      uint8_t *vt = sm + s * STAGE + S_V;
+      const uint8_t *wt = sm + s * STAGE + S_W;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {  // 8 lanes cover one token row; rows past the sequence give U = 0
+        const int r = 32 * uw + 4 * i + (lane >> 3);
+        const uint32_t o = sw128(r, 8 * (lane & 7));
+        float vv[8], ww[8], uu[8];
+        unpack8(ld_s128(vt + o), vv);
+        unpack8(ld_s128(wt + o), ww);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) uu[t] = (r < Cc) ? vv[t] * ww[t] : 0.f;
+        st_s128(vt + o, pack8(uu));
+      }
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_UREADY0 + s));
+    }
+  } else {
+    // ---------------------------------------------------------- state side
+    const int ch = tid, quad = warp;
+    const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16);
+    const size_t s_off = (((size_t)n * a.H + h) * DK + ch) * (size_t)a.dv + j0;
+    float S[64];
+    if (a.S0) {
+#pragma unroll
+      for (int y = 0; y < 16; ++y) {
+        const float4 t = reinterpret_cast<const float4 *>(a.S0 + s_off)[y];
+        S[4 * y] = t.x; S[4 * y + 1] = t.y; S[4 * y + 2] = t.z; S[4 * y + 3] = t.w;
+      }
+    } else {
+#pragma unroll
+      for (int y = 0; y < 64; ++y) S[y] = 0.f;
+    }
+    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o);
+    for (int c = 0; c < nch; ++c) {
+      const int s = c & 1;
+      const uint32_t stg = sb + s * STAGE, sbf = sb + OFF_SB + (c & 1) * 16384;
+      const float *g1 = reinterpret_cast<const float *>(sm + s * STAGE + S_G);
+      const int Cc = min(C, len - c * C);
+      const int tok0 = (int)(bos + (int64_t)c * C);
+      // ---------------------------------------------------------- S -> shared (bf16), the B operand
+      // (this buffer was last read by the products of chunk c-2, complete since chunk c-1's D2)
+#pragma unroll
+      for (int y = 0; y < 8; ++y) st_s128(sm + OFF_SB + (c & 1) * 16384 + sw128(ch, 8 * y), pack8(&S[8 * y]));
+      fence_proxy_async();
+      if (!group_wait(BAR_STATE, NSTATE, bar(B_FULL0 + s), (c >> 1) & 1)) { ok = false; break; }
+      // ---------------------------------------------------------- D1 = Mt S + Nt U; D2 = [Qt; *] S + [Pt; *] U
+      if (ch == 0) {
+        bool u_ok = mbar_wait_bounded(bar(B_UREADY0 + s), (c >> 1) & 1, WAIT_NS);
+        if (u_ok) {
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < DK / 16; ++k)
+            mma_bf16(tmem + TM_D1, sdesc_sw128(stg + S_M + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
+                     sdesc_sw128(sbf + 2048 * k, 16384, 1024), ID_KM64, k > 0 ? 1u : 0u);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16(tmem + TM_D1, sdesc_sw128(stg + S_N + 32 * k, 16, 1024), sdesc_sw128(stg + S_V + 2048 * k, 8192, 1024),
+                     ID_KM64, 1u);
+          mma_commit(bar(B_D1));
+#pragma unroll
+          for (int k = 0; k < DK / 16; ++k)
+            mma_bf16(tmem + TM_D2, sdesc_sw128(stg + S_Q + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024),
+                     sdesc_sw128(sbf + 2048 * k, 16384, 1024), ID_KM64, k > 0 ? 1u : 0u);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16(tmem + TM_D2, sdesc_sw128(stg + S_P + 32 * k, 16, 1024), sdesc_sw128(stg + S_V + 2048 * k, 8192, 1024),
+                     ID_KM64, 1u);
+          mma_commit(bar(B_D2));
+        } else {
+          ok = false;
+        }
+      }
+      // ---------------------------------------------------------- S <- Diag(e^{g_C}) S + D1
+      if (!group_wait(BAR_STATE, NSTATE, bar(B_D1), c & 1, !ok)) { ok = false; break; }
+      tc_fence_after();
+      {
+        const float gc = g1[ch];
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          float v[32];
+          tmem_ld32(tl + TM_D1 + 32 * part, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) S[32 * part + j] = fmaf(gc, S[32 * part + j], v[j]);
+        }
+      }
+      // ---------------------------------------------------------- O (rows 0..63 of D2) -> global
+      if (!group_wait(BAR_STATE, NSTATE, bar(B_D2), c & 1)) { ok = false; break; }
+      tc_fence_after();
+      if (quad < 2) {  // warp-uniform: tcgen05.ld is a warp-collective instruction
+        const int r = 32 * quad + lane;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          float v[32];
+          tmem_ld32(tl + TM_D2 + 32 * part, v);
+          tmem_wait_ld();
+          if (r < Cc) {
+            __nv_bfloat16 *dst = o + ((size_t)(tok0 + r) * a.H + h) * (size_t)a.dv + j0 + 32 * part;
+#pragma unroll
+            for (int x = 0; x < 4; ++x) reinterpret_cast<uint4 *>(dst)[x] = pack8(&v[8 * x]);
+          }
+        }
+      }
+      tc_fence_before();
+      group_sync(BAR_STATE, NSTATE);
+      if (ch == 0) mbar_arrive(bar(B_EMPTY0 + s));  // stage s is free; D1 and D2 have been read
+    }
+    if (ok && a.ST) {
+#pragma unroll
+      for (int y = 0; y < 16; ++y)
+        reinterpret_cast<float4 *>(a.ST + s_off)[y] = make_float4(S[4 * y], S[4 * y + 1], S[4 * y + 2], S[4 * y + 3]);
+    }
+  }
+  if (!ok) atomicExch(p.status, 4);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// Chunk offsets of a packed batch: coff[0] = 0, coff[n+1] = coff[n] + ceil(len_n / 64).  One CTA.
+__global__ void __launch_bounds__(1024) chunk_offsets_kernel(const int32_t *cu, int N, int32_t *coff) {
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    carry = 0;
+    coff[0] = 0;
+  }
+  __syncthreads();
+  for (int base = 0; base < N; base += 1024) {
+    const int n = base + tid;
+    int x = n < N ? (cu[n + 1] - cu[n] + C - 1) / C : 0;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {  // inclusive scan inside the warp
+      const int y = __shfl_up_sync(0xffffffffu, x, d);
+      if (lane >= d) x += y;
+    }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int w = warp_sums[lane];
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, d);
+        if (lane >= d) w += y;
+      }
+      warp_sums[lane] = w;  // inclusive over warps
+    }
+    __syncthreads();
+    const int incl = carry + x + (warp > 0 ? warp_sums[warp - 1] : 0);
+    if (n < N) coff[n + 1] = incl;
+    __syncthreads();
+    if (tid == 1023) carry = incl;
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------ host side
+using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+  static EncodeTiled fn = nullptr;
+  if (!fn) {
+    void *q = nullptr;
+    cudaDriverEntryPointQueryResult r;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &q, cudaEnableDefault, &r) == cudaSuccess &&
+        r == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(q);
+  }
+  return fn;
+}
+
+// [tokens, H, D] bf16 token tensor, box = 64 channels x 1 head x 64 tokens, 128-byte swizzle
+bool map_tokens(CUtensorMap *m, const void *base, long long tokens, int H, int D) {
+  EncodeTiled enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)(tokens > 0 ? tokens : 1)};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  const cuuint32_t box[3] = {64, 1, 64};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [rows, cols] bf16 workspace matrix, box = 64 columns x box_rows rows, 128-byte swizzle
+bool map_matrix(CUtensorMap *m, void *base, long long rows, int cols, int box_rows) {
+  EncodeTiled enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Upper bound of the number of chunks of a batch: sum ceil(len_n / 64) <= floor((T + 63 N) / 64).
+long long chunk_capacity(int B, int T, bool packed) {
+  if (!packed) return (long long)B * ((T + C - 1) / C);
+  return ((long long)T + (long long)(C - 1) * B) / C;
+}
+
+// Workspace layout: Mt tiles | Nt tiles | Qt tiles | Pt tiles | e^{g_C} | chunk offsets (packed only)
+struct WsLayout {
+  long long records;
+  size_t m, n, q, p, g, coff, total;
+};
+WsLayout ws_layout(int B, int T, int H, bool packed) {
+  WsLayout L{};
+  L.records = chunk_capacity(B, T, packed) * H;
+  const size_t r = (size_t)L.records;
+  L.m = 0;
+  L.n = L.m + r * REC_M;
+  L.q = L.n + r * REC_N;
+  L.p = L.q + r * REC_Q;
+  L.g = L.p + r * REC_P;
+  L.coff = L.g + r * REC_G;
+  L.total = L.coff + (packed ? ((size_t)(B + 1) * 4 + 255) / 256 * 256 : 0);
+  return L;
+}
+
+}  // namespace
+
+bool chunk_wy_supported(int B, int T, int H, int dk, int dv, bool packed, bool bf16) {
+  if (!bf16 || dk != DK || dv % NV != 0) return false;
+  // TMA coordinates are int32: token rows (plus one chunk) and workspace rows (records x 128)
+  const long long tokens = packed ? (long long)T : (long long)B * T;
+  return tokens + C <= (long long)INT_MAX && chunk_capacity(B, T, packed) * H * 128 <= (long long)INT_MAX;
+}
+
+size_t chunk_wy_workspace_bytes(int B, int T, int H, bool packed) { return ws_layout(B, T, H, packed).total; }
+
+cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
+  const long long tokens = a.cu ? (long long)a.T : (long long)a.B * a.T;
+  const WsLayout L = ws_layout(a.B, a.T, a.H, a.cu != nullptr);
+  uint8_t *base = static_cast<uint8_t *>(ws);
+  WyParams p;
+  cudaError_t err = device_status_word(&p.status);
+  if (err != cudaSuccess) return err;
+  p.N = a.B;
+  p.nc = (a.T + C - 1) / C;
+  p.tokens = tokens;
+  p.coff = a.cu ? reinterpret_cast<const int32_t *>(base + L.coff) : nullptr;
+  p.g = reinterpret_cast<float *>(base + L.g);
+
+  CUtensorMap mq, mk, mb, mal, mv, mw, mm, mn, mqt, mp;
+  if (tokens > 0) {
+    if (!map_tokens(&mq, a.q, tokens, a.H, DK) || !map_tokens(&mk, a.k, tokens, a.H, DK) ||
+        !map_tokens(&mb, a.b, tokens, a.H, DK) || !map_tokens(&mal, a.alpha, tokens, a.H, DK) ||
+        !map_tokens(&mv, a.v, tokens, a.H, a.dv) || !map_tokens(&mw, a.w, tokens, a.H, a.dv) ||
+        !map_matrix(&mm, base + L.m, L.records * 128, 128, 128) ||
+        !map_matrix(&mn, base + L.n, L.records * 128, 64, 128) ||
+        !map_matrix(&mqt, base + L.q, L.records * 64, 128, 64) ||
+        !map_matrix(&mp, base + L.p, L.records * 64, 64, 64))
+      return cudaErrorInvalidValue;
+  } else {
+    // no token and no record: the state pass only copies S0 to S_T; its maps are never read
+    memset(&mv, 0, sizeof(mv));
+    mw = mm = mn = mqt = mp = mv;
+  }
+  if (a.cu) {
+    note_launch();
+    chunk_offsets_kernel<<<1, 1024, 0, stream>>>(a.cu, a.B, const_cast<int32_t *>(p.coff));
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  if (L.records > 0 && tokens > 0) {
+    err = cudaFuncSetAttribute(wy_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wy::SMEM_BYTES);
+    if (err != cudaSuccess) return err;
+    note_launch();
+    wy_factor_kernel<<<(unsigned)L.records, wy::NT, wy::SMEM_BYTES, stream>>>(a, p, mq, mk, mb, mal, mm, mn, mqt, mp);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  const long long blocks = (long long)a.B * a.H * (a.dv / NV);
+  err = cudaFuncSetAttribute(state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp::SMEM_BYTES);
+  if (err != cudaSuccess) return err;
+  note_launch();
+  state_pass_kernel<<<(unsigned)blocks, sp::NT, sp::SMEM_BYTES, stream>>>(a, p, mm, mn, mqt, mp, mv, mw);
+  return cudaGetLastError();
+}
+
+}  // namespace gdn2

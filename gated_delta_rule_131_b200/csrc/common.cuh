@@ -58,9 +58,17 @@ void note_launch();
 cudaError_t launch_chunk_simt(const ChunkArgs &a, bool bf16, cudaStream_t stream);
 bool chunk_tc_supported(const ChunkArgs &a, bool bf16);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream);
+// Two-kernel tensor-core path (WY factors of all chunks, then the state pass) over a workspace of
+// chunk_wy_workspace_bytes(...) bytes, 256-byte aligned, that it fully writes before reading.
+// The workspace depends only on the batch shape (B sequences, T tokens each or in total, H heads).
+bool chunk_wy_supported(int B, int T, int H, int dk, int dv, bool packed, bool bf16);
+size_t chunk_wy_workspace_bytes(int B, int T, int H, bool packed);
+cudaError_t launch_chunk_wy(const ChunkArgs &a, void *workspace, cudaStream_t stream);
 cudaError_t launch_bounded_wait_probe(uint64_t limit_ns, cudaStream_t stream);
 // Reads (and optionally clears) the device-side status word that bounded waits set.
 cudaError_t read_device_status(int *status, bool reset);
+// Device address of that word, for kernels compiled in other files.
+cudaError_t device_status_word(int **ptr);
 cudaError_t launch_decode(const DecodeArgs &a, bool bf16, cudaStream_t stream);
 
 }  // namespace gdn2

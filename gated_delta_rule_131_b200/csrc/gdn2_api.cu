@@ -2,6 +2,7 @@
 // See include/gdn2.h for the contract of every entry point.
 #include <atomic>
 #include <climits>
+#include <mutex>
 
 #include "common.cuh"
 #include "gdn2.h"
@@ -27,6 +28,53 @@ bool fits(long long a, long long b, long long c, long long d) {
     x *= y;
   }
   return true;
+}
+
+// Stream-ordered pool of the chunk workspaces, one per device, owned by the library.  Its release
+// threshold is unbounded, so memory freed back to it is kept for the next call instead of being
+// unmapped at every synchronisation.
+cudaError_t workspace_pool(cudaMemPool_t *pool) {
+  static std::mutex mu;
+  static cudaMemPool_t pools[64] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!pools[dev]) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t p = nullptr;
+    if ((err = cudaMemPoolCreate(&p, &props)) != cudaSuccess) return err;
+    uint64_t threshold = UINT64_MAX;
+    if ((err = cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &threshold)) != cudaSuccess) {
+      cudaMemPoolDestroy(p);
+      return err;
+    }
+    pools[dev] = p;
+  }
+  *pool = pools[dev];
+  return cudaSuccess;
+}
+
+// The tensor-core path with a workspace taken from the pool and returned to it on `stream`.
+cudaError_t run_chunk_wy(const gdn2::ChunkArgs &a, cudaStream_t stream) {
+  const size_t bytes = gdn2::chunk_wy_workspace_bytes(a.B, a.T, a.H, a.cu != nullptr);
+  void *ws = nullptr;
+  cudaError_t err;
+  if (bytes > 0) {
+    cudaMemPool_t pool;
+    if ((err = workspace_pool(&pool)) != cudaSuccess) return err;
+    if ((err = cudaMallocFromPoolAsync(&ws, bytes, pool, stream)) != cudaSuccess) return err;
+  }
+  err = gdn2::launch_chunk_wy(a, ws, stream);
+  if (ws) {
+    const cudaError_t ferr = cudaFreeAsync(ws, stream);
+    if (err == cudaSuccess) err = ferr;
+  }
+  return err;
 }
 
 }  // namespace
@@ -81,9 +129,18 @@ gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v, const vo
   const bool bf16 = dtype == GDN2_BF16;
   // bf16 with d_k = 128 runs on the tensor cores; fp32 (whose accuracy bf16 operands cannot
   // keep) and d_k = 64 run the SIMT kernel
-  const cudaError_t err = gdn2::chunk_tc_supported(a, bf16) ? gdn2::launch_chunk_tc(a, (cudaStream_t)stream)
+  const bool tc = gdn2::chunk_wy_supported(B, T, H, d_k, d_v, cu_seqlens != nullptr, bf16);
+  const cudaError_t err = tc ? run_chunk_wy(a, (cudaStream_t)stream)
                                                             : gdn2::launch_chunk_simt(a, bf16, (cudaStream_t)stream);
   return err == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+}
+
+size_t gdn2_chunk_fwd_workspace_bytes(int B, int T, int H, int d_k, int d_v, int chunk, int packed,
+                                      gdn2_dtype dtype) {
+  if (B <= 0 || T < 0 || H <= 0 || chunk != 64 || !supported_dk(d_k) || !supported_dv(d_v)) return 0;
+  if (dtype != GDN2_F32 && dtype != GDN2_BF16) return 0;
+  if (!gdn2::chunk_wy_supported(B, T, H, d_k, d_v, packed != 0, dtype == GDN2_BF16)) return 0;
+  return gdn2::chunk_wy_workspace_bytes(B, T, H, packed != 0);
 }
 
 gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v, const void *alpha,

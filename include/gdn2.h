@@ -26,8 +26,13 @@
  *
  * Conventions shared by every call:
  *   - All tensor pointers are DEVICE pointers owned by the caller, 16-byte
- *     aligned, densely packed row-major.  The library keeps no state between
- *     calls and allocates no device memory.
+ *     aligned, densely packed row-major.  The library keeps no per-call state
+ *     between calls.  gdn2_chunk_fwd on its tensor-core path (bf16, d_k = 128)
+ *     takes a workspace of gdn2_chunk_fwd_workspace_bytes() bytes from a
+ *     stream-ordered memory pool that the library creates once per device, and
+ *     gives it back on `stream` after its kernels; the pool keeps memory given
+ *     back to it for later calls until the process exits.  No other call
+ *     allocates device memory.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and never synchronise.  A validation failure returns before any
  *     launch and writes nothing.  A launch failure returns GDN2_ERR_CUDA.  No
@@ -90,12 +95,26 @@ typedef struct CUstream_st *gdn2_stream_t;
  * chunk: 64 (the only supported chunk length).
  * T == 0 (or an empty sequence) is valid: its S_T equals its S0; when the
  * batch holds no token at all, the token pointers (q .. w, o) may be NULL.
- * Returns GDN2_OK, or an error status with nothing launched.
+ * bf16 with d_k = 128 runs two tensor-core kernels over a workspace: the first
+ * forms the chunk's WY factors (T = (I + L)^-1, W = -T A, and the decay-
+ * absorbed q and k) for every chunk at once, the second carries the state
+ * through each sequence's chunks in order; other shapes and fp32 run one SIMT
+ * kernel without a workspace.
+ * Returns GDN2_OK, or an error status with nothing launched; GDN2_ERR_CUDA
+ * also when the workspace cannot be allocated.
  */
 GDN2_API gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *alpha,
                            const void *b, const void *w, const float *S0, void *o, float *S_T,
                            int B, int T, int H, int d_k, int d_v, int chunk,
                            const int32_t *cu_seqlens, gdn2_dtype dtype, gdn2_stream_t stream);
+
+/*
+ * gdn2_chunk_fwd_workspace_bytes -- device bytes gdn2_chunk_fwd takes from its pool for a call
+ * of this shape (packed != 0: a packed batch with cu_seqlens, B sequences, T tokens in total).
+ * 0 when the call runs without a workspace or the shape is not supported.  Host only.
+ */
+GDN2_API size_t gdn2_chunk_fwd_workspace_bytes(int B, int T, int H, int d_k, int d_v, int chunk, int packed,
+                                               gdn2_dtype dtype);
 
 /*
  * gdn2_decode_step -- one recurrent step for a batch of single tokens.
