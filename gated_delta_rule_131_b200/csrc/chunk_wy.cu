@@ -102,10 +102,15 @@ __device__ __forceinline__ bool group_or(int id, int count, bool pred) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-// Every thread of a warp group waits (bounded); the group agrees on the outcome.
+// Every thread of a warp group waits (bounded; try_wait suspends the thread in hardware, so polling
+// costs little); the group agrees on the outcome.
 __device__ __forceinline__ bool group_wait(int id, int count, uint32_t bar, uint32_t parity, bool fail = false) {
   const bool ok = mbar_wait_bounded(bar, parity, WAIT_NS);
   return !group_or(id, count, fail || !ok);
+}
+// The same for one warp.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, WAIT_NS));
 }
 
 // D (16 x 8) = A (16 x K) B (K x 8) on the warp-level tensor-core path (mma.sync, tf32 operands
@@ -601,27 +606,52 @@ done:
 }
 
 // ==================================================================== kernel 2: state pass
+// One CTA per (sequence, head, 128 value columns).  The products run transposed, with the state as
+// the A operand straight from tensor memory (value column = TMEM lane):
+//   D1^T = U^T Nt^T + S^T Mt^T   (128 value columns x 128 key channels)
+//   O^T  = S^T Qt^T + U^T Pt^T   (128 value columns x 64 tokens)
+// Roles: warps 0-7 hold the state (thread = value column v, key-channel half hf: S[64 hf ..][v]);
+// warp 8 loads chunks; warps 9-10 form U = w (.) v, and one of their threads stores O; warp 11
+// issues the products.
+// Tensor memory is double-buffered per chunk parity, so the U half of D1 and the output of chunk c
+// overlap the state chain, whose step per chunk is: S^T -> TMEM, S^T Mt^T, S update.
 namespace sp {
-constexpr int NT = 224;  // warps 0-3: state (thread = key channel); warp 4: loads; warps 5-6: U = w (.) v
-constexpr int NSTATE = 128;
+constexpr int VW = 128;        // value columns per CTA
+constexpr int NSTATE = 256;    // warps 0-7
+constexpr int NU = 64;         // warps 9-10
+constexpr int W_LOAD = 8, W_MMA = 11;
+constexpr int NT = 384;
 constexpr int BAR_STATE = 1;
-// one stage (chunk buffer); every MMA operand tile 1024-aligned
-constexpr uint32_t S_M = 0;                  // Mt: two 128-row tiles (input channel blocks)
-constexpr uint32_t S_N = S_M + REC_M;        // 32768: Nt
-constexpr uint32_t S_Q = S_N + REC_N;        // 49152: Qt: two 64-row tiles (an MMA reads 64 more rows past each)
-constexpr uint32_t S_P = S_Q + REC_Q;        // 65536: Pt
-constexpr uint32_t S_V = S_P + REC_P;        // 73728: v -> U = w (.) v (64 tokens x 64 columns)
-constexpr uint32_t S_W = S_V + 8192;         // 81920: w
-constexpr uint32_t S_G = S_W + 8192;         // 90112: e^{g_C}
-constexpr uint32_t STAGE = S_G + 1024;       // 91136
-constexpr uint32_t OFF_SB = 2 * STAGE;       // 182272: S (bf16), key channel rows x 64 columns; two buffers
-constexpr uint32_t OFF_BAR = OFF_SB + 2 * 16384;  // 215040
-constexpr uint32_t SMEM_USED = OFF_BAR + 128;
+// one stage (chunk buffer); every operand tile 1024-aligned
+constexpr uint32_t S_M = 0;                  // Mt: two tiles (input channel blocks), 128 rows each
+constexpr uint32_t S_N = S_M + REC_M;        // 32768: Nt, 128 rows
+constexpr uint32_t S_Q = S_N + REC_N;        // 49152: Qt: two tiles of 64 rows
+constexpr uint32_t S_P = S_Q + REC_Q;        // 65536: Pt, 64 rows
+constexpr uint32_t S_V = S_P + REC_P;        // 73728: v -> U = w (.) v: two 64-column tiles of 64 tokens
+constexpr uint32_t S_W = S_V + 16384;        // 90112: w
+constexpr uint32_t STAGE = S_W + 16384;      // 106496
+constexpr uint32_t OFF_OST = 2 * STAGE;      // 212992: O staging, two 64-column tiles of 64 tokens
+constexpr uint32_t OFF_G = OFF_OST + 16384;  // 229376: e^{g_C} of the two stages
+constexpr uint32_t OFF_BAR = OFF_G + 2 * REC_G;  // 230400
+constexpr uint32_t SMEM_USED = OFF_BAR + 256;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
-constexpr uint32_t TX_BYTES = REC_M + REC_N + REC_Q + REC_P + 2 * 8192 + REC_G;
-constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t TM_D1 = 0, TM_D2 = 64;  // D1: Mt S + Nt U; D2: rows 0..63 Qt S + Pt U
-enum { B_FULL0 = 0, B_FULL1, B_UREADY0, B_UREADY1, B_EMPTY0, B_EMPTY1, B_D1, B_D2, B_COUNT };
+constexpr uint32_t TX_BYTES = REC_M + REC_N + REC_Q + REC_P + 4 * 8192 + REC_G;
+constexpr uint32_t TMEM_COLS = 512;
+// per buffer b = chunk parity: S^T (bf16 pairs) 64 cols, D1^T 128 cols, O^T 64 cols
+constexpr uint32_t TM_AS = 0, TM_D1 = 128, TM_D2 = 384;
+constexpr uint32_t ID_D1 = idesc_bf16(128, 128, false, false), ID_D1U = idesc_bf16(128, 128, true, false);
+constexpr uint32_t ID_D2 = idesc_bf16(128, 64, false, false), ID_D2U = idesc_bf16(128, 64, true, false);
+enum {
+  B_FULL0 = 0, B_FULL1,      // stage loaded (TMA bytes)
+  B_UREADY0, B_UREADY1,      // U formed in the stage (one arrive per U warp)
+  B_SREADY,                  // S^T of the next chunk is in tensor memory
+  B_D1FULL0, B_D1FULL1,      // D1 of the buffer complete
+  B_D1FREE0, B_D1FREE1,      // D1 of the buffer read by the state warps
+  B_D2FULL0, B_D2FULL1,      // O^T of the buffer complete
+  B_OSTAGED0, B_OSTAGED1,    // O of the chunk read out (staged, or stored directly); O^T of the buffer free
+  B_OFREE,                   // the O staging buffer has been read by its store
+  B_COUNT
+};
 static_assert(SMEM_BYTES <= 232448, "one CTA per SM");
 }  // namespace sp
 
@@ -629,7 +659,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
     state_pass_kernel(const ChunkArgs a, const WyParams p, const __grid_constant__ CUtensorMap tm_wm,
                       const __grid_constant__ CUtensorMap tm_wn, const __grid_constant__ CUtensorMap tm_wq,
                       const __grid_constant__ CUtensorMap tm_wp, const __grid_constant__ CUtensorMap tm_v,
-                      const __grid_constant__ CUtensorMap tm_w) {
+                      const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_o) {
   using namespace sp;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -638,22 +668,23 @@ __global__ void __launch_bounds__(sp::NT, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 8 * B_COUNT);
   auto bar = [&](int i) { return sb + OFF_BAR + 8u * (uint32_t)i; };
 
-  const int tiles = a.dv / NV;
+  const int tiles = (a.dv + VW - 1) / VW;
   const int tile = blockIdx.x % tiles;
   const int h = (blockIdx.x / tiles) % a.H;
   const int n = blockIdx.x / (tiles * a.H);
-  const int j0 = tile * NV;
+  const int j0 = tile * VW;
   int64_t bos;
   int len;
   seq_span(a, n, bos, len);
   const int nch = (len + C - 1) / C;
   const int coff = p.coff ? p.coff[n] : n * p.nc;  // global chunk of this sequence's chunk 0
+  auto chunk_len = [&](int c) { return min(C, len - c * C); };
 
   if (tid == 0) {
-    for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), (i == B_UREADY0 || i == B_UREADY1) ? 2u : 1u);
+    for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), (i == B_UREADY0 || i == B_UREADY1) ? NU / 32 : 1u);
     fence_mbar_init();
     prefetch_tmap(&tm_wm); prefetch_tmap(&tm_wn); prefetch_tmap(&tm_wq); prefetch_tmap(&tm_wp);
-    prefetch_tmap(&tm_v); prefetch_tmap(&tm_w);
+    prefetch_tmap(&tm_v); prefetch_tmap(&tm_w); prefetch_tmap(&tm_o);
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
@@ -665,13 +696,17 @@ __global__ void __launch_bounds__(sp::NT, 1)
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
 
-  if (warp == 4) {
+  if (warp == W_LOAD) {
     // ---------------------------------------------------------- loads (one thread)
     if (lane == 0) {
       for (int c = 0; c < nch; ++c) {
         const int s = c & 1;
-        // stage s last held chunk c-2: wait until the state side is done with it
-        if (c >= 2 && !mbar_wait_bounded(bar(B_EMPTY0 + s), ((c - 2) >> 1) & 1, WAIT_NS)) { ok = false; break; }
+        // stage s last held chunk c-2: free once its products are complete and its e^{g_C} is read
+        if (c >= 2 && !(mbar_wait_bounded(bar(B_D2FULL0 + s), ((c - 2) >> 1) & 1, WAIT_NS) &&
+                        mbar_wait_bounded(bar(B_D1FREE0 + s), ((c - 2) >> 1) & 1, WAIT_NS))) {
+          ok = false;
+          break;
+        }
         const uint32_t st = sb + s * STAGE, full = bar(B_FULL0 + s);
         const int rec = (coff + c) * a.H + h;
         const int tok0 = (int)(bos + (int64_t)c * C);
@@ -682,130 +717,176 @@ __global__ void __launch_bounds__(sp::NT, 1)
         tma_load_2d(st + S_Q, &tm_wq, 0, rec * 64, full);
         tma_load_2d(st + S_Q + 8192, &tm_wq, 64, rec * 64, full);
         tma_load_2d(st + S_P, &tm_wp, 0, rec * 64, full);
-        tma_load_3d(st + S_V, &tm_v, j0, h, tok0, full);
-        tma_load_3d(st + S_W, &tm_w, j0, h, tok0, full);
-        bulk_load(st + S_G, p.g + (size_t)rec * 128, REC_G, full);
+#pragma unroll
+        for (int vb = 0; vb < 2; ++vb) {  // columns past d_v (d_v = 64) load as zeros
+          tma_load_3d(st + S_V + vb * 8192, &tm_v, j0 + 64 * vb, h, tok0, full);
+          tma_load_3d(st + S_W + vb * 8192, &tm_w, j0 + 64 * vb, h, tok0, full);
+        }
+        bulk_load(sb + OFF_G + s * REC_G, p.g + (size_t)rec * 128, REC_G, full);
       }
     }
-  } else if (warp >= 5) {
-    // ---------------------------------------------------------- U = w (.) v, in place of v
-    const int uw = warp - 5;  // rows 32 uw .. 32 uw + 31
+  } else if (warp == W_MMA) {
+    // ---------------------------------------------------------- products (one thread)
+    if (lane == 0) {
+      for (int c = 0; c < nch; ++c) {
+        const int s = c & 1, b = c & 1, ph = (c >> 1) & 1;
+        const uint32_t stg = sb + s * STAGE;
+        const uint32_t as = tmem + TM_AS + 64 * b, d1 = tmem + TM_D1 + 128 * b, d2 = tmem + TM_D2 + 64 * b;
+        if (!mbar_wait_bounded(bar(B_UREADY0 + s), ph, WAIT_NS)) { ok = false; break; }
+        if (c >= 2 && !mbar_wait_bounded(bar(B_D1FREE0 + b), ph ^ 1, WAIT_NS)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 4; ++k)  // U^T Nt^T, before the state is known
+          mma_bf16(d1, sdesc_sw128(stg + S_V + 2048 * k, 8192, 1024), sdesc_sw128(stg + S_N + 32 * k, 16, 1024), ID_D1U,
+                   k > 0 ? 1u : 0u);
+        if (!mbar_wait_bounded(bar(B_SREADY), c & 1, WAIT_NS)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < DK / 16; ++k)
+          mma_bf16_tmem_a(d1, as + 8 * k, sdesc_sw128(stg + S_M + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024), ID_D1, 1u);
+        mma_commit(bar(B_D1FULL0 + b));
+        if (c >= 2 && !mbar_wait_bounded(bar(B_OSTAGED0 + b), ph ^ 1, WAIT_NS)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < DK / 16; ++k)
+          mma_bf16_tmem_a(d2, as + 8 * k, sdesc_sw128(stg + S_Q + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024), ID_D2,
+                          k > 0 ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_bf16(d2, sdesc_sw128(stg + S_V + 2048 * k, 8192, 1024), sdesc_sw128(stg + S_P + 32 * k, 16, 1024), ID_D2U, 1u);
+        mma_commit(bar(B_D2FULL0 + b));
+      }
+    }
+  } else if (warp > W_LOAD) {
+    // ---------------------------------------------------------- U = w (.) v in place of v; O stores
+    const int u = tid - (W_LOAD + 1) * 32;  // 16 threads per token row, one 8-column chunk each
+    const bool storer = u == NU - 32;       // lane 0 of the second U warp
+    // O of chunk k, staged by the state warps, -> global; then the staging buffer is free
+    auto store_o = [&](int k) {
+      if (!mbar_wait_bounded(bar(B_OSTAGED0 + (k & 1)), (k >> 1) & 1, WAIT_NS)) return false;
+      if (chunk_len(k) == C) {
+        const int tok0 = (int)(bos + (int64_t)k * C);
+        tma_store_3d(&tm_o, j0, h, tok0, sb + OFF_OST);
+        if (j0 + 64 < a.dv) tma_store_3d(&tm_o, j0 + 64, h, tok0, sb + OFF_OST + 8192);
+        bulk_commit();
+        bulk_wait_read();
+      }
+      mbar_arrive(bar(B_OFREE));
+      return true;
+    };
     for (int c = 0; c < nch; ++c) {
       const int s = c & 1;
-      const int Cc = min(C, len - c * C);
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar(B_FULL0 + s), (c >> 1) & 1, WAIT_NS))) { ok = false; break; }
+      const int Cc = chunk_len(c);
+      if (!warp_wait(bar(B_FULL0 + s), (c >> 1) & 1)) { ok = false; break; }
       uint8_t *vt = sm + s * STAGE + S_V;
       const uint8_t *wt = sm + s * STAGE + S_W;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {  // 8 lanes cover one token row; rows past the sequence give U = 0
-        const int r = 32 * uw + 4 * i + (lane >> 3);
-        const uint32_t o = sw128(r, 8 * (lane & 7));
-        float vv[8], ww[8], uu[8];
-        unpack8(ld_s128(vt + o), vv);
-        unpack8(ld_s128(wt + o), ww);
-#pragma unroll
-        for (int t = 0; t < 8; ++t) uu[t] = (r < Cc) ? vv[t] * ww[t] : 0.f;
-        st_s128(vt + o, pack8(uu));
+      for (int i = 0; i < 64 * 16 / NU; ++i) {  // rows past the sequence give U = 0
+        const int r = (NU / 16) * i + (u >> 4), x = u & 15;
+        const uint32_t o = (x >> 3) * 8192 + sw128(r, 8 * (x & 7));
+        uint4 uu = make_uint4(0u, 0u, 0u, 0u);
+        if (r < Cc) {  // bf16 x bf16 is exact in fp32, so the packed product is the rounded fp32 one
+          const uint4 vv = ld_s128(vt + o), ww = ld_s128(wt + o);
+          uu.x = bf2_mul(vv.x, ww.x);
+          uu.y = bf2_mul(vv.y, ww.y);
+          uu.z = bf2_mul(vv.z, ww.z);
+          uu.w = bf2_mul(vv.w, ww.w);
+        }
+        st_s128(vt + o, uu);
       }
       fence_proxy_async();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_UREADY0 + s));
+      if (storer && c >= 1 && !store_o(c - 1)) ok = false;
+      if (!__all_sync(0xffffffffu, ok)) break;
     }
+    if (storer && ok && nch > 0 && !store_o(nch - 1)) ok = false;
   } else {
     // ---------------------------------------------------------- state side
-    const int ch = tid, quad = warp;
-    const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16);
-    const size_t s_off = (((size_t)n * a.H + h) * DK + ch) * (size_t)a.dv + j0;
+    const int q4 = warp & 3, hf = warp >> 2;
+    const int v = 32 * q4 + lane;            // value column within the tile (TMEM lane)
+    const bool vin = j0 + v < a.dv;
+    const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
+    const size_t s_base = (((size_t)n * a.H + h) * DK + 64 * hf) * (size_t)a.dv + j0 + v;  // S[64 hf][j0 + v]
     float S[64];
-    if (a.S0) {
 #pragma unroll
-      for (int y = 0; y < 16; ++y) {
-        const float4 t = reinterpret_cast<const float4 *>(a.S0 + s_off)[y];
-        S[4 * y] = t.x; S[4 * y + 1] = t.y; S[4 * y + 2] = t.z; S[4 * y + 3] = t.w;
-      }
-    } else {
-#pragma unroll
-      for (int y = 0; y < 64; ++y) S[y] = 0.f;
-    }
+    for (int i = 0; i < 64; ++i) S[i] = (a.S0 && vin) ? a.S0[s_base + (size_t)i * a.dv] : 0.f;
     __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o);
+    // S^T of the chunk about to start -> tensor memory buffer b (bf16 pairs); signals the issuer
+    auto put_state = [&](int b) {
+      uint32_t r[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) r[i] = f2_to_bf2(S[2 * i], S[2 * i + 1]);
+      tmem_st32(tl + TM_AS + 64 * b + 32 * hf, r);
+      tmem_wait_st();
+    };
+    if (nch > 0) {
+      put_state(0);
+      tc_fence_before();
+      group_sync(BAR_STATE, NSTATE);
+      if (tid == 0) mbar_arrive(bar(B_SREADY));
+    }
     for (int c = 0; c < nch; ++c) {
-      const int s = c & 1;
-      const uint32_t stg = sb + s * STAGE, sbf = sb + OFF_SB + (c & 1) * 16384;
-      const float *g1 = reinterpret_cast<const float *>(sm + s * STAGE + S_G);
-      const int Cc = min(C, len - c * C);
+      const int s = c & 1, b = c & 1, ph = (c >> 1) & 1;
+      const int Cc = chunk_len(c);
       const int tok0 = (int)(bos + (int64_t)c * C);
-      // ---------------------------------------------------------- S -> shared (bf16), the B operand
-      // (this buffer was last read by the products of chunk c-2, complete since chunk c-1's D2)
-#pragma unroll
-      for (int y = 0; y < 8; ++y) st_s128(sm + OFF_SB + (c & 1) * 16384 + sw128(ch, 8 * y), pack8(&S[8 * y]));
-      fence_proxy_async();
-      if (!group_wait(BAR_STATE, NSTATE, bar(B_FULL0 + s), (c >> 1) & 1)) { ok = false; break; }
-      // ---------------------------------------------------------- D1 = Mt S + Nt U; D2 = [Qt; *] S + [Pt; *] U
-      if (ch == 0) {
-        bool u_ok = mbar_wait_bounded(bar(B_UREADY0 + s), (c >> 1) & 1, WAIT_NS);
-        if (u_ok) {
-          tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < DK / 16; ++k)
-            mma_bf16(tmem + TM_D1, sdesc_sw128(stg + S_M + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
-                     sdesc_sw128(sbf + 2048 * k, 16384, 1024), ID_KM64, k > 0 ? 1u : 0u);
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16(tmem + TM_D1, sdesc_sw128(stg + S_N + 32 * k, 16, 1024), sdesc_sw128(stg + S_V + 2048 * k, 8192, 1024),
-                     ID_KM64, 1u);
-          mma_commit(bar(B_D1));
-#pragma unroll
-          for (int k = 0; k < DK / 16; ++k)
-            mma_bf16(tmem + TM_D2, sdesc_sw128(stg + S_Q + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024),
-                     sdesc_sw128(sbf + 2048 * k, 16384, 1024), ID_KM64, k > 0 ? 1u : 0u);
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16(tmem + TM_D2, sdesc_sw128(stg + S_P + 32 * k, 16, 1024), sdesc_sw128(stg + S_V + 2048 * k, 8192, 1024),
-                     ID_KM64, 1u);
-          mma_commit(bar(B_D2));
-        } else {
-          ok = false;
-        }
-      }
       // ---------------------------------------------------------- S <- Diag(e^{g_C}) S + D1
-      if (!group_wait(BAR_STATE, NSTATE, bar(B_D1), c & 1, !ok)) { ok = false; break; }
+      if (!group_wait(BAR_STATE, NSTATE, bar(B_D1FULL0 + b), ph)) { ok = false; break; }
       tc_fence_after();
       {
-        const float gc = g1[ch];
+        const float4 *g1 = reinterpret_cast<const float4 *>(sm + OFF_G + s * REC_G) + 16 * hf;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
-          float v[32];
-          tmem_ld32(tl + TM_D1 + 32 * part, v);
+          float d[32];
+          tmem_ld32(tmem + ((uint32_t)(32 * q4) << 16) + TM_D1 + 128 * b + 64 * hf + 32 * part, d);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) S[32 * part + j] = fmaf(gc, S[32 * part + j], v[j]);
+          for (int y = 0; y < 8; ++y) {
+            const float4 g = g1[8 * part + y];
+            const int i = 32 * part + 4 * y;
+            S[i] = fmaf(g.x, S[i], d[4 * y]);
+            S[i + 1] = fmaf(g.y, S[i + 1], d[4 * y + 1]);
+            S[i + 2] = fmaf(g.z, S[i + 2], d[4 * y + 2]);
+            S[i + 3] = fmaf(g.w, S[i + 3], d[4 * y + 3]);
+          }
         }
       }
-      // ---------------------------------------------------------- O (rows 0..63 of D2) -> global
-      if (!group_wait(BAR_STATE, NSTATE, bar(B_D2), c & 1)) { ok = false; break; }
+      // the next chunk's S^T goes into the other buffer (its last reader, O^T of chunk c-1, is complete)
+      if (c + 1 < nch) put_state(b ^ 1);
+      tc_fence_before();
+      group_sync(BAR_STATE, NSTATE);
+      if (tid == 0) {
+        mbar_arrive(bar(B_D1FREE0 + b));
+        if (c + 1 < nch) mbar_arrive(bar(B_SREADY));
+      }
+      // ---------------------------------------------------------- O: tokens 32 hf .. 32 hf + 31 of column v
+      if (!group_wait(BAR_STATE, NSTATE, bar(B_D2FULL0 + b), ph)) { ok = false; break; }
       tc_fence_after();
-      if (quad < 2) {  // warp-uniform: tcgen05.ld is a warp-collective instruction
-        const int r = 32 * quad + lane;
+      {
+        float d[32];
+        tmem_ld32(tl + TM_D2 + 64 * b + 32 * hf, d);
+        tmem_wait_ld();
+        if (Cc == C) {  // staged for one TMA store per 64-column tile, once the previous store has read it
+          if (c >= 1 && !group_wait(BAR_STATE, NSTATE, bar(B_OFREE), (c - 1) & 1)) { ok = false; break; }
+          uint8_t *ot = sm + OFF_OST + (v >> 6) * 8192;
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          float v[32];
-          tmem_ld32(tl + TM_D2 + 32 * part, v);
-          tmem_wait_ld();
-          if (r < Cc) {
-            __nv_bfloat16 *dst = o + ((size_t)(tok0 + r) * a.H + h) * (size_t)a.dv + j0 + 32 * part;
+          for (int j = 0; j < 32; ++j)
+            *reinterpret_cast<__nv_bfloat16 *>(ot + sw128(32 * hf + j, v & 63)) = __float2bfloat16_rn(d[j]);
+          fence_proxy_async();
+        } else if (vin) {
+          __nv_bfloat16 *dst = o + ((size_t)tok0 * a.H + h) * (size_t)a.dv + j0 + v;
 #pragma unroll
-            for (int x = 0; x < 4; ++x) reinterpret_cast<uint4 *>(dst)[x] = pack8(&v[8 * x]);
-          }
+          for (int j = 0; j < 32; ++j)
+            if (32 * hf + j < Cc) dst[(size_t)(32 * hf + j) * a.H * a.dv] = __float2bfloat16_rn(d[j]);
         }
       }
       tc_fence_before();
       group_sync(BAR_STATE, NSTATE);
-      if (ch == 0) mbar_arrive(bar(B_EMPTY0 + s));  // stage s is free; D1 and D2 have been read
+      if (tid == 0) mbar_arrive(bar(B_OSTAGED0 + s));
     }
-    if (ok && a.ST) {
+    if (ok && a.ST && vin) {
 #pragma unroll
-      for (int y = 0; y < 16; ++y)
-        reinterpret_cast<float4 *>(a.ST + s_off)[y] = make_float4(S[4 * y], S[4 * y + 1], S[4 * y + 2], S[4 * y + 3]);
+      for (int i = 0; i < 64; ++i) a.ST[s_base + (size_t)i * a.dv] = S[i];
     }
   }
   if (!ok) atomicExch(p.status, 4);
@@ -947,11 +1028,12 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   p.coff = a.cu ? reinterpret_cast<const int32_t *>(base + L.coff) : nullptr;
   p.g = reinterpret_cast<float *>(base + L.g);
 
-  CUtensorMap mq, mk, mb, mal, mv, mw, mm, mn, mqt, mp;
+  CUtensorMap mq, mk, mb, mal, mv, mw, mo, mm, mn, mqt, mp;
   if (tokens > 0) {
     if (!map_tokens(&mq, a.q, tokens, a.H, DK) || !map_tokens(&mk, a.k, tokens, a.H, DK) ||
         !map_tokens(&mb, a.b, tokens, a.H, DK) || !map_tokens(&mal, a.alpha, tokens, a.H, DK) ||
         !map_tokens(&mv, a.v, tokens, a.H, a.dv) || !map_tokens(&mw, a.w, tokens, a.H, a.dv) ||
+        !map_tokens(&mo, a.o, tokens, a.H, a.dv) ||
         !map_matrix(&mm, base + L.m, L.records * 128, 128, 128) ||
         !map_matrix(&mn, base + L.n, L.records * 128, 64, 128) ||
         !map_matrix(&mqt, base + L.q, L.records * 64, 128, 64) ||
@@ -960,7 +1042,7 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   } else {
     // no token and no record: the state pass only copies S0 to S_T; its maps are never read
     memset(&mv, 0, sizeof(mv));
-    mw = mm = mn = mqt = mp = mv;
+    mw = mo = mm = mn = mqt = mp = mv;
   }
   if (a.cu) {
     note_launch();
@@ -974,11 +1056,11 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
     wy_factor_kernel<<<(unsigned)L.records, wy::NT, wy::SMEM_BYTES, stream>>>(a, p, mq, mk, mb, mal, mm, mn, mqt, mp);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
-  const long long blocks = (long long)a.B * a.H * (a.dv / NV);
+  const long long blocks = (long long)a.B * a.H * ((a.dv + sp::VW - 1) / sp::VW);
   err = cudaFuncSetAttribute(state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp::SMEM_BYTES);
   if (err != cudaSuccess) return err;
   note_launch();
-  state_pass_kernel<<<(unsigned)blocks, sp::NT, sp::SMEM_BYTES, stream>>>(a, p, mm, mn, mqt, mp, mv, mw);
+  state_pass_kernel<<<(unsigned)blocks, sp::NT, sp::SMEM_BYTES, stream>>>(a, p, mm, mn, mqt, mp, mv, mw, mo);
   return cudaGetLastError();
 }
 
