@@ -82,6 +82,12 @@ __device__ __forceinline__ void unpack8(uint4 u, float *e) {
   t = bf2_to_f2(u.w); e[6] = t.x; e[7] = t.y;
 }
 __device__ __forceinline__ float fast_rcp(float x) { return __fdividef(1.f, x); }
+// Two fp32 products at once (sm_100 packed fp32 pipe; each lane rounds exactly like a scalar product).
+__device__ __forceinline__ void mul2(float *d, const float *a, const float *b) {
+  const float2 r = __fmul2_rn(make_float2(a[0], a[1]), make_float2(b[0], b[1]));
+  d[0] = r.x;
+  d[1] = r.y;
+}
 
 __device__ __forceinline__ void group_sync(int id, int count) {
   asm volatile("barrier.cta.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -137,6 +143,33 @@ __device__ __forceinline__ void mma_tf32_16x8(const float *A, const float *B, in
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
   }
 }
+// D (16 x 8) = A (16 x 32) Y (32 x 8) with Y in registers as two 16 x 8 accumulator fragments
+// (y0: rows 0..15, y1: rows 16..31, the layout mma_tf32_16x8 returns); each B fragment element is
+// fetched from the lane that holds it.
+__device__ __forceinline__ void mma_tf32_16x8_yreg(const float *A, const float (&y0)[4], const float (&y1)[4], int lane,
+                                                   float (&d)[4]) {
+  const int g = lane >> 2, t = lane & 3;
+  d[0] = d[1] = d[2] = d[3] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    const float(&y)[4] = kk < 2 ? y0 : y1;
+    const int hi = (kk & 1) ? 2 : 0;  // rows 8..15 of the fragment sit in elements 2, 3
+    // B[8 kk + t][g] and B[8 kk + t + 4][g]: fragment row t (or t + 4), column g
+    const float e0 = __shfl_sync(0xffffffffu, y[hi], 4 * t + (g >> 1));
+    const float o0 = __shfl_sync(0xffffffffu, y[hi + 1], 4 * t + (g >> 1));
+    const float e1 = __shfl_sync(0xffffffffu, y[hi], 4 * (t + 4) + (g >> 1));
+    const float o1 = __shfl_sync(0xffffffffu, y[hi + 1], 4 * (t + 4) + (g >> 1));
+    const uint32_t b0 = to_tf32((g & 1) ? o0 : e0), b1 = to_tf32((g & 1) ? o1 : e1);
+    const int k0 = 8 * kk;
+    const uint32_t a0 = to_tf32(A[g * LDF + k0 + t]), a1 = to_tf32(A[(g + 8) * LDF + k0 + t]);
+    const uint32_t a2 = to_tf32(A[g * LDF + k0 + t + 4]), a3 = to_tf32(A[(g + 8) * LDF + k0 + t + 4]);
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+}
 // Store a 16 x 8 tile (times `scale`) into a row-major fp32 block with row stride LDF.
 __device__ __forceinline__ void store_16x8(float *D, int lane, const float (&d)[4], float scale) {
   const int g = lane >> 2, t = lane & 3;
@@ -156,10 +189,11 @@ __device__ __forceinline__ void row_factors(uint8_t *pa, uint8_t *pk, uint32_t o
     unpack8(rq, qv);
     unpack8(rk, kv);
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      ea[t] = bb[t] * kv[t] * f[t];
-      eq[t] = qv[t] * f[t];
-      ek[t] = kv[t] * fi[t];
+    for (int t = 0; t < 8; t += 2) {  // (b k) f, q f, k / f
+      mul2(&ea[t], &bb[t], &kv[t]);
+      mul2(&ea[t], &ea[t], &f[t]);
+      mul2(&eq[t], &qv[t], &f[t]);
+      mul2(&ek[t], &kv[t], &fi[t]);
     }
     wa = pack8(ea);
     wq = pack8(eq);
@@ -202,6 +236,7 @@ static_assert(OFF_AL % 1024 == 0 && OFF_TS % 1024 == 0, "MMA operand tiles are 1
 
 struct WyParams {
   int *status;     // device status word: GDN2_ERR_TIMEOUT (4) when a bounded wait gave up
+  int prefetch_stride;  // WY CTAs resident at once (two per SM)
   int N;           // sequences
   int nc;          // chunks per sequence of a dense batch
   int64_t tokens;  // rows of the token tensors
@@ -257,6 +292,34 @@ __global__ void __launch_bounds__(wy::NT, 2)
       tma_load_3d(sb + OFF_XA + blk * XA_BLK + 8192, &tm_q, 64 * blk, h, tok0, bar_full);  // q -> rows 64..127
       tma_load_3d(sb + OFF_KT + blk * KT_BLK, &tm_k, 64 * blk, h, tok0, bar_full);
       tma_load_3d(sb + OFF_AL + blk * 8192, &tm_al, 64 * blk, h, tok0, bar_full);
+    }
+    // the record about one wave later (CTAs resident at once = prefetch_stride) into L2
+    const int nrec = rec + p.prefetch_stride;
+    if (nrec < (int)gridDim.x) {
+      const int nh = nrec % a.H, ng = nrec / a.H;
+      int nn = -1, ncc = 0;
+      if (p.coff) {
+        if (ng < p.coff[p.N]) {
+          nn = seq_of_chunk(p.coff, p.N, ng);
+          ncc = ng - p.coff[nn];
+        }
+      } else {
+        nn = ng / p.nc;
+        ncc = ng % p.nc;
+      }
+      if (nn >= 0) {
+        int64_t nbos;
+        int nlen;
+        seq_span(a, nn, nbos, nlen);
+        const int ntok = (int)(nbos + (int64_t)ncc * C);
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk) {
+          tma_prefetch_3d(&tm_b, 64 * blk, nh, ntok);
+          tma_prefetch_3d(&tm_q, 64 * blk, nh, ntok);
+          tma_prefetch_3d(&tm_k, 64 * blk, nh, ntok);
+          tma_prefetch_3d(&tm_al, 64 * blk, nh, ntok);
+        }
+      }
     }
   }
   if (warp == 0) {
@@ -441,17 +504,13 @@ __global__ void __launch_bounds__(wy::NT, 2)
     store_16x8(Ts + 16 * R * LDF + 16 * (R - 1) + 8 * nt, lane, d, -1.f);
   }
   __syncthreads();
-  {  // lower-left 32x32 block: Y = L[32:64, 0:32] T[0:32, 0:32], parked in L[0:32, 32:64]
+  {  // lower-left 32x32 block: T[32:64, 0:32] = -T[32:64, 32:64] Y with Y = L[32:64, 0:32] T[0:32, 0:32];
+     // warp (mt, nt) forms both row halves of Y's column tile nt itself and keeps them in registers
     const int mt = warp >> 2, nt = warp & 3;
-    float d[4];
-    mma_tf32_16x8<32>(Ls + (32 + 16 * mt) * LDF, Ts + 8 * nt, lane, d);
-    store_16x8(Ls + 16 * mt * LDF + 32 + 8 * nt, lane, d, 1.f);  // disjoint from what this stage reads
-  }
-  __syncthreads();
-  {  // T[32:64, 0:32] = -T[32:64, 32:64] Y
-    const int mt = warp >> 2, nt = warp & 3;
-    float d[4];
-    mma_tf32_16x8<32>(Ts + (32 + 16 * mt) * LDF + 32, Ls + 32 + 8 * nt, lane, d);
+    float y0[4], y1[4], d[4];
+    mma_tf32_16x8<32>(Ls + 32 * LDF, Ts + 8 * nt, lane, y0);
+    mma_tf32_16x8<32>(Ls + 48 * LDF, Ts + 8 * nt, lane, y1);
+    mma_tf32_16x8_yreg(Ts + (32 + 16 * mt) * LDF + 32, y0, y1, lane, d);
     store_16x8(Ts + (32 + 16 * mt) * LDF + 8 * nt, lane, d, -1.f);
   }
   __syncthreads();
@@ -517,8 +576,9 @@ __global__ void __launch_bounds__(wy::NT, 2)
       tmem_ld32(tl + 192 + 32 * khalf, v);
       tmem_wait_ld();
       const float g2 = s_egcm[row];
+      const float g2p[2] = {g2, g2};
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] *= g2;
+      for (int j = 0; j < 32; j += 2) mul2(&v[j], &v[j], g2p);
 #pragma unroll
       for (int y = 0; y < 4; ++y) st_s128(sm + OFF_TP + sw128(row, 32 * khalf + 8 * y), pack8(&v[8 * y]));
     }
@@ -553,8 +613,17 @@ __global__ void __launch_bounds__(wy::NT, 2)
         float v[32];
         tmem_ld32(tl + 64 * khalf + 32 * part, v);
         tmem_wait_ld();
+        const float4 *em4 = reinterpret_cast<const float4 *>(s_em + 64 * khalf + 32 * part);
+        const float g2p[2] = {g2, g2};
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] *= g2 * s_em[64 * khalf + 32 * part + j];
+        for (int y = 0; y < 8; ++y) {  // v (g2 e^m), as in the scalar order
+          const float4 e = em4[y];
+          float sc[4] = {e.x, e.y, e.z, e.w};
+          mul2(&sc[0], g2p, &sc[0]);
+          mul2(&sc[2], g2p, &sc[2]);
+          mul2(&v[4 * y], &v[4 * y], &sc[0]);
+          mul2(&v[4 * y + 2], &v[4 * y + 2], &sc[2]);
+        }
 #pragma unroll
         for (int y = 0; y < 4; ++y) st_s128(dst + sw128(row, 32 * part + 8 * y), pack8(&v[8 * y]));
       }
@@ -572,7 +641,12 @@ __global__ void __launch_bounds__(wy::NT, 2)
           float qm[8], e[8];
           unpack8(ld_s128(blk + 8192 + sw128(row, col)), qm);
 #pragma unroll
-          for (int t = 0; t < 8; ++t) e[t] = (qm[t] - v[8 * y + t]) * s_em[64 * khalf + col + t];
+          for (int t = 0; t < 8; t += 2) {
+            const float2 dq = __fadd2_rn(make_float2(qm[t], qm[t + 1]), make_float2(-v[8 * y + t], -v[8 * y + t + 1]));
+            const float2 r = __fmul2_rn(dq, *reinterpret_cast<const float2 *>(&s_em[64 * khalf + col + t]));
+            e[t] = r.x;
+            e[t + 1] = r.y;
+          }
           st_s128(blk + sw128(row, col), pack8(e));
         }
       }
@@ -699,6 +773,17 @@ __global__ void __launch_bounds__(sp::NT, 1)
   if (warp == W_LOAD) {
     // ---------------------------------------------------------- loads (one thread)
     if (lane == 0) {
+      if (nch > 1) {  // chunk 1 into L2 (chunk 0 is loaded at once; chunks c+2 follow chunk c's load)
+        const int rp = (coff + 1) * a.H + h, tp = (int)(bos + C);
+        tma_prefetch_2d(&tm_wm, 0, rp * 128);
+        tma_prefetch_2d(&tm_wm, 64, rp * 128);
+        tma_prefetch_2d(&tm_wn, 0, rp * 128);
+        tma_prefetch_2d(&tm_wq, 0, rp * 64);
+        tma_prefetch_2d(&tm_wq, 64, rp * 64);
+        tma_prefetch_2d(&tm_wp, 0, rp * 64);
+        tma_prefetch_3d(&tm_v, j0, h, tp);
+        tma_prefetch_3d(&tm_w, j0, h, tp);
+      }
       for (int c = 0; c < nch; ++c) {
         const int s = c & 1;
         // stage s last held chunk c-2: free once its products are complete and its e^{g_C} is read
@@ -723,6 +808,22 @@ __global__ void __launch_bounds__(sp::NT, 1)
           tma_load_3d(st + S_W + vb * 8192, &tm_w, j0 + 64 * vb, h, tok0, full);
         }
         bulk_load(sb + OFF_G + s * REC_G, p.g + (size_t)rec * 128, REC_G, full);
+        if (c + 2 < nch) {  // chunk c+2 into L2, so its load from there is short
+          const int rp = rec + 2 * a.H, tp = tok0 + 2 * C;
+          tma_prefetch_2d(&tm_wm, 0, rp * 128);
+          tma_prefetch_2d(&tm_wm, 64, rp * 128);
+          tma_prefetch_2d(&tm_wn, 0, rp * 128);
+          tma_prefetch_2d(&tm_wq, 0, rp * 64);
+          tma_prefetch_2d(&tm_wq, 64, rp * 64);
+          tma_prefetch_2d(&tm_wp, 0, rp * 64);
+#pragma unroll
+          for (int vb = 0; vb < 2; ++vb)
+            if (j0 + 64 * vb < a.dv) {
+              tma_prefetch_3d(&tm_v, j0 + 64 * vb, h, tp);
+              tma_prefetch_3d(&tm_w, j0 + 64 * vb, h, tp);
+            }
+          bulk_prefetch(p.g + (size_t)rp * 128, REC_G);
+        }
       }
     }
   } else if (warp == W_MMA) {
@@ -841,13 +942,13 @@ __global__ void __launch_bounds__(sp::NT, 1)
           tmem_ld32(tmem + ((uint32_t)(32 * q4) << 16) + TM_D1 + 128 * b + 64 * hf + 32 * part, d);
           tmem_wait_ld();
 #pragma unroll
-          for (int y = 0; y < 8; ++y) {
+          for (int y = 0; y < 8; ++y) {  // S = e^{g_C} S + D1, two channels per packed FMA
             const float4 g = g1[8 * part + y];
             const int i = 32 * part + 4 * y;
-            S[i] = fmaf(g.x, S[i], d[4 * y]);
-            S[i + 1] = fmaf(g.y, S[i + 1], d[4 * y + 1]);
-            S[i + 2] = fmaf(g.z, S[i + 2], d[4 * y + 2]);
-            S[i + 3] = fmaf(g.w, S[i + 3], d[4 * y + 3]);
+            const float2 lo = __ffma2_rn(make_float2(g.x, g.y), make_float2(S[i], S[i + 1]), make_float2(d[4 * y], d[4 * y + 1]));
+            const float2 hi =
+                __ffma2_rn(make_float2(g.z, g.w), make_float2(S[i + 2], S[i + 3]), make_float2(d[4 * y + 2], d[4 * y + 3]));
+            S[i] = lo.x; S[i + 1] = lo.y; S[i + 2] = hi.x; S[i + 3] = hi.y;
           }
         }
       }
@@ -1022,6 +1123,9 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   WyParams p;
   cudaError_t err = device_status_word(&p.status);
   if (err != cudaSuccess) return err;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  p.prefetch_stride = 2 * sms;
   p.N = a.B;
   p.nc = (a.T + C - 1) / C;
   p.tokens = tokens;
