@@ -56,8 +56,6 @@ void note_launch();
 
 // Launchers (return the CUDA error of the launch).
 cudaError_t launch_chunk_simt(const ChunkArgs &a, bool bf16, cudaStream_t stream);
-bool chunk_tc_supported(const ChunkArgs &a, bool bf16);
-cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream);
 // Two-kernel tensor-core path (WY factors of all chunks, then the state pass) over a workspace of
 // chunk_wy_workspace_bytes(...) bytes, 256-byte aligned, that it fully writes before reading.
 // The workspace depends only on the batch shape (B sequences, T tokens each or in total, H heads).
