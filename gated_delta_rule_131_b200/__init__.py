@@ -45,6 +45,8 @@ def lib():
         vp, ci = ctypes.c_void_p, ctypes.c_int
         L.gdn2_chunk_fwd.argtypes = [vp] * 9 + [ci] * 6 + [vp, ci, vp]
         L.gdn2_chunk_fwd.restype = ci
+        L.gdn2_chunk_fwd_noalloc.argtypes = [vp] * 9 + [ci] * 6 + [vp, ci, vp]
+        L.gdn2_chunk_fwd_noalloc.restype = ci
         L.gdn2_decode_step.argtypes = [vp] * 8 + [ci] * 5 + [vp]
         L.gdn2_decode_step.restype = ci
         L.gdn2_status_string.argtypes = [ci]
@@ -107,14 +109,7 @@ def _check_tensors(*ts):
             raise ValueError("gdn2: tensors on different devices")
 
 
-def chunk_fwd(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, chunk=64, o=None, S_T=None,
-              output_final_state=True, stream=None):
-    """Chunkwise forward.  Returns ``(o, S_T)`` (``S_T`` None if not requested).
-
-    Dense: q, k, alpha, b ``[B, T, H, d_k]``; v, w ``[B, T, H, d_v]``.
-    Packed (``cu_seqlens`` int32 ``[N+1]`` on the device): ``[T_total, H, d]``.
-    ``S0`` / ``S_T``: ``[N, H, d_k, d_v]`` float32.
-    """
+def _chunk(entry, q, k, v, alpha, b, w, S0, cu_seqlens, chunk, o, S_T, output_final_state, stream):
     if cu_seqlens is None:
         B, T, H, dk = q.shape
     else:
@@ -132,12 +127,39 @@ def chunk_fwd(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, chunk=64, o=None, 
     if S0 is not None and S0.dtype != torch.float32:
         raise ValueError("gdn2: S0 must be float32")
     _check_tensors(q, k, v, alpha, b, w, S0, o, S_T, cu_seqlens)
-    st = lib().gdn2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0),
-                              _ptr(o), _ptr(S_T), B, T, H, dk, dv, chunk, _ptr(cu_seqlens),
-                              _DTYPES[q.dtype], _stream(stream))
+    fn = getattr(lib(), entry)
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o), _ptr(S_T),
+            B, T, H, dk, dv, chunk, _ptr(cu_seqlens), _DTYPES[q.dtype], _stream(stream))
     if st != GDN2_OK:
-        raise Gdn2Error(st, "gdn2_chunk_fwd")
+        raise Gdn2Error(st, entry)
     return o, S_T
+
+
+def chunk_fwd(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, chunk=64, o=None, S_T=None,
+              output_final_state=True, stream=None):
+    """Chunkwise forward.  Returns ``(o, S_T)`` (``S_T`` None if not requested).
+
+    Dense: q, k, alpha, b ``[B, T, H, d_k]``; v, w ``[B, T, H, d_v]``.
+    Packed (``cu_seqlens`` int32 ``[N+1]`` on the device): ``[T_total, H, d]``.
+    ``S0`` / ``S_T``: ``[N, H, d_k, d_v]`` float32.
+    """
+    return _chunk("gdn2_chunk_fwd", q, k, v, alpha, b, w, S0, cu_seqlens, chunk, o, S_T,
+                  output_final_state, stream)
+
+
+def chunk_fwd_noalloc(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, chunk=64, o=None, S_T=None,
+                      output_final_state=True, stream=None):
+    """``chunk_fwd`` through the library's fixed workspace: the library allocates nothing.
+
+    Shapes whose workspace exceeds ``NOALLOC_WORKSPACE_BYTES`` raise ``Gdn2Error``
+    (``GDN2_ERR_UNSUPPORTED``).  Calls that overlap in time on one device race on the shared
+    workspace; calls on one stream are ordered.
+    """
+    return _chunk("gdn2_chunk_fwd_noalloc", q, k, v, alpha, b, w, S0, cu_seqlens, chunk, o, S_T,
+                  output_final_state, stream)
+
+
+NOALLOC_WORKSPACE_BYTES = 64 << 20  # GDN2_NOALLOC_WORKSPACE_BYTES in include/gdn2.h
 
 
 def decode_step(q, k, v, alpha, b, w, S, o=None, stream=None):

@@ -77,6 +77,28 @@ cudaError_t run_chunk_wy(const gdn2::ChunkArgs &a, cudaStream_t stream) {
   return err;
 }
 
+// The fixed workspace of gdn2_chunk_fwd_noalloc: a file-scope device array, so that entry point
+// allocates nothing.  Its device address is looked up once per device, with that device current.
+constexpr size_t kNoallocBytes = (size_t)GDN2_NOALLOC_WORKSPACE_BYTES;
+static __device__ __align__(256) uint8_t g_noalloc_ws[kNoallocBytes];
+
+cudaError_t noalloc_workspace(void **ptr) {
+  static std::mutex mu;
+  static void *addr[64] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void *a = nullptr;
+    if ((err = cudaGetSymbolAddress(&a, g_noalloc_ws)) != cudaSuccess) return err;
+    addr[dev] = a;
+  }
+  *ptr = addr[dev];
+  return cudaSuccess;
+}
+
 }  // namespace
 
 extern "C" {
@@ -106,10 +128,14 @@ gdn2_status gdn2_device_status(int reset) {
   return st == 0 ? GDN2_OK : GDN2_ERR_TIMEOUT;
 }
 
-gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *alpha,
-                           const void *b, const void *w, const float *S0, void *o, float *S_T,
-                           int B, int T, int H, int d_k, int d_v, int chunk,
-                           const int32_t *cu_seqlens, gdn2_dtype dtype, gdn2_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Validation shared by the chunk entry points; on success fills `a` and `tc` (tensor-core path).
+gdn2_status check_chunk(const void *q, const void *k, const void *v, const void *alpha, const void *b, const void *w,
+                        const float *S0, void *o, float *S_T, int B, int T, int H, int d_k, int d_v, int chunk,
+                        const int32_t *cu_seqlens, gdn2_dtype dtype, gdn2::ChunkArgs *a, bool *tc) {
   if (B < 0 || T < 0 || H <= 0) return GDN2_ERR_INVALID_ARG;
   if (dtype != GDN2_F32 && dtype != GDN2_BF16) return GDN2_ERR_INVALID_ARG;
   // with no tokens at all the token tensors are empty and may be NULL
@@ -123,15 +149,49 @@ gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v, const vo
   const long long tokens = cu_seqlens ? (long long)T : (long long)B * T;
   if (!fits(tokens, H, d_v > d_k ? d_v : d_k, 1) || !fits(B, H, d_k, d_v)) return GDN2_ERR_INVALID_ARG;
   if ((long long)B * H * 8 > INT_MAX) return GDN2_ERR_INVALID_ARG;
-  if (B == 0) return GDN2_OK;
-
-  gdn2::ChunkArgs a{q, k, v, alpha, b, w, S0, o, S_T, cu_seqlens, B, T, H, d_k, d_v};
-  const bool bf16 = dtype == GDN2_BF16;
+  *a = gdn2::ChunkArgs{q, k, v, alpha, b, w, S0, o, S_T, cu_seqlens, B, T, H, d_k, d_v};
   // bf16 with d_k = 128 runs on the tensor cores; fp32 (whose accuracy bf16 operands cannot
   // keep) and d_k = 64 run the SIMT kernel
-  const bool tc = gdn2::chunk_wy_supported(B, T, H, d_k, d_v, cu_seqlens != nullptr, bf16);
+  *tc = gdn2::chunk_wy_supported(B, T, H, d_k, d_v, cu_seqlens != nullptr, dtype == GDN2_BF16);
+  return GDN2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *alpha,
+                           const void *b, const void *w, const float *S0, void *o, float *S_T,
+                           int B, int T, int H, int d_k, int d_v, int chunk,
+                           const int32_t *cu_seqlens, gdn2_dtype dtype, gdn2_stream_t stream) {
+  gdn2::ChunkArgs a;
+  bool tc = false;
+  const gdn2_status st = check_chunk(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, chunk, cu_seqlens, dtype, &a, &tc);
+  if (st != GDN2_OK || B == 0) return st;
   const cudaError_t err = tc ? run_chunk_wy(a, (cudaStream_t)stream)
-                                                            : gdn2::launch_chunk_simt(a, bf16, (cudaStream_t)stream);
+                             : gdn2::launch_chunk_simt(a, dtype == GDN2_BF16, (cudaStream_t)stream);
+  return err == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+}
+
+gdn2_status gdn2_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *alpha,
+                                   const void *b, const void *w, const float *S0, void *o, float *S_T,
+                                   int B, int T, int H, int d_k, int d_v, int chunk,
+                                   const int32_t *cu_seqlens, gdn2_dtype dtype, gdn2_stream_t stream) {
+  gdn2::ChunkArgs a;
+  bool tc = false;
+  const gdn2_status st = check_chunk(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, chunk, cu_seqlens, dtype, &a, &tc);
+  if (st != GDN2_OK || B == 0) return st;
+  if (!tc) {  // the SIMT kernel needs no workspace
+    const cudaError_t err = gdn2::launch_chunk_simt(a, dtype == GDN2_BF16, (cudaStream_t)stream);
+    return err == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+  }
+  // checked on the host before any CUDA call: the shape must fit the fixed workspace
+  if (gdn2::chunk_wy_workspace_bytes(B, T, H, cu_seqlens != nullptr) > kNoallocBytes) return GDN2_ERR_UNSUPPORTED;
+  // nothing in the workspace has to start at zero: the chunk offsets and every record are written
+  // by this call's kernels before they are read
+  void *ws = nullptr;
+  cudaError_t err = noalloc_workspace(&ws);
+  if (err == cudaSuccess) err = gdn2::launch_chunk_wy(a, ws, (cudaStream_t)stream);
   return err == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
 }
 

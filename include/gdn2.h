@@ -109,6 +109,25 @@ GDN2_API gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v,
                            const int32_t *cu_seqlens, gdn2_dtype dtype, gdn2_stream_t stream);
 
 /*
+ * gdn2_chunk_fwd_noalloc -- gdn2_chunk_fwd without any device allocation.
+ *
+ * Same arguments, layouts, results and validation as gdn2_chunk_fwd.  It has no counterpart in the
+ * pages: it exists for callers that must not allocate (CUDA-graph capture without memory nodes,
+ * allocation-free serving loops).  Instead of the pooled workspace it uses one fixed device array of
+ * GDN2_NOALLOC_WORKSPACE_BYTES bytes compiled into the library (its address is looked up once per
+ * device, with that device current).  A tensor-core call (bf16, d_k = 128) whose workspace,
+ * gdn2_chunk_fwd_workspace_bytes(), exceeds that size returns GDN2_ERR_UNSUPPORTED before any CUDA
+ * call; calls that run the SIMT kernel need no workspace and are not limited.  The array is shared:
+ * calls that overlap in time on one device (different streams, or different host threads) race on
+ * it and must not be issued; calls on one stream are ordered and safe.
+ */
+#define GDN2_NOALLOC_WORKSPACE_BYTES (64u << 20) /* 64 MiB */
+GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *alpha,
+                                   const void *b, const void *w, const float *S0, void *o, float *S_T,
+                                   int B, int T, int H, int d_k, int d_v, int chunk,
+                                   const int32_t *cu_seqlens, gdn2_dtype dtype, gdn2_stream_t stream);
+
+/*
  * gdn2_chunk_fwd_workspace_bytes -- device bytes gdn2_chunk_fwd takes from its pool for a call
  * of this shape (packed != 0: a packed batch with cu_seqlens, B sequences, T tokens in total).
  * 0 when the call runs without a workspace or the shape is not supported.  Host only.
