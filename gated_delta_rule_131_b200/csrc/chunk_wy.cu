@@ -586,6 +586,12 @@ __global__ void __launch_bounds__(wy::NT, 2)
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
+  if (tid == 0) {  // Nt, Pt and e^{g_C} are final: store them while round 2 runs
+    tma_store_2d(&tm_wn, 0, rec * 128, sb + OFF_TP);
+    tma_store_2d(&tm_wp, 0, rec * 64, sb + OFF_TS);
+    bulk_store(p.g + (size_t)rec * 128, sb + OFF_SC + 256 * 4, REC_G);
+    bulk_commit();
+  }
 
   // ------------------------------------------------------------ round 2: K_m^T W and [Pt; *] A_m
   // TMEM cols 0..127: K_m^T W; cols 128..255: rows 0..63 Pt A_m (rows 64..127 read whatever follows Pt)
@@ -660,11 +666,8 @@ __global__ void __launch_bounds__(wy::NT, 2)
   if (tid == 0) {
     tma_store_2d(&tm_wm, 0, rec * 128, sb + OFF_KT);
     tma_store_2d(&tm_wm, 64, rec * 128, sb + OFF_AL);
-    tma_store_2d(&tm_wn, 0, rec * 128, sb + OFF_TP);
     tma_store_2d(&tm_wq, 0, rec * 64, sb + OFF_XA);
     tma_store_2d(&tm_wq, 64, rec * 64, sb + OFF_XA + XA_BLK);
-    tma_store_2d(&tm_wp, 0, rec * 64, sb + OFF_TS);
-    bulk_store(p.g + (size_t)rec * 128, sb + OFF_SC + 256 * 4, REC_G);
     bulk_commit();
     bulk_wait_read();
   }
@@ -689,6 +692,7 @@ done:
 // issues the products.
 // Tensor memory is double-buffered per chunk parity, so the U half of D1 and the output of chunk c
 // overlap the state chain, whose step per chunk is: S^T -> TMEM, S^T Mt^T, S update.
+// The two U products share one MMA of N = 192 (Nt and Pt lie back to back in shared memory).
 namespace sp {
 constexpr int VW = 128;        // value columns per CTA
 constexpr int NSTATE = 256;    // warps 0-7
@@ -698,9 +702,9 @@ constexpr int NT = 384;
 constexpr int BAR_STATE = 1;
 // one stage (chunk buffer); every operand tile 1024-aligned
 constexpr uint32_t S_M = 0;                  // Mt: two tiles (input channel blocks), 128 rows each
-constexpr uint32_t S_N = S_M + REC_M;        // 32768: Nt, 128 rows
-constexpr uint32_t S_Q = S_N + REC_N;        // 49152: Qt: two tiles of 64 rows
-constexpr uint32_t S_P = S_Q + REC_Q;        // 65536: Pt, 64 rows
+constexpr uint32_t S_Q = S_M + REC_M;        // 32768: Qt: two tiles of 64 rows
+constexpr uint32_t S_N = S_Q + REC_Q;        // 49152: Nt, 128 rows, and right after it
+constexpr uint32_t S_P = S_N + REC_N;        // 65536: Pt, 64 rows (together one 192-row operand)
 constexpr uint32_t S_V = S_P + REC_P;        // 73728: v -> U = w (.) v: two 64-column tiles of 64 tokens
 constexpr uint32_t S_W = S_V + 16384;        // 90112: w
 constexpr uint32_t STAGE = S_W + 16384;      // 106496
@@ -711,10 +715,11 @@ constexpr uint32_t SMEM_USED = OFF_BAR + 256;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 constexpr uint32_t TX_BYTES = REC_M + REC_N + REC_Q + REC_P + 4 * 8192 + REC_G;
 constexpr uint32_t TMEM_COLS = 512;
-// per buffer b = chunk parity: S^T (bf16 pairs) 64 cols, D1^T 128 cols, O^T 64 cols
-constexpr uint32_t TM_AS = 0, TM_D1 = 128, TM_D2 = 384;
-constexpr uint32_t ID_D1 = idesc_bf16(128, 128, false, false), ID_D1U = idesc_bf16(128, 128, true, false);
-constexpr uint32_t ID_D2 = idesc_bf16(128, 64, false, false), ID_D2U = idesc_bf16(128, 64, true, false);
+// per buffer b = chunk parity (256 columns at 256 b): S^T (bf16 pairs) 64 cols, then D1^T 128 cols
+// and O^T 64 cols side by side, so one MMA of N = 192 writes U^T [Nt^T | Pt^T] into both
+constexpr uint32_t TM_AS = 0, TM_D1 = 64, TM_D2 = 192;
+constexpr uint32_t ID_D1 = idesc_bf16(128, 128, false, false), ID_D2 = idesc_bf16(128, 64, false, false);
+constexpr uint32_t ID_U = idesc_bf16(128, 192, true, false);
 enum {
   B_FULL0 = 0, B_FULL1,      // stage loaded (TMA bytes)
   B_UREADY0, B_UREADY1,      // U formed in the stage (one arrive per U warp)
@@ -832,13 +837,18 @@ __global__ void __launch_bounds__(sp::NT, 1)
       for (int c = 0; c < nch; ++c) {
         const int s = c & 1, b = c & 1, ph = (c >> 1) & 1;
         const uint32_t stg = sb + s * STAGE;
-        const uint32_t as = tmem + TM_AS + 64 * b, d1 = tmem + TM_D1 + 128 * b, d2 = tmem + TM_D2 + 64 * b;
+        const uint32_t as = tmem + 256 * b + TM_AS, d1 = tmem + 256 * b + TM_D1, d2 = tmem + 256 * b + TM_D2;
         if (!mbar_wait_bounded(bar(B_UREADY0 + s), ph, WAIT_NS)) { ok = false; break; }
-        if (c >= 2 && !mbar_wait_bounded(bar(B_D1FREE0 + b), ph ^ 1, WAIT_NS)) { ok = false; break; }
+        // D1 and O^T of this buffer were last read by chunk c-2
+        if (c >= 2 && !(mbar_wait_bounded(bar(B_D1FREE0 + b), ph ^ 1, WAIT_NS) &&
+                        mbar_wait_bounded(bar(B_OSTAGED0 + b), ph ^ 1, WAIT_NS))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < 4; ++k)  // U^T Nt^T, before the state is known
-          mma_bf16(d1, sdesc_sw128(stg + S_V + 2048 * k, 8192, 1024), sdesc_sw128(stg + S_N + 32 * k, 16, 1024), ID_D1U,
+        for (int k = 0; k < 4; ++k)  // U^T [Nt^T | Pt^T], before the state is known
+          mma_bf16(d1, sdesc_sw128(stg + S_V + 2048 * k, 8192, 1024), sdesc_sw128(stg + S_N + 32 * k, 16, 1024), ID_U,
                    k > 0 ? 1u : 0u);
         if (!mbar_wait_bounded(bar(B_SREADY), c & 1, WAIT_NS)) { ok = false; break; }
         tc_fence_after();
@@ -846,15 +856,9 @@ __global__ void __launch_bounds__(sp::NT, 1)
         for (int k = 0; k < DK / 16; ++k)
           mma_bf16_tmem_a(d1, as + 8 * k, sdesc_sw128(stg + S_M + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024), ID_D1, 1u);
         mma_commit(bar(B_D1FULL0 + b));
-        if (c >= 2 && !mbar_wait_bounded(bar(B_OSTAGED0 + b), ph ^ 1, WAIT_NS)) { ok = false; break; }
-        tc_fence_after();
 #pragma unroll
         for (int k = 0; k < DK / 16; ++k)
-          mma_bf16_tmem_a(d2, as + 8 * k, sdesc_sw128(stg + S_Q + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024), ID_D2,
-                          k > 0 ? 1u : 0u);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma_bf16(d2, sdesc_sw128(stg + S_V + 2048 * k, 8192, 1024), sdesc_sw128(stg + S_P + 32 * k, 16, 1024), ID_D2U, 1u);
+          mma_bf16_tmem_a(d2, as + 8 * k, sdesc_sw128(stg + S_Q + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024), ID_D2, 1u);
         mma_commit(bar(B_D2FULL0 + b));
       }
     }
@@ -918,7 +922,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
       uint32_t r[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) r[i] = f2_to_bf2(S[2 * i], S[2 * i + 1]);
-      tmem_st32(tl + TM_AS + 64 * b + 32 * hf, r);
+      tmem_st32(tl + 256 * b + TM_AS + 32 * hf, r);
       tmem_wait_st();
     };
     if (nch > 0) {
@@ -939,7 +943,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
           float d[32];
-          tmem_ld32(tmem + ((uint32_t)(32 * q4) << 16) + TM_D1 + 128 * b + 64 * hf + 32 * part, d);
+          tmem_ld32(tl + 256 * b + TM_D1 + 64 * hf + 32 * part, d);
           tmem_wait_ld();
 #pragma unroll
           for (int y = 0; y < 8; ++y) {  // S = e^{g_C} S + D1, two channels per packed FMA
@@ -965,7 +969,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
       tc_fence_after();
       {
         float d[32];
-        tmem_ld32(tl + TM_D2 + 64 * b + 32 * hf, d);
+        tmem_ld32(tl + 256 * b + TM_D2 + 32 * hf, d);
         tmem_wait_ld();
         if (Cc == C) {  // staged for one TMA store per 64-column tile, once the previous store has read it
           if (c >= 1 && !group_wait(BAR_STATE, NSTATE, bar(B_OFREE), (c - 1) & 1)) { ok = false; break; }
