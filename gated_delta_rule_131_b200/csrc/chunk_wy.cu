@@ -114,10 +114,6 @@ __device__ __forceinline__ bool group_wait(int id, int count, uint32_t bar, uint
   const bool ok = mbar_wait_bounded(bar, parity, WAIT_NS);
   return !group_or(id, count, fail || !ok);
 }
-// The same for one warp.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
-  return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, WAIT_NS));
-}
 
 // D (16 x 8) = A (16 x K) B (K x 8) on the warp-level tensor-core path (mma.sync, tf32 operands
 // rounded from fp32, fp32 accumulate).  A points at element (0, 0) of a row-major fp32 block with
@@ -242,6 +238,7 @@ struct WyParams {
   int64_t tokens;  // rows of the token tensors
   const int32_t *coff;  // packed batch: chunk offsets [N+1]; dense: nullptr
   float *g;             // workspace e^{g_C} [records][128]
+  __nv_bfloat16 *u;     // workspace U = w (.) v, laid out like v
 };
 
 __global__ void __launch_bounds__(wy::NT, 2)
@@ -249,7 +246,8 @@ __global__ void __launch_bounds__(wy::NT, 2)
                      const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_al, const __grid_constant__ CUtensorMap tm_wm,
                      const __grid_constant__ CUtensorMap tm_wn, const __grid_constant__ CUtensorMap tm_wq,
-                     const __grid_constant__ CUtensorMap tm_wp) {
+                     const __grid_constant__ CUtensorMap tm_wp, const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_w) {
   using namespace wy;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -292,6 +290,10 @@ __global__ void __launch_bounds__(wy::NT, 2)
       tma_load_3d(sb + OFF_XA + blk * XA_BLK + 8192, &tm_q, 64 * blk, h, tok0, bar_full);  // q -> rows 64..127
       tma_load_3d(sb + OFF_KT + blk * KT_BLK, &tm_k, 64 * blk, h, tok0, bar_full);
       tma_load_3d(sb + OFF_AL + blk * 8192, &tm_al, 64 * blk, h, tok0, bar_full);
+    }
+    for (int vb = 0; vb < a.dv / 64; ++vb) {  // v and w of this chunk into L2, for U below
+      tma_prefetch_3d(&tm_v, 64 * vb, h, tok0);
+      tma_prefetch_3d(&tm_w, 64 * vb, h, tok0);
     }
     // the record about one wave later (CTAs resident at once = prefetch_stride) into L2
     const int nrec = rec + p.prefetch_stride;
@@ -442,6 +444,36 @@ __global__ void __launch_bounds__(wy::NT, 2)
       mma_bf16(tmem + 0, ad, bd, ID_LP, k > 0 ? 1u : 0u);
     }
     mma_commit(bar_mma);
+  }
+  {  // while M1 runs: U = w (.) v of this chunk's valid tokens -> workspace (16 threads per 256 B)
+    const int per_row = a.dv / 8;  // 16-byte pieces per token row
+    const size_t row0 = ((size_t)tok0 * a.H + h) * (size_t)a.dv, stride = (size_t)a.H * a.dv;
+    const uint4 *vg = reinterpret_cast<const uint4 *>(a.v), *wg = reinterpret_cast<const uint4 *>(a.w);
+    uint4 *ug = reinterpret_cast<uint4 *>(p.u);
+    for (int base = 0; base < Cc * per_row; base += 4 * NT) {
+      uint4 vv[4], ww[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = base + i * NT + tid, r = e / per_row;
+        if (r < Cc) {
+          const size_t off = (row0 + (size_t)r * stride) / 8 + (e % per_row);
+          vv[i] = __ldg(vg + off);
+          ww[i] = __ldg(wg + off);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {  // bf16 x bf16 is exact in fp32: the packed product is the rounded one
+        const int e = base + i * NT + tid, r = e / per_row;
+        if (r < Cc) {
+          uint4 uu;
+          uu.x = bf2_mul(vv[i].x, ww[i].x);
+          uu.y = bf2_mul(vv[i].y, ww[i].y);
+          uu.z = bf2_mul(vv[i].z, ww[i].z);
+          uu.w = bf2_mul(vv[i].w, ww[i].w);
+          ug[(row0 + (size_t)r * stride) / 8 + (e % per_row)] = uu;
+        }
+      }
+    }
   }
   if (!mbar_wait_bounded(bar_mma, 0, WAIT_NS)) ok = false;
   if (__syncthreads_or(!ok)) goto done;
@@ -688,32 +720,30 @@ done:
 //   D1^T = U^T Nt^T + S^T Mt^T   (128 value columns x 128 key channels)
 //   O^T  = S^T Qt^T + U^T Pt^T   (128 value columns x 64 tokens)
 // Roles: warps 0-7 hold the state (thread = value column v, key-channel half hf: S[64 hf ..][v]);
-// warp 8 loads chunks; warps 9-10 form U = w (.) v, and one of their threads stores O; warp 11
-// issues the products.
+// one thread of warp 8 loads chunks (U = w (.) v comes ready-made from the WY kernel); one thread
+// of warp 9 issues the products; one thread of warp 10 stores O.
 // Tensor memory is double-buffered per chunk parity, so the U half of D1 and the output of chunk c
 // overlap the state chain, whose step per chunk is: S^T -> TMEM, S^T Mt^T, S update.
 // The two U products share one MMA of N = 192 (Nt and Pt lie back to back in shared memory).
 namespace sp {
 constexpr int VW = 128;        // value columns per CTA
 constexpr int NSTATE = 256;    // warps 0-7
-constexpr int NU = 64;         // warps 9-10
-constexpr int W_LOAD = 8, W_MMA = 11;
-constexpr int NT = 384;
+constexpr int W_LOAD = 8, W_MMA = 9, W_STORE = 10;
+constexpr int NT = 352;
 constexpr int BAR_STATE = 1;
 // one stage (chunk buffer); every operand tile 1024-aligned
 constexpr uint32_t S_M = 0;                  // Mt: two tiles (input channel blocks), 128 rows each
 constexpr uint32_t S_Q = S_M + REC_M;        // 32768: Qt: two tiles of 64 rows
 constexpr uint32_t S_N = S_Q + REC_Q;        // 49152: Nt, 128 rows, and right after it
 constexpr uint32_t S_P = S_N + REC_N;        // 65536: Pt, 64 rows (together one 192-row operand)
-constexpr uint32_t S_V = S_P + REC_P;        // 73728: v -> U = w (.) v: two 64-column tiles of 64 tokens
-constexpr uint32_t S_W = S_V + 16384;        // 90112: w
-constexpr uint32_t STAGE = S_W + 16384;      // 106496
-constexpr uint32_t OFF_OST = 2 * STAGE;      // 212992: O staging, two 64-column tiles of 64 tokens
-constexpr uint32_t OFF_G = OFF_OST + 16384;  // 229376: e^{g_C} of the two stages
-constexpr uint32_t OFF_BAR = OFF_G + 2 * REC_G;  // 230400
+constexpr uint32_t S_U = S_P + REC_P;        // 73728: U = w (.) v: two 64-column tiles of 64 tokens
+constexpr uint32_t STAGE = S_U + 16384;      // 90112
+constexpr uint32_t OFF_OST = 2 * STAGE;      // 180224: O staging, two 64-column tiles of 64 tokens
+constexpr uint32_t OFF_G = OFF_OST + 16384;  // 196608: e^{g_C} of the two stages
+constexpr uint32_t OFF_BAR = OFF_G + 2 * REC_G;  // 197632
 constexpr uint32_t SMEM_USED = OFF_BAR + 256;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
-constexpr uint32_t TX_BYTES = REC_M + REC_N + REC_Q + REC_P + 4 * 8192 + REC_G;
+constexpr uint32_t TX_BYTES = REC_M + REC_N + REC_Q + REC_P + 2 * 8192 + REC_G;
 constexpr uint32_t TMEM_COLS = 512;
 // per buffer b = chunk parity (256 columns at 256 b): S^T (bf16 pairs) 64 cols, then D1^T 128 cols
 // and O^T 64 cols side by side, so one MMA of N = 192 writes U^T [Nt^T | Pt^T] into both
@@ -722,7 +752,7 @@ constexpr uint32_t ID_D1 = idesc_bf16(128, 128, false, false), ID_D2 = idesc_bf1
 constexpr uint32_t ID_U = idesc_bf16(128, 192, true, false);
 enum {
   B_FULL0 = 0, B_FULL1,      // stage loaded (TMA bytes)
-  B_UREADY0, B_UREADY1,      // U formed in the stage (one arrive per U warp)
+  B_UZERO,                   // rows of U past a sequence's end zeroed (its last, partial chunk) (one arrive per U warp)
   B_SREADY,                  // S^T of the next chunk is in tensor memory
   B_D1FULL0, B_D1FULL1,      // D1 of the buffer complete
   B_D1FREE0, B_D1FREE1,      // D1 of the buffer read by the state warps
@@ -737,8 +767,8 @@ static_assert(SMEM_BYTES <= 232448, "one CTA per SM");
 __global__ void __launch_bounds__(sp::NT, 1)
     state_pass_kernel(const ChunkArgs a, const WyParams p, const __grid_constant__ CUtensorMap tm_wm,
                       const __grid_constant__ CUtensorMap tm_wn, const __grid_constant__ CUtensorMap tm_wq,
-                      const __grid_constant__ CUtensorMap tm_wp, const __grid_constant__ CUtensorMap tm_v,
-                      const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_o) {
+                      const __grid_constant__ CUtensorMap tm_wp, const __grid_constant__ CUtensorMap tm_u,
+                      const __grid_constant__ CUtensorMap tm_o) {
   using namespace sp;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -760,10 +790,10 @@ __global__ void __launch_bounds__(sp::NT, 1)
   auto chunk_len = [&](int c) { return min(C, len - c * C); };
 
   if (tid == 0) {
-    for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), (i == B_UREADY0 || i == B_UREADY1) ? NU / 32 : 1u);
+    for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), 1u);
     fence_mbar_init();
     prefetch_tmap(&tm_wm); prefetch_tmap(&tm_wn); prefetch_tmap(&tm_wq); prefetch_tmap(&tm_wp);
-    prefetch_tmap(&tm_v); prefetch_tmap(&tm_w); prefetch_tmap(&tm_o);
+    prefetch_tmap(&tm_u); prefetch_tmap(&tm_o);
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
@@ -786,8 +816,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
         tma_prefetch_2d(&tm_wq, 0, rp * 64);
         tma_prefetch_2d(&tm_wq, 64, rp * 64);
         tma_prefetch_2d(&tm_wp, 0, rp * 64);
-        tma_prefetch_3d(&tm_v, j0, h, tp);
-        tma_prefetch_3d(&tm_w, j0, h, tp);
+        tma_prefetch_3d(&tm_u, j0, h, tp);
       }
       for (int c = 0; c < nch; ++c) {
         const int s = c & 1;
@@ -808,10 +837,8 @@ __global__ void __launch_bounds__(sp::NT, 1)
         tma_load_2d(st + S_Q + 8192, &tm_wq, 64, rec * 64, full);
         tma_load_2d(st + S_P, &tm_wp, 0, rec * 64, full);
 #pragma unroll
-        for (int vb = 0; vb < 2; ++vb) {  // columns past d_v (d_v = 64) load as zeros
-          tma_load_3d(st + S_V + vb * 8192, &tm_v, j0 + 64 * vb, h, tok0, full);
-          tma_load_3d(st + S_W + vb * 8192, &tm_w, j0 + 64 * vb, h, tok0, full);
-        }
+        for (int vb = 0; vb < 2; ++vb)  // columns past d_v (d_v = 64) load as zeros
+          tma_load_3d(st + S_U + vb * 8192, &tm_u, j0 + 64 * vb, h, tok0, full);
         bulk_load(sb + OFF_G + s * REC_G, p.g + (size_t)rec * 128, REC_G, full);
         if (c + 2 < nch) {  // chunk c+2 into L2, so its load from there is short
           const int rp = rec + 2 * a.H, tp = tok0 + 2 * C;
@@ -823,10 +850,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
           tma_prefetch_2d(&tm_wp, 0, rp * 64);
 #pragma unroll
           for (int vb = 0; vb < 2; ++vb)
-            if (j0 + 64 * vb < a.dv) {
-              tma_prefetch_3d(&tm_v, j0 + 64 * vb, h, tp);
-              tma_prefetch_3d(&tm_w, j0 + 64 * vb, h, tp);
-            }
+            if (j0 + 64 * vb < a.dv) tma_prefetch_3d(&tm_u, j0 + 64 * vb, h, tp);
           bulk_prefetch(p.g + (size_t)rp * 128, REC_G);
         }
       }
@@ -838,7 +862,8 @@ __global__ void __launch_bounds__(sp::NT, 1)
         const int s = c & 1, b = c & 1, ph = (c >> 1) & 1;
         const uint32_t stg = sb + s * STAGE;
         const uint32_t as = tmem + 256 * b + TM_AS, d1 = tmem + 256 * b + TM_D1, d2 = tmem + 256 * b + TM_D2;
-        if (!mbar_wait_bounded(bar(B_UREADY0 + s), ph, WAIT_NS)) { ok = false; break; }
+        if (!mbar_wait_bounded(bar(B_FULL0 + s), ph, WAIT_NS)) { ok = false; break; }
+        if (chunk_len(c) < C && !mbar_wait_bounded(bar(B_UZERO), 0, WAIT_NS)) { ok = false; break; }
         // D1 and O^T of this buffer were last read by chunk c-2
         if (c >= 2 && !(mbar_wait_bounded(bar(B_D1FREE0 + b), ph ^ 1, WAIT_NS) &&
                         mbar_wait_bounded(bar(B_OSTAGED0 + b), ph ^ 1, WAIT_NS))) {
@@ -848,7 +873,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 4; ++k)  // U^T [Nt^T | Pt^T], before the state is known
-          mma_bf16(d1, sdesc_sw128(stg + S_V + 2048 * k, 8192, 1024), sdesc_sw128(stg + S_N + 32 * k, 16, 1024), ID_U,
+          mma_bf16(d1, sdesc_sw128(stg + S_U + 2048 * k, 8192, 1024), sdesc_sw128(stg + S_N + 32 * k, 16, 1024), ID_U,
                    k > 0 ? 1u : 0u);
         if (!mbar_wait_bounded(bar(B_SREADY), c & 1, WAIT_NS)) { ok = false; break; }
         tc_fence_after();
@@ -862,51 +887,22 @@ __global__ void __launch_bounds__(sp::NT, 1)
         mma_commit(bar(B_D2FULL0 + b));
       }
     }
-  } else if (warp > W_LOAD) {
-    // ---------------------------------------------------------- U = w (.) v in place of v; O stores
-    const int u = tid - (W_LOAD + 1) * 32;  // 16 threads per token row, one 8-column chunk each
-    const bool storer = u == NU - 32;       // lane 0 of the second U warp
-    // O of chunk k, staged by the state warps, -> global; then the staging buffer is free
-    auto store_o = [&](int k) {
-      if (!mbar_wait_bounded(bar(B_OSTAGED0 + (k & 1)), (k >> 1) & 1, WAIT_NS)) return false;
-      if (chunk_len(k) == C) {
-        const int tok0 = (int)(bos + (int64_t)k * C);
-        tma_store_3d(&tm_o, j0, h, tok0, sb + OFF_OST);
-        if (j0 + 64 < a.dv) tma_store_3d(&tm_o, j0 + 64, h, tok0, sb + OFF_OST + 8192);
-        bulk_commit();
-        bulk_wait_read();
-      }
-      mbar_arrive(bar(B_OFREE));
-      return true;
-    };
-    for (int c = 0; c < nch; ++c) {
-      const int s = c & 1;
-      const int Cc = chunk_len(c);
-      if (!warp_wait(bar(B_FULL0 + s), (c >> 1) & 1)) { ok = false; break; }
-      uint8_t *vt = sm + s * STAGE + S_V;
-      const uint8_t *wt = sm + s * STAGE + S_W;
-#pragma unroll
-      for (int i = 0; i < 64 * 16 / NU; ++i) {  // rows past the sequence give U = 0
-        const int r = (NU / 16) * i + (u >> 4), x = u & 15;
-        const uint32_t o = (x >> 3) * 8192 + sw128(r, 8 * (x & 7));
-        uint4 uu = make_uint4(0u, 0u, 0u, 0u);
-        if (r < Cc) {  // bf16 x bf16 is exact in fp32, so the packed product is the rounded fp32 one
-          const uint4 vv = ld_s128(vt + o), ww = ld_s128(wt + o);
-          uu.x = bf2_mul(vv.x, ww.x);
-          uu.y = bf2_mul(vv.y, ww.y);
-          uu.z = bf2_mul(vv.z, ww.z);
-          uu.w = bf2_mul(vv.w, ww.w);
+  } else if (warp == W_STORE) {
+    // ---------------------------------------------------------- O stores (one thread)
+    if (lane == 0) {
+      for (int k = 0; k < nch; ++k) {  // O of chunk k, staged by the state warps -> global
+        if (!mbar_wait_bounded(bar(B_OSTAGED0 + (k & 1)), (k >> 1) & 1, WAIT_NS)) { ok = false; break; }
+        if (chunk_len(k) == C) {
+          const int tok0 = (int)(bos + (int64_t)k * C);
+          tma_store_3d(&tm_o, j0, h, tok0, sb + OFF_OST);
+          if (j0 + 64 < a.dv) tma_store_3d(&tm_o, j0 + 64, h, tok0, sb + OFF_OST + 8192);
+          bulk_commit();
+          bulk_wait_read();
         }
-        st_s128(vt + o, uu);
+        mbar_arrive(bar(B_OFREE));  // the staging buffer is free again
       }
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_UREADY0 + s));
-      if (storer && c >= 1 && !store_o(c - 1)) ok = false;
-      if (!__all_sync(0xffffffffu, ok)) break;
     }
-    if (storer && ok && nch > 0 && !store_o(nch - 1)) ok = false;
-  } else {
+  } else if (warp < NSTATE / 32) {
     // ---------------------------------------------------------- state side
     const int q4 = warp & 3, hf = warp >> 2;
     const int v = 32 * q4 + lane;            // value column within the tile (TMEM lane)
@@ -935,6 +931,17 @@ __global__ void __launch_bounds__(sp::NT, 1)
       const int s = c & 1, b = c & 1, ph = (c >> 1) & 1;
       const int Cc = chunk_len(c);
       const int tok0 = (int)(bos + (int64_t)c * C);
+      if (Cc < C) {  // the last chunk: the tile's rows past the sequence hold the next one's U
+        if (!group_wait(BAR_STATE, NSTATE, bar(B_FULL0 + s), ph)) { ok = false; break; }
+        uint8_t *ut = sm + s * STAGE + S_U;
+        for (int e = tid; e < 64 * 16; e += NSTATE) {
+          const int r = e >> 4, x = e & 15;
+          if (r >= Cc) st_s128(ut + (x >> 3) * 8192 + sw128(r, 8 * (x & 7)), make_uint4(0u, 0u, 0u, 0u));
+        }
+        fence_proxy_async();
+        group_sync(BAR_STATE, NSTATE);
+        if (tid == 0) mbar_arrive(bar(B_UZERO));
+      }
       // ---------------------------------------------------------- S <- Diag(e^{g_C}) S + D1
       if (!group_wait(BAR_STATE, NSTATE, bar(B_D1FULL0 + b), ph)) { ok = false; break; }
       tc_fence_after();
@@ -1090,22 +1097,26 @@ long long chunk_capacity(int B, int T, bool packed) {
   return ((long long)T + (long long)(C - 1) * B) / C;
 }
 
-// Workspace layout: Mt tiles | Nt tiles | Qt tiles | Pt tiles | e^{g_C} | chunk offsets (packed only)
+// Workspace layout: Mt tiles | Nt tiles | Qt tiles | Pt tiles | e^{g_C} | U (like v) | chunk offsets
+// (packed only); every array starts on a 256-byte boundary
 struct WsLayout {
   long long records;
-  size_t m, n, q, p, g, coff, total;
+  size_t m, n, q, p, g, u, coff, total;
 };
-WsLayout ws_layout(int B, int T, int H, bool packed) {
+size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+WsLayout ws_layout(int B, int T, int H, int dv, bool packed) {
   WsLayout L{};
   L.records = chunk_capacity(B, T, packed) * H;
   const size_t r = (size_t)L.records;
+  const size_t tokens = packed ? (size_t)T : (size_t)B * T;
   L.m = 0;
   L.n = L.m + r * REC_M;
   L.q = L.n + r * REC_N;
   L.p = L.q + r * REC_Q;
   L.g = L.p + r * REC_P;
-  L.coff = L.g + r * REC_G;
-  L.total = L.coff + (packed ? ((size_t)(B + 1) * 4 + 255) / 256 * 256 : 0);
+  L.u = up256(L.g + r * REC_G);
+  L.coff = up256(L.u + tokens * H * dv * 2);
+  L.total = L.coff + (packed ? up256((size_t)(B + 1) * 4) : 0);
   return L;
 }
 
@@ -1118,11 +1129,13 @@ bool chunk_wy_supported(int B, int T, int H, int dk, int dv, bool packed, bool b
   return tokens + C <= (long long)INT_MAX && chunk_capacity(B, T, packed) * H * 128 <= (long long)INT_MAX;
 }
 
-size_t chunk_wy_workspace_bytes(int B, int T, int H, bool packed) { return ws_layout(B, T, H, packed).total; }
+size_t chunk_wy_workspace_bytes(int B, int T, int H, int dv, bool packed) {
+  return ws_layout(B, T, H, dv, packed).total;
+}
 
 cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   const long long tokens = a.cu ? (long long)a.T : (long long)a.B * a.T;
-  const WsLayout L = ws_layout(a.B, a.T, a.H, a.cu != nullptr);
+  const WsLayout L = ws_layout(a.B, a.T, a.H, a.dv, a.cu != nullptr);
   uint8_t *base = static_cast<uint8_t *>(ws);
   WyParams p;
   cudaError_t err = device_status_word(&p.status);
@@ -1135,13 +1148,14 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   p.tokens = tokens;
   p.coff = a.cu ? reinterpret_cast<const int32_t *>(base + L.coff) : nullptr;
   p.g = reinterpret_cast<float *>(base + L.g);
+  p.u = reinterpret_cast<__nv_bfloat16 *>(base + L.u);
 
-  CUtensorMap mq, mk, mb, mal, mv, mw, mo, mm, mn, mqt, mp;
+  CUtensorMap mq, mk, mb, mal, mv, mw, mu, mo, mm, mn, mqt, mp;
   if (tokens > 0) {
     if (!map_tokens(&mq, a.q, tokens, a.H, DK) || !map_tokens(&mk, a.k, tokens, a.H, DK) ||
         !map_tokens(&mb, a.b, tokens, a.H, DK) || !map_tokens(&mal, a.alpha, tokens, a.H, DK) ||
         !map_tokens(&mv, a.v, tokens, a.H, a.dv) || !map_tokens(&mw, a.w, tokens, a.H, a.dv) ||
-        !map_tokens(&mo, a.o, tokens, a.H, a.dv) ||
+        !map_tokens(&mo, a.o, tokens, a.H, a.dv) || !map_tokens(&mu, base + L.u, tokens, a.H, a.dv) ||
         !map_matrix(&mm, base + L.m, L.records * 128, 128, 128) ||
         !map_matrix(&mn, base + L.n, L.records * 128, 64, 128) ||
         !map_matrix(&mqt, base + L.q, L.records * 64, 128, 64) ||
@@ -1150,7 +1164,7 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   } else {
     // no token and no record: the state pass only copies S0 to S_T; its maps are never read
     memset(&mv, 0, sizeof(mv));
-    mw = mo = mm = mn = mqt = mp = mv;
+    mw = mu = mo = mm = mn = mqt = mp = mv;
   }
   if (a.cu) {
     note_launch();
@@ -1161,14 +1175,15 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
     err = cudaFuncSetAttribute(wy_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wy::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     note_launch();
-    wy_factor_kernel<<<(unsigned)L.records, wy::NT, wy::SMEM_BYTES, stream>>>(a, p, mq, mk, mb, mal, mm, mn, mqt, mp);
+    wy_factor_kernel<<<(unsigned)L.records, wy::NT, wy::SMEM_BYTES, stream>>>(a, p, mq, mk, mb, mal, mm, mn, mqt, mp, mv,
+                                                                              mw);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   const long long blocks = (long long)a.B * a.H * ((a.dv + sp::VW - 1) / sp::VW);
   err = cudaFuncSetAttribute(state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp::SMEM_BYTES);
   if (err != cudaSuccess) return err;
   note_launch();
-  state_pass_kernel<<<(unsigned)blocks, sp::NT, sp::SMEM_BYTES, stream>>>(a, p, mm, mn, mqt, mp, mv, mw, mo);
+  state_pass_kernel<<<(unsigned)blocks, sp::NT, sp::SMEM_BYTES, stream>>>(a, p, mm, mn, mqt, mp, mu, mo);
   return cudaGetLastError();
 }
 

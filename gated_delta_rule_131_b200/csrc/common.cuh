@@ -58,9 +58,9 @@ void note_launch();
 cudaError_t launch_chunk_simt(const ChunkArgs &a, bool bf16, cudaStream_t stream);
 // Two-kernel tensor-core path (WY factors of all chunks, then the state pass) over a workspace of
 // chunk_wy_workspace_bytes(...) bytes, 256-byte aligned, that it fully writes before reading.
-// The workspace depends only on the batch shape (B sequences, T tokens each or in total, H heads).
+// The workspace depends only on the batch shape (B sequences, T tokens each or in total, H heads, d_v).
 bool chunk_wy_supported(int B, int T, int H, int dk, int dv, bool packed, bool bf16);
-size_t chunk_wy_workspace_bytes(int B, int T, int H, bool packed);
+size_t chunk_wy_workspace_bytes(int B, int T, int H, int dv, bool packed);
 cudaError_t launch_chunk_wy(const ChunkArgs &a, void *workspace, cudaStream_t stream);
 cudaError_t launch_bounded_wait_probe(uint64_t limit_ns, cudaStream_t stream);
 // Reads (and optionally clears) the device-side status word that bounded waits set.

@@ -61,7 +61,7 @@ cudaError_t workspace_pool(cudaMemPool_t *pool) {
 
 // The tensor-core path with a workspace taken from the pool and returned to it on `stream`.
 cudaError_t run_chunk_wy(const gdn2::ChunkArgs &a, cudaStream_t stream) {
-  const size_t bytes = gdn2::chunk_wy_workspace_bytes(a.B, a.T, a.H, a.cu != nullptr);
+  const size_t bytes = gdn2::chunk_wy_workspace_bytes(a.B, a.T, a.H, a.dv, a.cu != nullptr);
   void *ws = nullptr;
   cudaError_t err;
   if (bytes > 0) {
@@ -186,7 +186,7 @@ gdn2_status gdn2_chunk_fwd_noalloc(const void *q, const void *k, const void *v, 
     return err == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
   }
   // checked on the host before any CUDA call: the shape must fit the fixed workspace
-  if (gdn2::chunk_wy_workspace_bytes(B, T, H, cu_seqlens != nullptr) > kNoallocBytes) return GDN2_ERR_UNSUPPORTED;
+  if (gdn2::chunk_wy_workspace_bytes(B, T, H, d_v, cu_seqlens != nullptr) > kNoallocBytes) return GDN2_ERR_UNSUPPORTED;
   // nothing in the workspace has to start at zero: the chunk offsets and every record are written
   // by this call's kernels before they are read
   void *ws = nullptr;
@@ -200,7 +200,7 @@ size_t gdn2_chunk_fwd_workspace_bytes(int B, int T, int H, int d_k, int d_v, int
   if (B <= 0 || T < 0 || H <= 0 || chunk != 64 || !supported_dk(d_k) || !supported_dv(d_v)) return 0;
   if (dtype != GDN2_F32 && dtype != GDN2_BF16) return 0;
   if (!gdn2::chunk_wy_supported(B, T, H, d_k, d_v, packed != 0, dtype == GDN2_BF16)) return 0;
-  return gdn2::chunk_wy_workspace_bytes(B, T, H, packed != 0);
+  return gdn2::chunk_wy_workspace_bytes(B, T, H, d_v, packed != 0);
 }
 
 gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v, const void *alpha,
