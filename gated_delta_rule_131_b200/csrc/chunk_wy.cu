@@ -743,13 +743,12 @@ constexpr uint32_t OFF_G = OFF_OST + 16384;  // 196608: e^{g_C} of the two stage
 constexpr uint32_t OFF_BAR = OFF_G + 2 * REC_G;  // 197632
 constexpr uint32_t SMEM_USED = OFF_BAR + 256;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
-constexpr uint32_t TX_BYTES = REC_M + REC_N + REC_Q + REC_P + 2 * 8192 + REC_G;
 constexpr uint32_t TMEM_COLS = 512;
 // per buffer b = chunk parity (256 columns at 256 b): S^T (bf16 pairs) 64 cols, then D1^T 128 cols
 // and O^T 64 cols side by side, so one MMA of N = 192 writes U^T [Nt^T | Pt^T] into both
 constexpr uint32_t TM_AS = 0, TM_D1 = 64, TM_D2 = 192;
 constexpr uint32_t ID_D1 = idesc_bf16(128, 128, false, false), ID_D2 = idesc_bf16(128, 64, false, false);
-constexpr uint32_t ID_U = idesc_bf16(128, 192, true, false);
+constexpr uint32_t ID_U = idesc_bf16(128, 192, true, false), ID_U1 = idesc_bf16(128, 128, true, false);
 enum {
   B_FULL0 = 0, B_FULL1,      // stage loaded (TMA bytes)
   B_UZERO,                   // rows of U past a sequence's end zeroed (its last, partial chunk) (one arrive per U warp)
@@ -764,8 +763,23 @@ enum {
 static_assert(SMEM_BYTES <= 232448, "one CTA per SM");
 }  // namespace sp
 
+// How one state-pass CTA is placed and what it produces.  Mode 0 walks whole sequences.  For long
+// sequences with few heads the walk is split into segments of `seg_len` chunks (two-level scan):
+// mode 1 summarises every segment but the last as an affine map X -> A_j X + B_j of the entering
+// state (A_j from the identity without U, B_j from zero, or from S0 for j = 0, with U); after the
+// combine kernel has chained the maps into each segment's entry state, mode 2 walks every segment
+// from its entry state and writes O (and S_T after the last).
+struct ScanParams {
+  int mode;        // 0 whole sequences, 1 segment summaries, 2 segments from their entry states
+  int seg_len;     // chunks per segment (modes 1, 2)
+  int nseg;        // segments per sequence (modes 1, 2; dense batches only)
+  float *sum_a;    // [N][H][nseg-1][128][128]: A_j (mode 1)
+  float *sum_b;    // [N][H][nseg-1][128][d_v]: B_j (mode 1)
+  float *s_start;  // [N][H][nseg][128][d_v]: entry state of segment j >= 1 (mode 2)
+};
+
 __global__ void __launch_bounds__(sp::NT, 1)
-    state_pass_kernel(const ChunkArgs a, const WyParams p, const __grid_constant__ CUtensorMap tm_wm,
+    state_pass_kernel(const ChunkArgs a, const WyParams p, const ScanParams q, const __grid_constant__ CUtensorMap tm_wm,
                       const __grid_constant__ CUtensorMap tm_wn, const __grid_constant__ CUtensorMap tm_wq,
                       const __grid_constant__ CUtensorMap tm_wp, const __grid_constant__ CUtensorMap tm_u,
                       const __grid_constant__ CUtensorMap tm_o) {
@@ -777,17 +791,42 @@ __global__ void __launch_bounds__(sp::NT, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 8 * B_COUNT);
   auto bar = [&](int i) { return sb + OFF_BAR + 8u * (uint32_t)i; };
 
+  // ------------------------------------------------------------ placement
   const int tiles = (a.dv + VW - 1) / VW;
-  const int tile = blockIdx.x % tiles;
-  const int h = (blockIdx.x / tiles) % a.H;
-  const int n = blockIdx.x / (tiles * a.H);
+  int n, h, tile = 0, seg = 0;
+  bool ident = false;  // mode 1, A_j: the state starts as the identity and U is left out
+  if (q.mode == 1) {
+    const int per = 1 + tiles;  // A_j, then one CTA per value tile for B_j
+    const int t = blockIdx.x % per;
+    seg = (blockIdx.x / per) % (q.nseg - 1);
+    h = (blockIdx.x / (per * (q.nseg - 1))) % a.H;
+    n = blockIdx.x / (per * (q.nseg - 1) * a.H);
+    ident = t == 0;
+    tile = ident ? 0 : t - 1;
+    if (ident && seg == 0) return;  // segment 0 starts from S0: its end state is all that is needed
+  } else if (q.mode == 2) {
+    tile = blockIdx.x % tiles;
+    seg = (blockIdx.x / tiles) % q.nseg;
+    h = (blockIdx.x / (tiles * q.nseg)) % a.H;
+    n = blockIdx.x / (tiles * q.nseg * a.H);
+  } else {
+    tile = blockIdx.x % tiles;
+    h = (blockIdx.x / tiles) % a.H;
+    n = blockIdx.x / (tiles * a.H);
+  }
   const int j0 = tile * VW;
+  const int cols = ident ? DK : a.dv;  // column count of the state this CTA carries
+  const bool use_u = !ident, use_o = q.mode != 1;
   int64_t bos;
   int len;
   seq_span(a, n, bos, len);
   const int nch = (len + C - 1) / C;
+  const int cb = q.mode == 0 ? 0 : seg * q.seg_len;
+  const int ce = q.mode == 0 ? nch : min(nch, cb + q.seg_len);
+  const int nk = max(ce - cb, 0);  // chunks of this CTA, local index k -> chunk cb + k
   const int coff = p.coff ? p.coff[n] : n * p.nc;  // global chunk of this sequence's chunk 0
   auto chunk_len = [&](int c) { return min(C, len - c * C); };
+  const uint32_t tx_bytes = REC_M + REC_G + (use_u ? REC_N + 2 * 8192 : 0) + (use_o ? REC_Q + REC_P : 0);
 
   if (tid == 0) {
     for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), 1u);
@@ -808,92 +847,98 @@ __global__ void __launch_bounds__(sp::NT, 1)
   if (warp == W_LOAD) {
     // ---------------------------------------------------------- loads (one thread)
     if (lane == 0) {
-      if (nch > 1) {  // chunk 1 into L2 (chunk 0 is loaded at once; chunks c+2 follow chunk c's load)
-        const int rp = (coff + 1) * a.H + h, tp = (int)(bos + C);
+      auto prefetch = [&](int c) {  // chunk c into L2, so its later load from there is short
+        const int rp = (coff + c) * a.H + h, tp = (int)(bos + (int64_t)c * C);
         tma_prefetch_2d(&tm_wm, 0, rp * 128);
         tma_prefetch_2d(&tm_wm, 64, rp * 128);
-        tma_prefetch_2d(&tm_wn, 0, rp * 128);
-        tma_prefetch_2d(&tm_wq, 0, rp * 64);
-        tma_prefetch_2d(&tm_wq, 64, rp * 64);
-        tma_prefetch_2d(&tm_wp, 0, rp * 64);
-        tma_prefetch_3d(&tm_u, j0, h, tp);
-      }
-      for (int c = 0; c < nch; ++c) {
-        const int s = c & 1;
-        // stage s last held chunk c-2: free once its products are complete and its e^{g_C} is read
-        if (c >= 2 && !(mbar_wait_bounded(bar(B_D2FULL0 + s), ((c - 2) >> 1) & 1, WAIT_NS) &&
-                        mbar_wait_bounded(bar(B_D1FREE0 + s), ((c - 2) >> 1) & 1, WAIT_NS))) {
+        if (use_u) {
+          tma_prefetch_2d(&tm_wn, 0, rp * 128);
+#pragma unroll
+          for (int vb = 0; vb < 2; ++vb)
+            if (j0 + 64 * vb < a.dv) tma_prefetch_3d(&tm_u, j0 + 64 * vb, h, tp);
+        }
+        if (use_o) {
+          tma_prefetch_2d(&tm_wq, 0, rp * 64);
+          tma_prefetch_2d(&tm_wq, 64, rp * 64);
+          tma_prefetch_2d(&tm_wp, 0, rp * 64);
+        }
+        bulk_prefetch(p.g + (size_t)rp * 128, REC_G);
+      };
+      if (nk > 1) prefetch(cb + 1);  // chunk cb is loaded at once; chunk c+2 follows chunk c's load
+      for (int k = 0; k < nk; ++k) {
+        const int s = k & 1, c = cb + k;
+        // stage s last held chunk k-2: free once its products are complete and its e^{g_C} is read
+        if (k >= 2 && !(mbar_wait_bounded(bar(B_D2FULL0 + s), ((k - 2) >> 1) & 1, WAIT_NS) &&
+                        mbar_wait_bounded(bar(B_D1FREE0 + s), ((k - 2) >> 1) & 1, WAIT_NS))) {
           ok = false;
           break;
         }
         const uint32_t st = sb + s * STAGE, full = bar(B_FULL0 + s);
         const int rec = (coff + c) * a.H + h;
         const int tok0 = (int)(bos + (int64_t)c * C);
-        mbar_expect_tx(full, TX_BYTES);
+        mbar_expect_tx(full, tx_bytes);
         tma_load_2d(st + S_M, &tm_wm, 0, rec * 128, full);
         tma_load_2d(st + S_M + 16384, &tm_wm, 64, rec * 128, full);
-        tma_load_2d(st + S_N, &tm_wn, 0, rec * 128, full);
-        tma_load_2d(st + S_Q, &tm_wq, 0, rec * 64, full);
-        tma_load_2d(st + S_Q + 8192, &tm_wq, 64, rec * 64, full);
-        tma_load_2d(st + S_P, &tm_wp, 0, rec * 64, full);
+        if (use_u) {
+          tma_load_2d(st + S_N, &tm_wn, 0, rec * 128, full);
 #pragma unroll
-        for (int vb = 0; vb < 2; ++vb)  // columns past d_v (d_v = 64) load as zeros
-          tma_load_3d(st + S_U + vb * 8192, &tm_u, j0 + 64 * vb, h, tok0, full);
-        bulk_load(sb + OFF_G + s * REC_G, p.g + (size_t)rec * 128, REC_G, full);
-        if (c + 2 < nch) {  // chunk c+2 into L2, so its load from there is short
-          const int rp = rec + 2 * a.H, tp = tok0 + 2 * C;
-          tma_prefetch_2d(&tm_wm, 0, rp * 128);
-          tma_prefetch_2d(&tm_wm, 64, rp * 128);
-          tma_prefetch_2d(&tm_wn, 0, rp * 128);
-          tma_prefetch_2d(&tm_wq, 0, rp * 64);
-          tma_prefetch_2d(&tm_wq, 64, rp * 64);
-          tma_prefetch_2d(&tm_wp, 0, rp * 64);
-#pragma unroll
-          for (int vb = 0; vb < 2; ++vb)
-            if (j0 + 64 * vb < a.dv) tma_prefetch_3d(&tm_u, j0 + 64 * vb, h, tp);
-          bulk_prefetch(p.g + (size_t)rp * 128, REC_G);
+          for (int vb = 0; vb < 2; ++vb)  // columns past d_v (d_v = 64) load as zeros
+            tma_load_3d(st + S_U + vb * 8192, &tm_u, j0 + 64 * vb, h, tok0, full);
         }
+        if (use_o) {
+          tma_load_2d(st + S_Q, &tm_wq, 0, rec * 64, full);
+          tma_load_2d(st + S_Q + 8192, &tm_wq, 64, rec * 64, full);
+          tma_load_2d(st + S_P, &tm_wp, 0, rec * 64, full);
+        }
+        bulk_load(sb + OFF_G + s * REC_G, p.g + (size_t)rec * 128, REC_G, full);
+        if (k + 2 < nk) prefetch(c + 2);
       }
     }
   } else if (warp == W_MMA) {
     // ---------------------------------------------------------- products (one thread)
     if (lane == 0) {
-      for (int c = 0; c < nch; ++c) {
-        const int s = c & 1, b = c & 1, ph = (c >> 1) & 1;
+      for (int k = 0; k < nk; ++k) {
+        const int s = k & 1, b = k & 1, ph = (k >> 1) & 1, c = cb + k;
         const uint32_t stg = sb + s * STAGE;
         const uint32_t as = tmem + 256 * b + TM_AS, d1 = tmem + 256 * b + TM_D1, d2 = tmem + 256 * b + TM_D2;
         if (!mbar_wait_bounded(bar(B_FULL0 + s), ph, WAIT_NS)) { ok = false; break; }
-        if (chunk_len(c) < C && !mbar_wait_bounded(bar(B_UZERO), 0, WAIT_NS)) { ok = false; break; }
-        // D1 and O^T of this buffer were last read by chunk c-2
-        if (c >= 2 && !(mbar_wait_bounded(bar(B_D1FREE0 + b), ph ^ 1, WAIT_NS) &&
+        if (use_u && chunk_len(c) < C && !mbar_wait_bounded(bar(B_UZERO), 0, WAIT_NS)) { ok = false; break; }
+        // D1 and O^T of this buffer were last read by chunk k-2
+        if (k >= 2 && !(mbar_wait_bounded(bar(B_D1FREE0 + b), ph ^ 1, WAIT_NS) &&
                         mbar_wait_bounded(bar(B_OSTAGED0 + b), ph ^ 1, WAIT_NS))) {
           ok = false;
           break;
         }
         tc_fence_after();
+        if (use_u) {  // U^T Nt^T (and U^T Pt^T for the output), before the state is known
 #pragma unroll
-        for (int k = 0; k < 4; ++k)  // U^T [Nt^T | Pt^T], before the state is known
-          mma_bf16(d1, sdesc_sw128(stg + S_U + 2048 * k, 8192, 1024), sdesc_sw128(stg + S_N + 32 * k, 16, 1024), ID_U,
-                   k > 0 ? 1u : 0u);
-        if (!mbar_wait_bounded(bar(B_SREADY), c & 1, WAIT_NS)) { ok = false; break; }
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(d1, sdesc_sw128(stg + S_U + 2048 * kk, 8192, 1024), sdesc_sw128(stg + S_N + 32 * kk, 16, 1024),
+                     use_o ? ID_U : ID_U1, kk > 0 ? 1u : 0u);
+        }
+        if (!mbar_wait_bounded(bar(B_SREADY), k & 1, WAIT_NS)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < DK / 16; ++k)
-          mma_bf16_tmem_a(d1, as + 8 * k, sdesc_sw128(stg + S_M + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024), ID_D1, 1u);
+        for (int kk = 0; kk < DK / 16; ++kk)
+          mma_bf16_tmem_a(d1, as + 8 * kk, sdesc_sw128(stg + S_M + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), ID_D1,
+                          (use_u || kk > 0) ? 1u : 0u);
         mma_commit(bar(B_D1FULL0 + b));
+        if (use_o) {
 #pragma unroll
-        for (int k = 0; k < DK / 16; ++k)
-          mma_bf16_tmem_a(d2, as + 8 * k, sdesc_sw128(stg + S_Q + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024), ID_D2, 1u);
-        mma_commit(bar(B_D2FULL0 + b));
+          for (int kk = 0; kk < DK / 16; ++kk)
+            mma_bf16_tmem_a(d2, as + 8 * kk, sdesc_sw128(stg + S_Q + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), ID_D2,
+                            1u);
+        }
+        mma_commit(bar(B_D2FULL0 + b));  // with no output products this completes with D1
       }
     }
   } else if (warp == W_STORE) {
     // ---------------------------------------------------------- O stores (one thread)
-    if (lane == 0) {
-      for (int k = 0; k < nch; ++k) {  // O of chunk k, staged by the state warps -> global
+    if (lane == 0 && use_o) {
+      for (int k = 0; k < nk; ++k) {  // O of chunk cb + k, staged by the state warps -> global
         if (!mbar_wait_bounded(bar(B_OSTAGED0 + (k & 1)), (k >> 1) & 1, WAIT_NS)) { ok = false; break; }
-        if (chunk_len(k) == C) {
-          const int tok0 = (int)(bos + (int64_t)k * C);
+        if (chunk_len(cb + k) == C) {
+          const int tok0 = (int)(bos + (int64_t)(cb + k) * C);
           tma_store_3d(&tm_o, j0, h, tok0, sb + OFF_OST);
           if (j0 + 64 < a.dv) tma_store_3d(&tm_o, j0 + 64, h, tok0, sb + OFF_OST + 8192);
           bulk_commit();
@@ -905,13 +950,26 @@ __global__ void __launch_bounds__(sp::NT, 1)
   } else if (warp < NSTATE / 32) {
     // ---------------------------------------------------------- state side
     const int q4 = warp & 3, hf = warp >> 2;
-    const int v = 32 * q4 + lane;            // value column within the tile (TMEM lane)
-    const bool vin = j0 + v < a.dv;
+    const int v = 32 * q4 + lane;            // column within the tile (TMEM lane)
+    const bool vin = j0 + v < cols;
     const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
-    const size_t s_base = (((size_t)n * a.H + h) * DK + 64 * hf) * (size_t)a.dv + j0 + v;  // S[64 hf][j0 + v]
+    const size_t nh = (size_t)n * a.H + h;
+    // S[64 hf + i][j0 + v] lives at base + i * cols in every [.., 128, cols] state array
+    const size_t s_base = (nh * DK + 64 * hf) * (size_t)a.dv + j0 + v;
     float S[64];
+    {
+      const float *src = nullptr;
+      size_t base = s_base, ld = (size_t)a.dv;
+      if (q.mode == 2) {  // every segment, the first included, starts from its entry state (S_T may alias S0)
+        src = q.s_start;
+        base = ((nh * q.nseg + seg) * DK + 64 * hf) * (size_t)a.dv + j0 + v;
+      } else if (!ident && seg == 0) {
+        src = a.S0;
+      }
 #pragma unroll
-    for (int i = 0; i < 64; ++i) S[i] = (a.S0 && vin) ? a.S0[s_base + (size_t)i * a.dv] : 0.f;
+      for (int i = 0; i < 64; ++i)
+        S[i] = ident ? (64 * hf + i == v ? 1.f : 0.f) : ((src && vin) ? src[base + (size_t)i * ld] : 0.f);
+    }
     __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o);
     // S^T of the chunk about to start -> tensor memory buffer b (bf16 pairs); signals the issuer
     auto put_state = [&](int b) {
@@ -921,17 +979,17 @@ __global__ void __launch_bounds__(sp::NT, 1)
       tmem_st32(tl + 256 * b + TM_AS + 32 * hf, r);
       tmem_wait_st();
     };
-    if (nch > 0) {
+    if (nk > 0) {
       put_state(0);
       tc_fence_before();
       group_sync(BAR_STATE, NSTATE);
       if (tid == 0) mbar_arrive(bar(B_SREADY));
     }
-    for (int c = 0; c < nch; ++c) {
-      const int s = c & 1, b = c & 1, ph = (c >> 1) & 1;
+    for (int k = 0; k < nk; ++k) {
+      const int s = k & 1, b = k & 1, ph = (k >> 1) & 1, c = cb + k;
       const int Cc = chunk_len(c);
       const int tok0 = (int)(bos + (int64_t)c * C);
-      if (Cc < C) {  // the last chunk: the tile's rows past the sequence hold the next one's U
+      if (use_u && Cc < C) {  // the last chunk: the tile's rows past the sequence hold the next one's U
         if (!group_wait(BAR_STATE, NSTATE, bar(B_FULL0 + s), ph)) { ok = false; break; }
         uint8_t *ut = sm + s * STAGE + S_U;
         for (int e = tid; e < 64 * 16; e += NSTATE) {
@@ -963,14 +1021,16 @@ __global__ void __launch_bounds__(sp::NT, 1)
           }
         }
       }
-      // the next chunk's S^T goes into the other buffer (its last reader, O^T of chunk c-1, is complete)
-      if (c + 1 < nch) put_state(b ^ 1);
+      // the next chunk's S^T goes into the other buffer (its last reader, O^T of chunk k-1, is complete)
+      if (k + 1 < nk) put_state(b ^ 1);
       tc_fence_before();
       group_sync(BAR_STATE, NSTATE);
       if (tid == 0) {
         mbar_arrive(bar(B_D1FREE0 + b));
-        if (c + 1 < nch) mbar_arrive(bar(B_SREADY));
+        if (k + 1 < nk) mbar_arrive(bar(B_SREADY));
+        if (!use_o) mbar_arrive(bar(B_OSTAGED0 + s));
       }
+      if (!use_o) continue;
       // ---------------------------------------------------------- O: tokens 32 hf .. 32 hf + 31 of column v
       if (!group_wait(BAR_STATE, NSTATE, bar(B_D2FULL0 + b), ph)) { ok = false; break; }
       tc_fence_after();
@@ -979,7 +1039,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
         tmem_ld32(tl + 256 * b + TM_D2 + 32 * hf, d);
         tmem_wait_ld();
         if (Cc == C) {  // staged for one TMA store per 64-column tile, once the previous store has read it
-          if (c >= 1 && !group_wait(BAR_STATE, NSTATE, bar(B_OFREE), (c - 1) & 1)) { ok = false; break; }
+          if (k >= 1 && !group_wait(BAR_STATE, NSTATE, bar(B_OFREE), (k - 1) & 1)) { ok = false; break; }
           uint8_t *ot = sm + OFF_OST + (v >> 6) * 8192;
 #pragma unroll
           for (int j = 0; j < 32; ++j)
@@ -996,9 +1056,21 @@ __global__ void __launch_bounds__(sp::NT, 1)
       group_sync(BAR_STATE, NSTATE);
       if (tid == 0) mbar_arrive(bar(B_OSTAGED0 + s));
     }
-    if (ok && a.ST && vin) {
+    // ---------------------------------------------------------- the state after this CTA's chunks
+    if (ok && vin) {
+      float *dst = nullptr;
+      size_t base = s_base;
+      if (q.mode == 1) {
+        const size_t js = nh * (q.nseg - 1) + seg;
+        dst = ident ? q.sum_a : q.sum_b;
+        base = (js * DK + 64 * hf) * (size_t)cols + j0 + v;
+      } else if (q.mode == 0 || seg == q.nseg - 1) {
+        dst = a.ST;
+      }
+      if (dst) {
 #pragma unroll
-      for (int i = 0; i < 64; ++i) a.ST[s_base + (size_t)i * a.dv] = S[i];
+        for (int i = 0; i < 64; ++i) dst[base + (size_t)i * cols] = S[i];
+      }
     }
   }
   if (!ok) atomicExch(p.status, 4);
@@ -1007,6 +1079,73 @@ __global__ void __launch_bounds__(sp::NT, 1)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// Two-level scan, between the two state passes: chains the segment maps into entry states,
+// E_0 = S0, E_1 = B_0 and E_{j+1} = A_j E_j + B_j (fp32), one CTA per (sequence, head, 128 value
+// columns).  E_0 is copied too, so the final pass never reads S0 while its last segment writes S_T.
+__global__ void __launch_bounds__(256) segment_chain_kernel(const ChunkArgs a, const ScanParams q) {
+  extern __shared__ float csm[];
+  float *E = csm;                 // [128][128 + 4] entry state, columns of this tile
+  float *At = csm + 128 * 132;    // [32][128 + 4] a slab of A_j, transposed (k rows, i columns)
+  const int tiles = (a.dv + 127) / 128;
+  const int tile = blockIdx.x % tiles, h = (blockIdx.x / tiles) % a.H, n = blockIdx.x / (tiles * a.H);
+  const int j0 = 128 * tile, tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const size_t nh = (size_t)n * a.H + h;
+  const int cols = min(128, a.dv - j0);
+  for (int e = tid; e < 128 * 128; e += 256) {  // E_0 = S0 (zeros without one)
+    const int i = e >> 7, v = e & 127;
+    if (v < cols)
+      q.s_start[((nh * q.nseg) * DK + i) * (size_t)a.dv + j0 + v] = a.S0 ? a.S0[(nh * DK + i) * (size_t)a.dv + j0 + v] : 0.f;
+  }
+  // E_1 = B_0
+  for (int e = tid; e < 128 * 128; e += 256) {
+    const int i = e >> 7, v = e & 127;
+    E[i * 132 + v] = v < cols ? q.sum_b[(nh * (q.nseg - 1) * DK + i) * (size_t)a.dv + j0 + v] : 0.f;
+  }
+  __syncthreads();
+  for (int j = 1; j < q.nseg; ++j) {
+    // E_j -> s_start[j]
+    for (int e = tid; e < 128 * 128; e += 256) {
+      const int i = e >> 7, v = e & 127;
+      if (v < cols) q.s_start[((nh * q.nseg + j) * DK + i) * (size_t)a.dv + j0 + v] = E[i * 132 + v];
+    }
+    if (j == q.nseg - 1) break;
+    // E_{j+1} = A_j E_j + B_j: thread (ty, tx) owns rows 8 ty .. +7, columns 8 tx .. +7
+    const float *A = q.sum_a + (nh * (q.nseg - 1) + j) * DK * DK;
+    const float *Bj = q.sum_b + ((nh * (q.nseg - 1) + j) * DK) * (size_t)a.dv + j0;
+    float acc[8][8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[r][c] = (8 * tx + c < cols) ? Bj[(size_t)(8 * ty + r) * a.dv + 8 * tx + c] : 0.f;
+    for (int k0 = 0; k0 < DK; k0 += 32) {
+      __syncthreads();
+      for (int e = tid; e < 32 * 128; e += 256) {  // At[kk][i] = A[i][k0 + kk]
+        const int i = e >> 5, kk = e & 31;
+        At[kk * 132 + i] = A[i * DK + k0 + kk];
+      }
+      __syncthreads();
+#pragma unroll 4
+      for (int kk = 0; kk < 32; ++kk) {
+        float av[8], ev[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) av[r] = At[kk * 132 + 8 * ty + r];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) ev[c] = E[(k0 + kk) * 132 + 8 * tx + c];
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+          for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(av[r], ev[c], acc[r][c]);
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) E[(8 * ty + r) * 132 + 8 * tx + c] = acc[r][c];
+    __syncthreads();
   }
 }
 
@@ -1097,25 +1236,57 @@ long long chunk_capacity(int B, int T, bool packed) {
   return ((long long)T + (long long)(C - 1) * B) / C;
 }
 
-// Workspace layout: Mt tiles | Nt tiles | Qt tiles | Pt tiles | e^{g_C} | U (like v) | chunk offsets
-// (packed only); every array starts on a 256-byte boundary
+// SMs of the current device (148 on B200 if the query fails).
+int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      sms <= 0)
+    sms = 148;
+  return sms;
+}
+
+// Segments per sequence of the two-level state scan (1: one walk per sequence).  It pays only when
+// the (sequence, head, value tile) walks cannot fill the GPU: then the walk is cut into segments of
+// at least 16 chunks, as many as let the summary pass run in one wave.
+int scan_segments(int B, int T, int H, int dv, bool packed, int sms, int *seg_len) {
+  *seg_len = 0;
+  if (packed) return 1;
+  const int nch = (T + C - 1) / C, tiles = (dv + 127) / 128;
+  const long long walks = (long long)B * H * tiles;
+  if (walks * 4 > sms) return 1;
+  int nseg = 1 + (int)(sms / ((long long)B * H * (1 + tiles)));
+  nseg = min(nseg, nch / 16);
+  if (nseg < 2) return 1;
+  const int len = (nch + nseg - 1) / nseg;
+  *seg_len = len;
+  return (nch + len - 1) / len;
+}
+
+// Workspace layout: Mt tiles | Nt tiles | Qt tiles | Pt tiles | e^{g_C} | U (like v) | two-level scan
+// maps and entry states (long sequences only) | chunk offsets (packed only); 256-byte aligned arrays
 struct WsLayout {
   long long records;
-  size_t m, n, q, p, g, u, coff, total;
+  int nseg, seg_len;
+  size_t m, n, q, p, g, u, sa, sbm, ss, coff, total;
 };
 size_t up256(size_t x) { return (x + 255) / 256 * 256; }
-WsLayout ws_layout(int B, int T, int H, int dv, bool packed) {
+WsLayout ws_layout(int B, int T, int H, int dv, bool packed, int sms) {
   WsLayout L{};
   L.records = chunk_capacity(B, T, packed) * H;
+  L.nseg = scan_segments(B, T, H, dv, packed, sms, &L.seg_len);
   const size_t r = (size_t)L.records;
   const size_t tokens = packed ? (size_t)T : (size_t)B * T;
+  const size_t pairs = (size_t)B * H, ns = L.nseg > 1 ? (size_t)L.nseg : 0;
   L.m = 0;
   L.n = L.m + r * REC_M;
   L.q = L.n + r * REC_N;
   L.p = L.q + r * REC_Q;
   L.g = L.p + r * REC_P;
   L.u = up256(L.g + r * REC_G);
-  L.coff = up256(L.u + tokens * H * dv * 2);
+  L.sa = up256(L.u + tokens * H * dv * 2);
+  L.sbm = up256(L.sa + (ns ? pairs * (ns - 1) * DK * DK * 4 : 0));
+  L.ss = up256(L.sbm + (ns ? pairs * (ns - 1) * DK * dv * 4 : 0));
+  L.coff = up256(L.ss + pairs * ns * DK * dv * 4);
   L.total = L.coff + (packed ? up256((size_t)(B + 1) * 4) : 0);
   return L;
 }
@@ -1130,18 +1301,17 @@ bool chunk_wy_supported(int B, int T, int H, int dk, int dv, bool packed, bool b
 }
 
 size_t chunk_wy_workspace_bytes(int B, int T, int H, int dv, bool packed) {
-  return ws_layout(B, T, H, dv, packed).total;
+  return ws_layout(B, T, H, dv, packed, device_sms()).total;
 }
 
 cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   const long long tokens = a.cu ? (long long)a.T : (long long)a.B * a.T;
-  const WsLayout L = ws_layout(a.B, a.T, a.H, a.dv, a.cu != nullptr);
+  const int sms = device_sms();
+  const WsLayout L = ws_layout(a.B, a.T, a.H, a.dv, a.cu != nullptr, sms);
   uint8_t *base = static_cast<uint8_t *>(ws);
   WyParams p;
   cudaError_t err = device_status_word(&p.status);
   if (err != cudaSuccess) return err;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   p.prefetch_stride = 2 * sms;
   p.N = a.B;
   p.nc = (a.T + C - 1) / C;
@@ -1179,11 +1349,36 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
                                                                               mw);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
-  const long long blocks = (long long)a.B * a.H * ((a.dv + sp::VW - 1) / sp::VW);
+  const long long tiles = (a.dv + sp::VW - 1) / sp::VW;
   err = cudaFuncSetAttribute(state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp::SMEM_BYTES);
   if (err != cudaSuccess) return err;
+  ScanParams q{};
+  if (L.nseg <= 1) {  // one walk per (sequence, head, value tile)
+    note_launch();
+    state_pass_kernel<<<(unsigned)(a.B * a.H * tiles), sp::NT, sp::SMEM_BYTES, stream>>>(a, p, q, mm, mn, mqt, mp, mu, mo);
+    return cudaGetLastError();
+  }
+  // two-level scan: segment maps, their chain into entry states, then the segments' walks
+  q.seg_len = L.seg_len;
+  q.nseg = L.nseg;
+  q.sum_a = reinterpret_cast<float *>(base + L.sa);
+  q.sum_b = reinterpret_cast<float *>(base + L.sbm);
+  q.s_start = reinterpret_cast<float *>(base + L.ss);
+  q.mode = 1;
   note_launch();
-  state_pass_kernel<<<(unsigned)blocks, sp::NT, sp::SMEM_BYTES, stream>>>(a, p, mm, mn, mqt, mp, mu, mo);
+  state_pass_kernel<<<(unsigned)(a.B * a.H * (L.nseg - 1) * (1 + tiles)), sp::NT, sp::SMEM_BYTES, stream>>>(
+      a, p, q, mm, mn, mqt, mp, mu, mo);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  const int chain_smem = (128 * 132 + 32 * 132) * 4;
+  err = cudaFuncSetAttribute(segment_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, chain_smem);
+  if (err != cudaSuccess) return err;
+  note_launch();
+  segment_chain_kernel<<<(unsigned)(a.B * a.H * tiles), 256, chain_smem, stream>>>(a, q);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  q.mode = 2;
+  note_launch();
+  state_pass_kernel<<<(unsigned)(a.B * a.H * L.nseg * tiles), sp::NT, sp::SMEM_BYTES, stream>>>(a, p, q, mm, mn, mqt,
+                                                                                                  mp, mu, mo);
   return cudaGetLastError();
 }
 

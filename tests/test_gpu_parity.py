@@ -205,3 +205,27 @@ def test_bounded_wait_timeout_is_reported_and_context_survives(g):
     wl = W.Workload("after_timeout", B=1, T=100, H=2, dk=128, dv=128)
     run_case(g, wl, seed=21)
     assert g.device_status() == g.GDN2_OK
+
+
+# ------------------------------------------------------------------ two-level (segment) state scan
+# Long dense sequences over few (sequence, head) pairs take the segmented path: segment maps,
+# their chain into entry states, then every segment from its entry state.
+
+@pytest.mark.parametrize("B,T,H,dv", [(1, 2500, 2, 128), (1, 4100, 1, 256), (1, 3000, 2, 64)])
+def test_two_level_scan_matches_oracle(g, B, T, H, dv):
+    wl = W.Workload("segmented", B=B, T=T, H=H, dk=128, dv=dv)
+    run_case(g, wl, seed=41)
+
+
+def test_two_level_scan_zero_state_and_aliased_final_state(g):
+    wl = W.Workload("segmented_alias", B=1, T=2600, H=2, dk=128, dv=128)
+    d = W.chunk_inputs(wl, device="cuda", seed=42)
+    o, _ = g.chunk_fwd(*[d[n] for n in TOK], S0=None, output_final_state=False)
+    S = d["S0"].clone()
+    o2, _ = g.chunk_fwd(*[d[n] for n in TOK], S0=S, S_T=S)
+    torch.cuda.synchronize()
+    o_ref, _ = oracle.recurrent(*[np64(d[n]) for n in TOK])
+    check_bf16(np64(o), o_ref, "o, zero initial state")
+    o_ref2, S_ref2 = oracle.recurrent(*[np64(d[n]) for n in TOK], S0=np64(d["S0"]))
+    check_bf16(np64(o2), o_ref2, "o")
+    check_bf16(S.cpu().double().numpy(), S_ref2, "aliased S_T")
