@@ -21,6 +21,12 @@ Functions and the passages they follow:
   :func:`recurrent`.
 * :func:`recurrent_planted` -- the recurrence with one planted mistake, used
   only to show that the pins catch each mistake.
+* :func:`block_prologue`, :func:`block_epilogue` -- the elementwise and
+  short-convolution work around the mixer in its block (short causal
+  convolution, SiLU, L2 normalisation of q and k; decay and gates; RMS
+  normalisation times a SiLU output gate), from "NVIDIA AIがGated DeltaNet-2を発表"
+  (ai.warp-studio.com), section "アーキテクチャとパフォーマンスベンチマーク";
+  the code is in ``block_oracle.c``.
 """
 import ctypes
 import os
@@ -63,6 +69,10 @@ def _load():
         lib.oracle_gdn2_chunkwise.argtypes = common + [ci, ci]
         lib.oracle_gdn2_chunkwise.restype = ci
         lib.oracle_plant_count.restype = ci
+        lib.oracle_block_prologue.argtypes = [dp] * 15 + [ci] * 6 + [i64p]
+        lib.oracle_block_prologue.restype = ci
+        lib.oracle_block_epilogue.argtypes = [dp] * 4 + [ctypes.c_int64, ci, ci]
+        lib.oracle_block_epilogue.restype = ci
         lib.oracle_max_threads.restype = ci
         _lib = lib
     return _lib
@@ -154,3 +164,41 @@ def decode_step(q, k, v, alpha, b, w, S):
     ex = lambda x: _f64(x)[:, None]  # noqa: E731  -- a length-1 sequence per batch entry
     o, ST = recurrent(ex(q), ex(k), ex(v), ex(alpha), ex(b), ex(w), S0=S)
     return o[:, 0], ST
+
+
+def block_prologue(xq, xk, xv, xa, xb, xw, Wq, Wk, Wv, cu_seqlens=None):
+    """q, k, v, alpha, b, w from the projections' outputs (see ``block_oracle.c``).
+
+    Dense: token tensors ``[N, T, H, d]``; packed: ``[T_total, H, d]`` with ``cu_seqlens`` (N+1).
+    Convolution weights ``[H*d, K]``.  Returns six fp64 arrays shaped like the inputs.
+    """
+    xq, xk, xv, xa, xb, xw, Wq, Wk, Wv = (_f64(x) for x in (xq, xk, xv, xa, xb, xw, Wq, Wk, Wv))
+    if cu_seqlens is None:
+        N, T, H, dk = xq.shape
+        cu = None
+    else:
+        T, H, dk = xq.shape
+        N = len(cu_seqlens) - 1
+        cu = np.ascontiguousarray(cu_seqlens, dtype=np.int64)
+    dv = xv.shape[-1]
+    K = Wq.shape[1]
+    outs = [np.zeros_like(x) for x in (xq, xk, xv, xa, xb, xw)]
+    i64p = ctypes.POINTER(ctypes.c_int64)
+    rc = _load().oracle_block_prologue(*[_ptr(x) for x in (xq, xk, xv, xa, xb, xw, Wq, Wk, Wv)],
+                                       *[_ptr(x) for x in outs], N, T, H, dk, dv, K,
+                                       None if cu is None else cu.ctypes.data_as(i64p))
+    if rc != 0:
+        raise ValueError(f"oracle_block_prologue failed ({rc})")
+    return tuple(outs)
+
+
+def block_epilogue(o, z, g):
+    """y = RMSNorm(o) * g * SiLU(z) per (token, head) over d_v (see ``block_oracle.c``)."""
+    o, z, g = _f64(o), _f64(z), _f64(g)
+    H, dv = o.shape[-2], o.shape[-1]
+    tokens = o.size // (H * dv)
+    y = np.zeros_like(o)
+    rc = _load().oracle_block_epilogue(_ptr(o), _ptr(z), _ptr(g), _ptr(y), tokens, H, dv)
+    if rc != 0:
+        raise ValueError(f"oracle_block_epilogue failed ({rc})")
+    return y
