@@ -47,6 +47,10 @@ def lib():
         L.gdn2_chunk_fwd.restype = ci
         L.gdn2_chunk_fwd_noalloc.argtypes = [vp] * 9 + [ci] * 6 + [vp, ci, vp]
         L.gdn2_chunk_fwd_noalloc.restype = ci
+        L.gdn2_block_prologue.argtypes = [vp] * 15 + [ci] * 6 + [vp, ci, vp]
+        L.gdn2_block_prologue.restype = ci
+        L.gdn2_block_epilogue.argtypes = [vp] * 4 + [ctypes.c_longlong, ci, ci, ci, vp]
+        L.gdn2_block_epilogue.restype = ci
         L.gdn2_decode_step.argtypes = [vp] * 8 + [ci] * 5 + [vp]
         L.gdn2_decode_step.restype = ci
         L.gdn2_status_string.argtypes = [ci]
@@ -160,6 +164,52 @@ def chunk_fwd_noalloc(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, chunk=64, 
 
 
 NOALLOC_WORKSPACE_BYTES = 64 << 20  # GDN2_NOALLOC_WORKSPACE_BYTES in include/gdn2.h
+
+
+def block_prologue(xq, xk, xv, xa, xb, xw, conv_q, conv_k, conv_v, cu_seqlens=None, stream=None):
+    """The mixer's inputs from the projections' outputs: returns ``(q, k, v, alpha, b, w)``.
+
+    Token tensors ``[B, T, H, d]`` (dense) or ``[T_total, H, d]`` with ``cu_seqlens``; convolution
+    weights ``[H*d, K]`` float32 with K in 1..4.  See ``gdn2_block_prologue`` in ``include/gdn2.h``.
+    """
+    if cu_seqlens is None:
+        B, T, H, dk = xq.shape
+    else:
+        if cu_seqlens.dtype != torch.int32:
+            raise ValueError("gdn2: cu_seqlens must be int32")
+        B = cu_seqlens.numel() - 1
+        T, H, dk = xq.shape
+    dv = xv.shape[-1]
+    if xq.dtype not in _DTYPES or any(x.dtype != xq.dtype for x in (xk, xv, xa, xb, xw)):
+        raise ValueError("gdn2: the pre-activations must share dtype float32 or bfloat16")
+    if any(W.dtype != torch.float32 for W in (conv_q, conv_k, conv_v)):
+        raise ValueError("gdn2: convolution weights must be float32")
+    outs = [torch.empty_like(x) for x in (xq, xk, xv, xa, xb, xw)]
+    _check_tensors(xq, xk, xv, xa, xb, xw, conv_q, conv_k, conv_v, *outs, cu_seqlens)
+    st = lib().gdn2_block_prologue(*[_ptr(x) for x in (xq, xk, xv, xa, xb, xw, conv_q, conv_k, conv_v)],
+                                   *[_ptr(x) for x in outs], B, T, H, dk, dv, conv_q.shape[1],
+                                   _ptr(cu_seqlens), _DTYPES[xq.dtype], _stream(stream))
+    if st != GDN2_OK:
+        raise Gdn2Error(st, "gdn2_block_prologue")
+    return tuple(outs)
+
+
+def block_epilogue(o, gate, norm_weight, y=None, stream=None):
+    """``y = RMSNorm(o) * norm_weight * SiLU(gate)`` per (token, head) over d_v; ``y`` may be ``o``."""
+    H, dv = o.shape[-2], o.shape[-1]
+    tokens = o.numel() // (H * dv)
+    if o.dtype not in _DTYPES or gate.dtype != o.dtype:
+        raise ValueError("gdn2: o and gate must share dtype float32 or bfloat16")
+    if norm_weight.dtype != torch.float32:
+        raise ValueError("gdn2: norm_weight must be float32")
+    if y is None:
+        y = torch.empty_like(o)
+    _check_tensors(o, gate, norm_weight, y)
+    st = lib().gdn2_block_epilogue(_ptr(o), _ptr(gate), _ptr(norm_weight), _ptr(y), tokens, H, dv,
+                                   _DTYPES[o.dtype], _stream(stream))
+    if st != GDN2_OK:
+        raise Gdn2Error(st, "gdn2_block_epilogue")
+    return y
 
 
 def decode_step(q, k, v, alpha, b, w, S, o=None, stream=None):

@@ -51,6 +51,23 @@ __device__ __forceinline__ void seq_span(const ChunkArgs &a, int n, int64_t &bos
   }
 }
 
+// Arguments of the block prologue / epilogue around the mixer (validated by the API layer).
+struct BlockPrologueArgs {
+  const void *xq, *xk, *xv, *xa, *xb, *xw;  // pre-activations, [tokens, H, d]
+  const float *Wq, *Wk, *Wv;                // short causal convolution weights, [H * d, K]
+  void *q, *k, *v, *alpha, *b, *w;          // outputs, [tokens, H, d]
+  const int32_t *cu;                        // packed batch offsets [B+1] or nullptr
+  int B, T, H, dk, dv, K;
+  long long tokens;
+};
+struct BlockEpilogueArgs {
+  const void *o, *z;  // mixer output and output-gate pre-activation, [tokens, H, d_v]
+  const float *g;     // RMS-normalisation weight [d_v]
+  void *y;
+  long long tokens;
+  int H, dv;
+};
+
 // Host side: every kernel launch of the library is counted here.
 void note_launch();
 
@@ -68,5 +85,7 @@ cudaError_t read_device_status(int *status, bool reset);
 // Device address of that word, for kernels compiled in other files.
 cudaError_t device_status_word(int **ptr);
 cudaError_t launch_decode(const DecodeArgs &a, bool bf16, cudaStream_t stream);
+cudaError_t launch_block_prologue(const BlockPrologueArgs &p, bool bf16, cudaStream_t stream);
+cudaError_t launch_block_epilogue(const BlockEpilogueArgs &p, bool bf16, cudaStream_t stream);
 
 }  // namespace gdn2

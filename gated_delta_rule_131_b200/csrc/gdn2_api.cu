@@ -203,6 +203,48 @@ size_t gdn2_chunk_fwd_workspace_bytes(int B, int T, int H, int d_k, int d_v, int
   return gdn2::chunk_wy_workspace_bytes(B, T, H, d_v, packed != 0);
 }
 
+gdn2_status gdn2_block_prologue(const void *x_q, const void *x_k, const void *x_v, const void *x_alpha,
+                                const void *x_b, const void *x_w, const float *conv_q, const float *conv_k,
+                                const float *conv_v, void *q, void *k, void *v, void *alpha, void *b, void *w,
+                                int B, int T, int H, int d_k, int d_v, int conv_len, const int32_t *cu_seqlens,
+                                gdn2_dtype dtype, gdn2_stream_t stream) {
+  if (B < 0 || T < 0 || H <= 0) return GDN2_ERR_INVALID_ARG;
+  if (dtype != GDN2_F32 && dtype != GDN2_BF16) return GDN2_ERR_INVALID_ARG;
+  if (!supported_dk(d_k) || !supported_dv(d_v) || conv_len < 1 || conv_len > 4) return GDN2_ERR_UNSUPPORTED;
+  const long long tokens = cu_seqlens ? (long long)T : (long long)B * T;
+  if (!fits(tokens, H, d_v > d_k ? d_v : d_k, 1)) return GDN2_ERR_INVALID_ARG;
+  if (!conv_q || !conv_k || !conv_v) return GDN2_ERR_INVALID_ARG;
+  for (const float *p : {conv_q, conv_k, conv_v})
+    if (reinterpret_cast<uintptr_t>(p) & 3u) return GDN2_ERR_INVALID_ARG;
+  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return GDN2_ERR_INVALID_ARG;
+  if (tokens > 0) {
+    for (const void *p : {x_q, x_k, x_v, x_alpha, x_b, x_w, (const void *)q, (const void *)k, (const void *)v,
+                          (const void *)alpha, (const void *)b, (const void *)w})
+      if (!p || !aligned16(p)) return GDN2_ERR_INVALID_ARG;
+  }
+  if (B == 0 || tokens == 0) return GDN2_OK;
+  gdn2::BlockPrologueArgs a{x_q, x_k, x_v, x_alpha, x_b, x_w, conv_q, conv_k, conv_v, q, k, v, alpha, b, w,
+                            cu_seqlens, B, T, H, d_k, d_v, conv_len, tokens};
+  const cudaError_t err = gdn2::launch_block_prologue(a, dtype == GDN2_BF16, (cudaStream_t)stream);
+  return err == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+}
+
+gdn2_status gdn2_block_epilogue(const void *o, const void *gate, const float *norm_weight, void *y, long long tokens,
+                                int H, int d_v, gdn2_dtype dtype, gdn2_stream_t stream) {
+  if (tokens < 0 || H <= 0) return GDN2_ERR_INVALID_ARG;
+  if (dtype != GDN2_F32 && dtype != GDN2_BF16) return GDN2_ERR_INVALID_ARG;
+  if (!supported_dv(d_v)) return GDN2_ERR_UNSUPPORTED;
+  if (!fits(tokens, H, d_v, 1)) return GDN2_ERR_INVALID_ARG;
+  if (!norm_weight || (reinterpret_cast<uintptr_t>(norm_weight) & 3u)) return GDN2_ERR_INVALID_ARG;
+  if (tokens > 0)
+    for (const void *p : {o, gate, (const void *)y})
+      if (!p || !aligned16(p)) return GDN2_ERR_INVALID_ARG;
+  if (tokens == 0) return GDN2_OK;
+  gdn2::BlockEpilogueArgs a{o, gate, norm_weight, y, tokens, H, d_v};
+  const cudaError_t err = gdn2::launch_block_epilogue(a, dtype == GDN2_BF16, (cudaStream_t)stream);
+  return err == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+}
+
 gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v, const void *alpha,
                              const void *b, const void *w, float *S, void *o, int B, int H,
                              int d_k, int d_v, gdn2_dtype dtype, gdn2_stream_t stream) {

@@ -173,6 +173,46 @@ def chunk_inputs(wl: Workload, device="cpu", seed: int = 0, lengths: Optional[Li
     return out
 
 
+def block_inputs(wl: Workload, device="cpu", seed: int = 0, conv_len: int = 4,
+                 lengths: Optional[List[int]] = None) -> dict:
+    """Inputs of the block prologue and epilogue around the mixer (the projections' outputs).
+
+    Token tensors xq, xk, xa, xb [.., H, d_k] and xv, xw, z [.., H, d_v] ~ N(0, 1) (xa shifted by
+    -alpha_shift, the bias of the decay branch), cast to the workload dtype; dense [B, T, H, d] or
+    packed [T_total, H, d] with cu_seqlens.  Convolution weights conv_q, conv_k [H*d_k, K] and
+    conv_v [H*d_v, K] ~ N(0, 1/K) fp32; norm_weight [d_v] ~ U(0.5, 1.5) fp32.
+    """
+    lens = seq_lengths(wl, seed) if lengths is None else list(lengths)
+    dt = TORCH_DTYPE[wl.dtype]
+    per = []
+    for i, L in enumerate(lens):
+        g = _gen(device, seed, "block_seq", i)
+        f32 = dict(device=device, dtype=torch.float32, generator=g)
+        d = {n: torch.randn(L, wl.H, wl.dk if n in ("xq", "xk", "xa", "xb") else wl.dv, **f32)
+             for n in ("xq", "xk", "xv", "xa", "xb", "xw", "z")}
+        d["xa"] = d["xa"] - wl.alpha_shift
+        per.append({n: t.to(dt) for n, t in d.items()})
+    names = ("xq", "xk", "xv", "xa", "xb", "xw", "z")
+    if wl.varlen:
+        out = {n: torch.cat([p[n] for p in per], 0).contiguous() for n in names}
+        cu = [0]
+        for L in lens:
+            cu.append(cu[-1] + L)
+        out["cu_seqlens"] = torch.tensor(cu, dtype=torch.int32, device=device)
+    else:
+        out = {n: torch.stack([p[n] for p in per], 0).contiguous() for n in names}
+        out["cu_seqlens"] = None
+    g = _gen(device, seed, "block_weights")
+    f32 = dict(device=device, dtype=torch.float32, generator=g)
+    out["conv_q"] = torch.randn(wl.H * wl.dk, conv_len, **f32) / conv_len ** 0.5
+    out["conv_k"] = torch.randn(wl.H * wl.dk, conv_len, **f32) / conv_len ** 0.5
+    out["conv_v"] = torch.randn(wl.H * wl.dv, conv_len, **f32) / conv_len ** 0.5
+    out["norm_weight"] = torch.rand(wl.dv, **f32) + 0.5
+    out["S0"] = initial_state(wl, len(lens), device, seed)
+    out["lengths"] = lens
+    return out
+
+
 def sequence_inputs(wl: Workload, index: int, device="cpu", seed: int = 0) -> dict:
     """The inputs of one sequence of ``chunk_inputs`` alone: [len, H, d] tensors and S0 [H, d_k, d_v]."""
     L = seq_lengths(wl, seed)[index]

@@ -148,6 +148,44 @@ GDN2_API gdn2_status gdn2_decode_step(const void *q, const void *k, const void *
                              const void *b, const void *w, float *S, void *o, int B, int H,
                              int d_k, int d_v, gdn2_dtype dtype, gdn2_stream_t stream);
 
+/*
+ * gdn2_block_prologue -- the mixer's inputs from the block's projections.
+ *
+ * "NVIDIA AIがGated DeltaNet-2を発表" (ai.warp-studio.com), section
+ * "アーキテクチャとパフォーマンスベンチマーク": the query and key paths apply a short causal
+ * convolution, SiLU and L2 normalisation to their projection, the value path a short convolution
+ * and SiLU; the decay and both gates come from their own linear branches.  The projections
+ * (matrix products) are the caller's; this call takes their outputs:
+ *   x_q, x_k, x_alpha, x_b : [tokens, H, d_k]     x_v, x_w : [tokens, H, d_v]   (dtype)
+ *   conv_q, conv_k : [H * d_k, conv_len] fp32     conv_v : [H * d_v, conv_len] fp32
+ * and writes, in the layouts gdn2_chunk_fwd reads:
+ *   q = L2norm(SiLU(conv_q * x_q)), k likewise (over d_k per token and head, eps 1e-6 under the
+ *   root), v = SiLU(conv_v * x_v), alpha = exp(-softplus(x_alpha)), b = sigmoid(x_b),
+ *   w = sigmoid(x_w).
+ * The convolution is depthwise and causal, y_t = sum_j conv[c][conv_len-1-j] x_{t-j}[c] (the last
+ * tap multiplies the current token), and restarts at every sequence start: dense batches are B
+ * sequences of T tokens; packed batches (cu_seqlens != NULL, device int32 [B+1]) have T tokens in
+ * total.  conv_len: 1 to 4.  d_k in {64, 128}, d_v in {64, 128, 256}.  Token tensors 16-byte
+ * aligned, weights 4-byte aligned; outputs must not overlap the inputs.  fp32 arithmetic.
+ * Asynchronous on `stream`; validation errors return before any launch.
+ */
+GDN2_API gdn2_status gdn2_block_prologue(const void *x_q, const void *x_k, const void *x_v, const void *x_alpha,
+                                         const void *x_b, const void *x_w, const float *conv_q, const float *conv_k,
+                                         const float *conv_v, void *q, void *k, void *v, void *alpha, void *b,
+                                         void *w, int B, int T, int H, int d_k, int d_v, int conv_len,
+                                         const int32_t *cu_seqlens, gdn2_dtype dtype, gdn2_stream_t stream);
+
+/*
+ * gdn2_block_epilogue -- the output gate after the mixer (same page and section): the recurrent
+ * output is RMS-normalised and multiplied by a SiLU output gate (before the output projection,
+ * the caller's).  For every token and head, over its d_v values:
+ *   y = o / sqrt(mean(o^2) + 1e-5) * norm_weight * SiLU(gate)
+ *   o, gate, y : [tokens, H, d_v] (dtype, 16-byte aligned)   norm_weight : [d_v] fp32
+ * y may alias o.  d_v in {64, 128, 256}.  fp32 arithmetic.  Asynchronous on `stream`.
+ */
+GDN2_API gdn2_status gdn2_block_epilogue(const void *o, const void *gate, const float *norm_weight, void *y,
+                                         long long tokens, int H, int d_v, gdn2_dtype dtype, gdn2_stream_t stream);
+
 /* Human-readable name of a status; never NULL. */
 GDN2_API const char *gdn2_status_string(gdn2_status status);
 
