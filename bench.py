@@ -7,7 +7,8 @@ H=16, d_k=d_v=128, chunk 64, bf16 inputs, fp32 state, seeded synthetic data).
 ``value`` is tokens/s over all ranks (each rank runs its own batch; no
 collective on the data path: weak scaling).  The same JSON line carries the
 decode measurement (256 x 16 heads, 1024 single-token steps replayed from one
-CUDA graph) as ``decode_step``, the roofline of the dominant kernel, the CPU
+CUDA graph) as ``decode_step``, the block prologue and epilogue around the mixer
+(``block_prologue``, ``block_epilogue``), the roofline of the dominant kernel, the CPU
 oracle baseline, the end-to-end number through host buffers, and clocks.
 
 ``--impl reference`` times the fp64 CPU oracle (the only reference that
@@ -232,6 +233,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-block", action="store_true", help="skip the block prologue/epilogue measurement")
     ap.add_argument("--profile-case", choices=["chunk", "decode"],
                     help="run one warm-up and one measured launch of that kernel on its full workload, for ncu")
     args = ap.parse_args()
@@ -319,6 +321,9 @@ def main():
     if not args.no_decode:
         line["decode_step"] = bench_decode(gdn2, dev, stream, pk, pk_kind)
         line["gpu_launches_decode"] = line["decode_step"].pop("launches")
+    # ------------------------------------------------------------ block prologue / epilogue around the mixer
+    if not args.no_block:
+        line.update(bench_block(gdn2, dev, stream, pk, pk_kind))
 
     # ------------------------------------------------------------ end to end through host buffers
     line["e2e"] = bench_e2e(gdn2, wl, sets[0], dev, stream, ws, tokens)
@@ -397,6 +402,48 @@ def bench_decode(gdn2, dev, stream, pk, pk_kind):
                          "frac": gbs / pk["hbm_gbs"], "traffic": tr["dram_bytes_per_launch"] if tr else None,
                          "peak_source": pk_kind, "algorithmic_bytes_per_launch": bytes_step},
             "launches": per_replay * reps}
+
+
+def block_bytes(wl, tokens):
+    """Algorithmic bytes of the block prologue and epilogue (every element read and written once)."""
+    e = 2 if wl.dtype == "bf16" else 4
+    th = tokens * wl.H
+    pro = th * 2 * (4 * wl.dk + 2 * wl.dv) * e + 3 * 4 * wl.H * (2 * wl.dk + wl.dv) * 4  # + conv weights
+    epi = th * 3 * wl.dv * e + wl.dv * 4
+    return pro, epi
+
+
+def bench_block(gdn2, dev, stream, pk, pk_kind, reps=20):
+    """The block prologue and epilogue around the mixer on the 1.3B-layer shape (4 taps)."""
+    wl = W.WORKLOADS["layer_1p3b"]
+    tokens = wl.B * wl.T
+    d = W.block_inputs(wl, device=dev, seed=0, conv_len=4)
+    pre = [d[n] for n in ("xq", "xk", "xv", "xa", "xb", "xw", "conv_q", "conv_k", "conv_v")]
+    o = d["xv"]
+    y = torch.empty_like(o)
+    pro_b, epi_b = block_bytes(wl, tokens)
+    out = {}
+    for name, fn, nbytes in (("block_prologue", lambda: gdn2.block_prologue(*pre, stream=stream), pro_b),
+                             ("block_epilogue", lambda: gdn2.block_epilogue(o, d["z"], d["norm_weight"], y=y,
+                                                                            stream=stream), epi_b)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        c0 = gdn2.launch_count()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in ev:
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out[name] = {"value": gbs, "unit": "GB/s", "workload": "layer_1p3b", "conv_len": 4,
+                     "us_per_call": ms * 1e3, "launches": gdn2.launch_count() - c0,
+                     "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                  "frac": gbs / pk["hbm_gbs"], "traffic": None, "peak_source": pk_kind,
+                                  "algorithmic_bytes_per_launch": nbytes}}
+    return out
 
 
 def bench_e2e(gdn2, wl, d, dev, stream, ws, tokens, steps=3):
