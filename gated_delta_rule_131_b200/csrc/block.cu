@@ -8,24 +8,51 @@
 // All three kernels are HBM-bound streams: every input element is read once and every output
 // element written once, in fp32 arithmetic.
 #include <algorithm>
+#include <climits>
 
 #include "common.cuh"
 
 namespace gdn2 {
 namespace {
 
-constexpr int TT = 64;          // tokens per convolution tile
+constexpr int CE = 8;  // channels per lane in the convolution kernel
 constexpr float L2_EPS = 1e-6f, RMS_EPS = 1e-5f;
 
-// 16-byte asynchronous copy global -> shared (L2 only), and the wait for all of this thread's copies.
+constexpr int CS = 3;  // load batches in a convolution lane's ring (two in flight while one is used)
+
+// 16-byte asynchronous copy global -> shared (through L2), a commit of this thread's copies issued
+// so far as one group, and a wait until at most N of its groups are pending.
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
                "l"(gmem)
                : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 __device__ __forceinline__ float silu(float y) { return __fdividef(y, 1.f + __expf(-y)); }
+
+// SiLU of a pair, y / (1 + e^-y) with e^-y = 2^(-y log2 e), from the PTX approximate base-2
+// exponential and reciprocal (large negative y: e^-y = inf, reciprocal 0, result -0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float2 silu2(float2 y) {
+  constexpr float NEG_LOG2E = -1.4426950408889634f;
+  const float2 m = __fmul2_rn(y, make_float2(NEG_LOG2E, NEG_LOG2E));
+  const float2 den = __fadd2_rn(make_float2(ex2_approx(m.x), ex2_approx(m.y)), make_float2(1.f, 1.f));
+  return __fmul2_rn(y, make_float2(rcp_approx(den.x), rcp_approx(den.y)));
+}
 __device__ __forceinline__ float sigmoid(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 
 struct ConvPath {
@@ -40,94 +67,194 @@ struct ConvArgs {
   const int32_t *cu;
   int N, T, H, K;
   long long tokens;
+  int R;             // tokens per run (a multiple of the tokens a lane loads at once)
 };
 
-// First token of the sequence holding token t.
-__device__ __forceinline__ long long seq_start(const ConvArgs &a, long long t) {
-  if (!a.cu) return (t / a.T) * (long long)a.T;
-  int lo = 0, hi = a.N;
-  while (lo < hi) {  // largest n with cu[n] <= t
-    const int mid = (lo + hi + 1) >> 1;
-    if (a.cu[mid] <= t) lo = mid; else hi = mid - 1;
+// The CE channels of one token that a lane holds, as pairs, from / to their stored type.
+__device__ __forceinline__ void unpack(const uint4 (&r)[1], float2 (&f)[CE / 2]) {
+  const uint32_t w[4] = {r[0].x, r[0].y, r[0].z, r[0].w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) f[i] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
+}
+__device__ __forceinline__ void unpack(const uint4 (&r)[2], float2 (&f)[CE / 2]) {
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    f[2 * i] = make_float2(__uint_as_float(r[i].x), __uint_as_float(r[i].y));
+    f[2 * i + 1] = make_float2(__uint_as_float(r[i].z), __uint_as_float(r[i].w));
   }
-  return a.cu[lo];
+}
+__device__ __forceinline__ void pack(const float2 (&f)[CE / 2], uint4 (&r)[1]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 h = __float22bfloat162_rn(f[i]);
+    w[i] = *reinterpret_cast<const uint32_t *>(&h);
+  }
+  r[0] = make_uint4(w[0], w[1], w[2], w[3]);
+}
+__device__ __forceinline__ void pack(const float2 (&f)[CE / 2], uint4 (&r)[2]) {
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    r[i] = make_uint4(__float_as_uint(f[2 * i].x), __float_as_uint(f[2 * i].y), __float_as_uint(f[2 * i + 1].x),
+                      __float_as_uint(f[2 * i + 1].y));
 }
 
-// One CTA of 256 threads per (64-token tile, head, path).  The tile's input rows (and the 3 rows
-// before it) are staged in shared memory with 16-byte loads.  Thread = (channel, run of tokens): it
-// keeps its channel's taps and convolution window in registers and walks its run from shared
-// memory into an output tile; for q and k each token is then L2-normalised by one warp (from the
-// activated values as stored), and the tile leaves with 16-byte stores.  Dynamic shared memory:
-// (2 TT + 3) rows of the widest path.
+// Depthwise causal convolution of K <= 4 taps, SiLU, and (q, k) L2 normalisation, streamed through
+// registers.  A group of G = d / CE lanes holds one (token, head) row, CE consecutive channels per
+// lane, and walks a run of R consecutive tokens of one head: it loads the run's rows 16 bytes per
+// lane, CU tokens at a time, keeps its taps and the three previous tokens in registers, clears
+// that window where a sequence starts, and reduces the row's sum of squares with shuffles inside
+// the group.  Loads go through a ring of CS batches in shared memory with asynchronous copies, so
+// that two batches are in flight while one is used; each lane reads back only its own copies, so
+// the block never synchronises.  Every row is read once (plus three halo rows per run) and written
+// once.  grid = (blocks of the widest path, 3 paths); the host picks R so that the grid is one wave.
 template <typename T>
-__global__ void __launch_bounds__(256) conv_silu_kernel(const ConvArgs a) {
-  extern __shared__ __align__(16) uint8_t dsm[];
-  __shared__ int s_start[TT];  // per token of the tile: index (relative to the tile) of its sequence's first token
-  const ConvPath P = blockIdx.z == 0 ? a.path[0] : (blockIdx.z == 1 ? a.path[1] : a.path[2]);
-  const int d = P.d, tid = threadIdx.x;
-  const int h = blockIdx.y;
-  const long long t0 = (long long)blockIdx.x * TT;
-  const int nt = (int)min((long long)TT, a.tokens - t0);
-  const int halo = (int)min(t0, 3LL);  // staged rows before the tile
-  const int nrows = nt + halo;
-  T *__restrict__ tin = reinterpret_cast<T *>(dsm);       // [nrows][d], row halo + i = token t0 + i
-  T *__restrict__ tout = tin + (TT + 3) * d;               // [nt][d]
-  const T *x = reinterpret_cast<const T *>(P.x);
-  T *out = reinterpret_cast<T *>(P.out);
-  const size_t stride = (size_t)a.H * d;  // elements between consecutive tokens
-  constexpr int V = 16 / sizeof(T);       // elements per 16-byte vector
-  const int vrow = d / V;
-  const T *xbase = x + (size_t)(t0 - halo) * stride + (size_t)h * d;
-  for (int i = tid; i < nt; i += 256) s_start[i] = (int)max(seq_start(a, t0 + i) - t0, -4LL);
-  for (int e = tid; e < nrows * vrow; e += 256) {  // all of the tile's loads in flight at once
-    const int r = e / vrow, vc = e - r * vrow;
-    cp_async16(reinterpret_cast<uint4 *>(tin) + e, reinterpret_cast<const uint4 *>(xbase + (size_t)r * stride) + vc);
-  }
-  cp_async_wait_all();
-  __syncthreads();
+__global__ void __launch_bounds__(256, 2) conv_silu_kernel(const ConvArgs a) {
+  constexpr int NV = CE * (int)sizeof(T) / 16;  // 16-byte vectors per lane and token
+  constexpr int CU = 8 / NV;                    // tokens per load batch
+  extern __shared__ uint4 ring[];               // [CS][CU][NV][256 threads]
+  const ConvPath P = blockIdx.y == 0 ? a.path[0] : (blockIdx.y == 1 ? a.path[1] : a.path[2]);
+  const int G = P.d / CE;  // 8, 16 or 32 lanes, aligned within the warp
+  const long long gid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / G;
+  const long long runs = (a.tokens + a.R - 1) / a.R;
+  if (gid >= runs * a.H) return;  // whole groups leave together
+  const int lane = threadIdx.x & 31, gl = lane & (G - 1);
+  const unsigned gmask = G == 32 ? 0xffffffffu : ((1u << G) - 1u) << (lane & ~(G - 1));
+  const int h = (int)(gid % a.H);
+  const long long t0 = (gid / a.H) * a.R, t1 = min(t0 + (long long)a.R, a.tokens);
+  const size_t stride = (size_t)a.H * P.d;  // elements between consecutive tokens
+  const T *x = static_cast<const T *>(P.x) + (size_t)h * P.d + gl * CE;
+  T *out = static_cast<T *>(P.out) + (size_t)h * P.d + gl * CE;
+
+  float2 w0[CE / 2], w1[CE / 2], w2[CE / 2], w3[CE / 2];  // w_j multiplies x_{t-j}: the taps reversed
   {
-    const int per = (256 / d);           // threads per channel: 1, 2 or 4
-    const int c = tid % d, run = TT / per, i0 = (tid / d) * run;
-    const float *W = P.W + ((size_t)h * d + c) * a.K;
-    float wr[4];  // wr[j] multiplies x_{t-j}: the taps in reverse (the last tap is the current token)
+    const float *W = P.W + ((size_t)h * P.d + gl * CE) * a.K;
+    const int K = a.K;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) wr[j] = j < a.K ? W[a.K - 1 - j] : 0.f;
-    // window xs[j] = x_{t-j}, j = 1..3, for t = t0 + i0 (zero before the sequence start)
-    float xs[4] = {0.f, 0.f, 0.f, 0.f};
-    const int st0 = i0 < nt ? s_start[i0] : 0;
-#pragma unroll
-    for (int j = 1; j < 4; ++j)
-      if (i0 - j >= st0 && i0 - j + halo >= 0) xs[j] = to_f32(tin[(i0 - j + halo) * d + c]);
-    const int i1 = min(i0 + run, nt);
-    for (int i = i0; i < i1; ++i) {
-      if (i > i0 && s_start[i] == i) xs[1] = xs[2] = xs[3] = 0.f;  // a new sequence starts here
-      const float xt = to_f32(tin[(i + halo) * d + c]);
-      const float y = fmaf(wr[3], xs[3], fmaf(wr[2], xs[2], fmaf(wr[1], xs[1], wr[0] * xt)));
-      tout[i * d + c] = from_f32<T>(silu(y));
-      xs[3] = xs[2];
-      xs[2] = xs[1];
-      xs[1] = xt;
+    for (int i = 0; i < CE / 2; ++i) {
+      const float *c0 = W + (2 * i) * K, *c1 = c0 + K;
+      w0[i] = make_float2(c0[K - 1], c1[K - 1]);
+      w1[i] = K > 1 ? make_float2(c0[K - 2], c1[K - 2]) : make_float2(0.f, 0.f);
+      w2[i] = K > 2 ? make_float2(c0[K - 3], c1[K - 3]) : make_float2(0.f, 0.f);
+      w3[i] = K > 3 ? make_float2(c0[K - 4], c1[K - 4]) : make_float2(0.f, 0.f);
     }
   }
-  __syncthreads();
-  if (P.l2) {  // L2 normalisation: one warp per token, lanes over the channels
-    const int warp = tid >> 5, lane = tid & 31;
-    for (int i = warp; i < nt; i += 8) {
-      float ss = 0.f;
-      for (int c = lane; c < d; c += 32) {
-        const float v = to_f32(tout[i * d + c]);
-        ss = fmaf(v, v, ss);
+  // The sequence holding t0: its first token s0 and the next sequence start nb (beyond: none).
+  long long s0, nb;
+  int n = 0;
+  if (!a.cu) {
+    s0 = t0 - t0 % a.T;
+    nb = s0 + a.T;
+  } else {
+    int lo = 0, hi = a.N - 1;
+    while (lo < hi) {  // largest n < N with cu[n] <= t0
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.cu[mid] <= t0) lo = mid; else hi = mid - 1;
+    }
+    n = lo;
+    s0 = a.cu[n];
+    nb = a.cu[n + 1];
+    if (nb <= t0) nb = LLONG_MAX;
+  }
+  float2 x1[CE / 2], x2[CE / 2], x3[CE / 2];  // x_{t-1}, x_{t-2}, x_{t-3}; zero before the sequence
+#pragma unroll
+  for (int i = 0; i < CE / 2; ++i) x1[i] = x2[i] = x3[i] = make_float2(0.f, 0.f);
+  {
+    uint4 r[NV];
+#pragma unroll
+    for (int j = 1; j <= 3; ++j)
+      if (t0 - j >= s0) {
+#pragma unroll
+        for (int v = 0; v < NV; ++v) r[v] = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)(t0 - j) * stride) + v);
+        unpack(r, j == 1 ? x1 : (j == 2 ? x2 : x3));
       }
-      ss = warp_allreduce_sum(ss);
-      const float inv = rsqrtf(ss + L2_EPS);
-      for (int c = lane; c < d; c += 32) tout[i * d + c] = from_f32<T>(to_f32(tout[i * d + c]) * inv);
-    }
-    __syncthreads();
   }
-  T *obase = out + (size_t)t0 * stride + (size_t)h * d;
-  for (int e = tid; e < nt * vrow; e += 256) {
-    const int r = e / vrow, vc = e - r * vrow;
-    reinterpret_cast<uint4 *>(obase + (size_t)r * stride)[vc] = reinterpret_cast<const uint4 *>(tout)[e];
+  // Token indices below are relative to t0 (a run is at most 2^20 tokens).
+  const T *xr = x + (size_t)t0 * stride;
+  T *orow = out + (size_t)t0 * stride;
+  const int ntok = (int)(t1 - t0), ist = (int)stride;
+  int nbr = (int)min(nb - t0, (long long)INT_MAX);  // next sequence start, relative
+  const int nbatch = (ntok + CU - 1) / CU;
+  auto issue = [&](int bt) {  // copies of batch bt (tokens before t1 only), committed as one group
+    const int slot = bt % CS;
+#pragma unroll
+    for (int u = 0; u < CU; ++u) {
+      const int i = bt * CU + u;
+      if (bt < nbatch && i < ntok)
+#pragma unroll
+        for (int v = 0; v < NV; ++v)
+          cp_async16(&ring[((slot * CU + u) * NV + v) * 256 + threadIdx.x],
+                     reinterpret_cast<const uint4 *>(xr + (long long)i * ist) + v);
+    }
+    cp_async_commit();
+  };
+  // One token: convolution, SiLU, (q, k) L2 normalisation, store; then the window moves on.
+  auto token = [&](int i, int slot, int u) {
+    float2 xt[CE / 2], y[CE / 2];
+    {
+      uint4 r[NV];
+#pragma unroll
+      for (int v = 0; v < NV; ++v) r[v] = ring[((slot * CU + u) * NV + v) * 256 + threadIdx.x];
+      unpack(r, xt);
+    }
+    float2 ss = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < CE / 2; ++k) {
+      float2 c = __fmul2_rn(w0[k], xt[k]);
+      c = __ffma2_rn(w1[k], x1[k], c);
+      c = __ffma2_rn(w2[k], x2[k], c);
+      c = __ffma2_rn(w3[k], x3[k], c);
+      y[k] = silu2(c);
+      ss = __ffma2_rn(y[k], y[k], ss);
+      x3[k] = x2[k];
+      x2[k] = x1[k];
+      x1[k] = xt[k];
+    }
+    if (P.l2) {
+      float sum = ss.x + ss.y;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+        if (o < G) sum += __shfl_xor_sync(gmask, sum, o);
+      const float inv = rsqrtf(sum + L2_EPS);
+#pragma unroll
+      for (int k = 0; k < CE / 2; ++k) y[k] = __fmul2_rn(y[k], make_float2(inv, inv));
+    }
+    uint4 r[NV];
+    pack(y, r);
+#pragma unroll
+    for (int v = 0; v < NV; ++v) reinterpret_cast<uint4 *>(orow + (long long)i * ist)[v] = r[v];
+  };
+#pragma unroll
+  for (int bt = 0; bt < CS - 1; ++bt) issue(bt);
+  for (int bt = 0; bt < nbatch; ++bt) {
+    issue(bt + CS - 1);  // into the slot batch bt - 1 used
+    cp_async_wait<CS - 1>();
+    const int ib = bt * CU, slot = bt % CS;
+    if (ib + CU <= ntok && nbr >= ib + CU) {  // a full batch inside one sequence: no checks
+#pragma unroll
+      for (int u = 0; u < CU; ++u) token(ib + u, slot, u);
+    } else {
+      for (int u = 0; u < CU; ++u) {
+        const int i = ib + u;
+        if (i >= ntok) break;  // uniform in the group
+        if (i == nbr) {        // a new sequence starts here (uniform in the group)
+#pragma unroll
+          for (int k = 0; k < CE / 2; ++k) x1[k] = x2[k] = x3[k] = make_float2(0.f, 0.f);
+          const long long t = t0 + i;
+          if (!a.cu) {
+            nb += a.T;
+          } else {
+            int m = n + 1;  // cu[m] == t; skip empty sequences
+            while (m + 1 < a.N && a.cu[m + 1] <= t) ++m;
+            n = m;
+            nb = m + 1 <= a.N ? (long long)a.cu[m + 1] : LLONG_MAX;
+            if (nb <= t) nb = LLONG_MAX;
+          }
+          nbr = (int)min(nb - t0, (long long)INT_MAX);
+        }
+        token(i, slot, u);
+      }
+    }
   }
 }
 
@@ -202,10 +329,37 @@ __global__ void __launch_bounds__(256) rms_gate_kernel(const T *o, const T *z, c
   }
 }
 
+constexpr int CONV_SMEM = CS * 8 * 16 * 256;  // the ring: CS batches of 8 16-byte vectors per thread
+
+// Resident 256-thread blocks of conv_silu_kernel<T> on the current device (per SM times SMs); sets
+// the kernel's shared-memory limit on first use.
+template <typename T>
+cudaError_t conv_slots(int &slots) {
+  static int cache[64] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 64 && cache[dev] > 0) {
+    slots = cache[dev];
+    return cudaSuccess;
+  }
+  int per_sm = 0, sms = 0;
+  err = cudaFuncSetAttribute(conv_silu_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, CONV_SMEM);
+  if (err == cudaSuccess)
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, conv_silu_kernel<T>, 256, CONV_SMEM);
+  if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (err != cudaSuccess) return err;
+  slots = std::max(1, per_sm) * std::max(1, sms);
+  if (dev < 64) cache[dev] = slots;
+  return cudaSuccess;
+}
+
 template <typename T>
 cudaError_t prologue_t(const BlockPrologueArgs &p, cudaStream_t stream) {
-  const int smem = (2 * TT + 3) * std::max(p.dk, p.dv) * (int)sizeof(T);
-  cudaError_t err = cudaFuncSetAttribute(conv_silu_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (p.tokens <= 0) return cudaSuccess;
+  constexpr int CU = 8 * 16 / (CE * (int)sizeof(T));  // tokens a lane loads at once (as in the kernel)
+  int slots = 0;
+  cudaError_t err = conv_slots<T>(slots);
   if (err != cudaSuccess) return err;
   ConvArgs a{};
   a.path[0] = ConvPath{p.xq, p.Wq, p.q, p.dk, 1};
@@ -217,22 +371,24 @@ cudaError_t prologue_t(const BlockPrologueArgs &p, cudaStream_t stream) {
   a.H = p.H;
   a.K = p.K;
   a.tokens = p.tokens;
-  if (p.tokens > 0) {
-    const dim3 grid((unsigned)((p.tokens + TT - 1) / TT), (unsigned)p.H, 3);
-    note_launch();
-    conv_silu_kernel<T><<<grid, 256, smem, stream>>>(a);
-    err = cudaGetLastError();
-    if (err != cudaSuccess) return err;
-    const size_t nk = (size_t)p.tokens * p.H * p.dk, nv = (size_t)p.tokens * p.H * p.dv;
-    const size_t vecs = (nk + nv) / (16 / sizeof(T));
-    const unsigned blocks = (unsigned)std::min<size_t>((vecs + 255) / 256, (size_t)148 * 16);
-    note_launch();
-    gates_kernel<T><<<blocks, 256, 0, stream>>>(static_cast<const T *>(p.xa), static_cast<const T *>(p.xb),
-                                                 static_cast<const T *>(p.xw), static_cast<T *>(p.alpha),
-                                                 static_cast<T *>(p.b), static_cast<T *>(p.w), nk, nv);
-    return cudaGetLastError();
-  }
-  return cudaSuccess;
+  // One wave: lanes x tokens of all three paths over the resident lanes, in whole load batches.
+  const long long lane_tokens = p.tokens * p.H * (long long)(2 * p.dk + p.dv) / CE;
+  const long long per_lane = (lane_tokens + (long long)slots * 256 - 1) / ((long long)slots * 256);
+  a.R = (int)std::min<long long>(std::max<long long>((per_lane + CU - 1) / CU * CU, CU), 1 << 20);
+  const long long runs = (p.tokens + a.R - 1) / a.R;
+  const long long blocks = (runs * p.H * (std::max(p.dk, p.dv) / CE) + 255) / 256;
+  note_launch();
+  conv_silu_kernel<T><<<dim3((unsigned)blocks, 3), 256, CONV_SMEM, stream>>>(a);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const size_t nk = (size_t)p.tokens * p.H * p.dk, nv = (size_t)p.tokens * p.H * p.dv;
+  const size_t vecs = (nk + nv) / (16 / sizeof(T));
+  const unsigned gblocks = (unsigned)std::min<size_t>((vecs + 255) / 256, (size_t)148 * 16);
+  note_launch();
+  gates_kernel<T><<<gblocks, 256, 0, stream>>>(static_cast<const T *>(p.xa), static_cast<const T *>(p.xb),
+                                               static_cast<const T *>(p.xw), static_cast<T *>(p.alpha),
+                                               static_cast<T *>(p.b), static_cast<T *>(p.w), nk, nv);
+  return cudaGetLastError();
 }
 
 template <typename T>
