@@ -70,11 +70,17 @@ struct ConvArgs {
   int R;             // tokens per run (a multiple of the tokens a lane loads at once)
 };
 
+// A bf16 is the top half of the fp32 of the same value, so widening is a shift or a mask (integer
+// pipe, exact).
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
 // The CE channels of one token that a lane holds, as pairs, from / to their stored type.
 __device__ __forceinline__ void unpack(const uint4 (&r)[1], float2 (&f)[CE / 2]) {
-  const uint32_t w[4] = {r[0].x, r[0].y, r[0].z, r[0].w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) f[i] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
+  f[0] = bf2_to_f2(r[0].x);
+  f[1] = bf2_to_f2(r[0].y);
+  f[2] = bf2_to_f2(r[0].z);
+  f[3] = bf2_to_f2(r[0].w);
 }
 __device__ __forceinline__ void unpack(const uint4 (&r)[2], float2 (&f)[CE / 2]) {
 #pragma unroll
