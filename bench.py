@@ -234,7 +234,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-block", action="store_true", help="skip the block prologue/epilogue measurement")
-    ap.add_argument("--profile-case", choices=["chunk", "decode"],
+    ap.add_argument("--profile-case", choices=["chunk", "decode", "block"],
                     help="run one warm-up and one measured launch of that kernel on its full workload, for ncu")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -351,6 +351,12 @@ def profile_case(which):
         d = W.chunk_inputs(wl, device=dev, seed=0)
         for _ in range(2):
             gdn2.chunk_fwd(*[d[n] for n in TOK], S0=d["S0"])
+    elif which == "block":
+        wl = W.WORKLOADS["layer_1p3b"]
+        d = W.block_inputs(wl, device=dev, seed=0, conv_len=4)
+        for _ in range(2):
+            gdn2.block_prologue(*[d[n] for n in ("xq", "xk", "xv", "xa", "xb", "xw", "conv_q", "conv_k", "conv_v")])
+            gdn2.block_epilogue(d["xv"], d["z"], d["norm_weight"])
     else:
         wl = W.WORKLOADS["decode"]
         S = W.decode_state(wl, device=dev, seed=0)
@@ -438,10 +444,12 @@ def bench_block(gdn2, dev, stream, pk, pk_kind, reps=20):
         torch.cuda.synchronize(dev)
         ms = statistics.median(a.elapsed_time(b) for a, b in ev)
         gbs = nbytes / (ms / 1e3) / 1e9
+        tr = traffic_record(name)
         out[name] = {"value": gbs, "unit": "GB/s", "workload": "layer_1p3b", "conv_len": 4,
                      "us_per_call": ms * 1e3, "launches": gdn2.launch_count() - c0,
                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                                  "frac": gbs / pk["hbm_gbs"], "traffic": None, "peak_source": pk_kind,
+                                  "frac": gbs / pk["hbm_gbs"],
+                                  "traffic": tr["dram_bytes_per_launch"] if tr else None, "peak_source": pk_kind,
                                   "algorithmic_bytes_per_launch": nbytes}}
     return out
 

@@ -113,3 +113,14 @@ def test_prologue_guard_bands_untouched(g):
     assert st == g.GDN2_OK
     for buf in bufs:
         assert torch.all(buf[:pad] == canary) and torch.all(buf[-pad:] == canary)
+
+
+def test_full_layer_shape_in_the_benchmark_launch(g):
+    """The 1.3B-layer shape (4 x 2048 tokens, 16 heads, d = 128, 4 taps), launched as the benchmark
+    launches it (one wave of long token runs), against the oracle on every output element."""
+    wl = W.WORKLOADS["layer_1p3b"]
+    d, outs = prologue_case(g, wl, 4, seed=0)
+    y = g.block_epilogue(d["xv"], d["z"], d["norm_weight"])
+    torch.cuda.synchronize()
+    ref = oracle.block_epilogue(np64(d["xv"]), np64(d["z"]), np64(d["norm_weight"]))
+    check(np64(y), ref, wl.dtype, "epilogue")
