@@ -27,6 +27,9 @@ Functions and the passages they follow:
   normalisation times a SiLU output gate), from "NVIDIA AIがGated DeltaNet-2を発表"
   (ai.warp-studio.com), section "アーキテクチャとパフォーマンスベンチマーク";
   the code is in ``block_oracle.c``.
+* :func:`recurrent_bwd` -- the reverse-mode gradient of :func:`recurrent`
+  (erase reading R1) with respect to q, k, v, alpha, b, w and S0, taken step by
+  step backwards through the same token loop; the code is in ``bwd_oracle.c``.
 """
 import ctypes
 import os
@@ -73,6 +76,8 @@ def _load():
         lib.oracle_block_prologue.restype = ci
         lib.oracle_block_epilogue.argtypes = [dp] * 4 + [ctypes.c_int64, ci, ci]
         lib.oracle_block_epilogue.restype = ci
+        lib.oracle_gdn2_recurrent_bwd.argtypes = [dp] * 16 + [ci] * 5 + [i64p, ci]
+        lib.oracle_gdn2_recurrent_bwd.restype = ci
         lib.oracle_max_threads.restype = ci
         _lib = lib
     return _lib
@@ -132,6 +137,27 @@ def recurrent(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, orientation=ERASE_
     if rc != 0:
         raise RuntimeError(f"oracle_gdn2_recurrent failed with {rc}")
     return o, ST
+
+
+def recurrent_bwd(q, k, v, alpha, b, w, dO, S0=None, dST=None, cu_seqlens=None, nthreads=0):
+    """Gradients of a loss L through the token loop, given ``dO = dL/do`` (the layout of o) and
+    ``dST = dL/dS_T`` (``[N, H, d_k, d_v]`` or ``None``: zero).
+
+    Returns ``(dq, dk, dv, dalpha, db, dw, dS0)`` as float64 arrays in the layouts of their inputs.
+    """
+    (q, k, v, alpha, b, w, S0, o, ST, N, T, H, dk_, dv_, cu, cup) = _prep(q, k, v, alpha, b, w, S0, cu_seqlens)
+    dO = _f64(dO)
+    if dO.shape != o.shape:
+        raise ValueError("dO must have the layout of o")
+    dST = None if dST is None else _f64(dST).reshape(N, H, dk_, dv_)
+    grads = [np.zeros_like(x) for x in (q, k, v, alpha, b, w)]
+    dS0 = np.zeros((N, H, dk_, dv_), dtype=np.float64)
+    rc = _load().oracle_gdn2_recurrent_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w),
+                                           _ptr(S0), _ptr(dO), _ptr(dST), *[_ptr(g) for g in grads],
+                                           _ptr(dS0), N, T, H, dk_, dv_, cup, int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_gdn2_recurrent_bwd failed with {rc}")
+    return (*grads, dS0)
 
 
 def recurrent_planted(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, plant=0):

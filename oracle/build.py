@@ -7,7 +7,7 @@ import subprocess
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "gdn2_oracle.c")
-SOURCES = [SRC, os.path.join(HERE, "block_oracle.c")]
+SOURCES = [SRC, os.path.join(HERE, "block_oracle.c"), os.path.join(HERE, "bwd_oracle.c")]
 OUT_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(OUT_DIR, "libgdn2_oracle.so")
 

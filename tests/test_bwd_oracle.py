@@ -1,0 +1,120 @@
+"""Pins of the backward oracle (the gradient of the token loop; CPU only).
+
+The gradient in ``oracle/bwd_oracle.c`` is derived by hand from the recurrence of
+"[논문] 게이트형 DeltaNet-2" (euno.news), section "방법론", and
+"NVIDIA AIがGated DeltaNet-2を発表" (ai.warp-studio.com), section "Gated DeltaNet-2の核心".
+It is pinned against two things that do not share its derivation:
+
+* central finite differences of the forward oracle, element by element, on tiny
+  dense and packed problems (every term of the chain rule moves some element);
+* torch autograd through a token loop written here from the same definition.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+rng = np.random.default_rng(7)
+
+
+def _problem(N, T, H, dk, dv, packed=None):
+    lead = (int(sum(packed)), H) if packed else (N, T, H)
+    x = {n: rng.standard_normal(lead + (dk,)) for n in ("q", "k", "b")}
+    x["alpha"] = rng.uniform(0.4, 1.0, lead + (dk,))
+    x["v"], x["w"], x["dO"] = (rng.standard_normal(lead + (dv,)) for _ in range(3))
+    nseq = len(packed) if packed else N
+    x["S0"] = rng.standard_normal((nseq, H, dk, dv)) * 0.3
+    x["dST"] = rng.standard_normal((nseq, H, dk, dv))
+    cu = None if not packed else np.concatenate([[0], np.cumsum(packed)]).astype(np.int64)
+    return x, cu
+
+
+def _loss(x, cu):
+    o, ST = oracle.recurrent(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"], S0=x["S0"], cu_seqlens=cu)
+    return float(np.sum(o * x["dO"]) + np.sum(ST * x["dST"]))
+
+
+NAMES = ("q", "k", "v", "alpha", "b", "w", "S0")
+
+
+def _grads(x, cu):
+    return dict(zip(NAMES, oracle.recurrent_bwd(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"], x["dO"],
+                                                S0=x["S0"], dST=x["dST"], cu_seqlens=cu)))
+
+
+@pytest.mark.parametrize("packed", [None, [3, 1, 0, 4]])
+def test_every_element_matches_central_differences(packed):
+    x, cu = _problem(2, 5, 2, 3, 2, packed)
+    g = _grads(x, cu)
+    eps = 1e-6
+    for name in NAMES:
+        flat = x[name].reshape(-1)
+        fd = np.empty_like(flat)
+        for e in range(flat.size):
+            keep = flat[e]
+            flat[e] = keep + eps
+            up = _loss(x, cu)
+            flat[e] = keep - eps
+            dn = _loss(x, cu)
+            flat[e] = keep
+            fd[e] = (up - dn) / (2 * eps)
+        np.testing.assert_allclose(g[name].reshape(-1), fd, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def _torch_loop(q, k, v, alpha, b, w, S0):
+    """Token loop for one (sequence, head), [T, d] tensors; returns o [T, d_v] and S_T."""
+    S = S0
+    outs = []
+    for t in range(q.shape[0]):
+        Sp = alpha[t][:, None] * S
+        delta = w[t] * v[t] - Sp.T @ (b[t] * k[t])
+        S = Sp + torch.outer(k[t], delta)
+        outs.append(S.T @ q[t])
+    return torch.stack(outs), S
+
+
+def test_matches_autograd_of_an_independent_loop():
+    N, T, H, dk, dv = 2, 17, 2, 6, 5
+    x, _ = _problem(N, T, H, dk, dv)
+    g = _grads(x, None)
+    for n in range(N):
+        for h in range(H):
+            leaves = {nm: torch.tensor(x[nm][n, :, h], requires_grad=True)
+                      for nm in ("q", "k", "v", "alpha", "b", "w")}
+            S0 = torch.tensor(x["S0"][n, h], requires_grad=True)
+            o, ST = _torch_loop(*[leaves[nm] for nm in ("q", "k", "v", "alpha", "b", "w")], S0)
+            L = (o * torch.tensor(x["dO"][n, :, h])).sum() + (ST * torch.tensor(x["dST"][n, h])).sum()
+            L.backward()
+            for nm, leaf in leaves.items():
+                np.testing.assert_allclose(g[nm][n, :, h], leaf.grad.numpy(), rtol=1e-10, atol=1e-12, err_msg=nm)
+            np.testing.assert_allclose(g["S0"][n, h], S0.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_empty_sequence_passes_the_state_gradient_through():
+    x, cu = _problem(1, 0, 2, 3, 4, packed=[2, 0, 3])
+    g = _grads(x, cu)
+    # the empty sequence 1 has S_T = S0, so dS0 = dST
+    np.testing.assert_array_equal(g["S0"][1], x["dST"][1])
+
+
+def test_zero_upstream_gives_zero_gradients():
+    x, cu = _problem(1, 6, 1, 4, 3)
+    x["dO"][:] = 0.0
+    x["dST"][:] = 0.0
+    for name, gr in _grads(x, cu).items():
+        assert not gr.any(), name
+
+
+def test_linearity_in_the_upstream_gradients():
+    # L is linear in (dO, dST), so the gradients are too: g(dO, dST) = g(dO, 0) + g(0, dST)
+    x, cu = _problem(2, 7, 2, 3, 3)
+    both = _grads(x, cu)
+    keep = x["dST"].copy()
+    x["dST"][:] = 0.0
+    only_o = _grads(x, cu)
+    x["dST"] = keep
+    x["dO"] = np.zeros_like(x["dO"])
+    only_s = _grads(x, cu)
+    for name in NAMES:
+        np.testing.assert_allclose(both[name], only_o[name] + only_s[name], rtol=1e-12, atol=1e-13)
