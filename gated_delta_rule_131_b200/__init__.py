@@ -10,8 +10,12 @@ Entry points (same names as the C ABI):
 
 * :func:`chunk_fwd` -- chunkwise parallel forward over whole sequences
   (``gdn2_chunk_fwd``);
+* :func:`chunk_bwd` -- gradients through the chunkwise forward
+  (``gdn2_chunk_bwd``);
 * :func:`decode_step` -- one recurrent step for a batch of single tokens
-  (``gdn2_decode_step``).
+  (``gdn2_decode_step``);
+* :func:`block_prologue`, :func:`block_epilogue` -- the work around the mixer
+  in its block (``gdn2_block_prologue``, ``gdn2_block_epilogue``).
 """
 import ctypes
 import os
@@ -63,6 +67,10 @@ def lib():
         L.gdn2_chunk_fwd_workspace_bytes.argtypes = [ci] * 7 + [ci]
         L.gdn2_chunk_fwd_workspace_bytes.restype = ctypes.c_size_t
         L.gdn2_launch_count.restype = ctypes.c_uint64
+        L.gdn2_chunk_bwd.argtypes = [vp] * 16 + [ci] * 5 + [vp, ci, vp]
+        L.gdn2_chunk_bwd.restype = ci
+        L.gdn2_chunk_bwd_workspace_bytes.argtypes = [ci] * 6
+        L.gdn2_chunk_bwd_workspace_bytes.restype = ctypes.c_size_t
         _lib = L
     return _lib
 
@@ -164,6 +172,41 @@ def chunk_fwd_noalloc(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, chunk=64, 
 
 
 NOALLOC_WORKSPACE_BYTES = 64 << 20  # GDN2_NOALLOC_WORKSPACE_BYTES in include/gdn2.h
+
+
+def chunk_bwd(q, k, v, alpha, b, w, dO, S0=None, dS_T=None, cu_seqlens=None, want_dS0=True, stream=None):
+    """Gradients of a loss through ``chunk_fwd`` given ``dO = dL/do`` and ``dS_T = dL/dS_T`` (or None).
+
+    Returns ``(dq, dk, dv, dalpha, db, dw, dS0)`` in the layouts and dtype of the inputs (``dS0``
+    float32 ``[N, H, d_k, d_v]``, None unless ``want_dS0``).  See ``gdn2_chunk_bwd`` in ``include/gdn2.h``.
+    """
+    if cu_seqlens is None:
+        B, T, H, dk = q.shape
+    else:
+        if cu_seqlens.dtype != torch.int32:
+            raise ValueError("gdn2: cu_seqlens must be int32")
+        B = cu_seqlens.numel() - 1
+        T, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype not in _DTYPES or any(x.dtype != q.dtype for x in (k, v, alpha, b, w, dO)):
+        raise ValueError("gdn2: q, k, v, alpha, b, w, dO must share dtype float32 or bfloat16")
+    if any(x is not None and x.dtype != torch.float32 for x in (S0, dS_T)):
+        raise ValueError("gdn2: S0 and dS_T must be float32")
+    grads = [torch.empty_like(x) for x in (q, k, v, alpha, b, w)]
+    dS0 = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device) if want_dS0 else None
+    _check_tensors(q, k, v, alpha, b, w, dO, S0, dS_T, *grads, dS0, cu_seqlens)
+    st = lib().gdn2_chunk_bwd(*[_ptr(x) for x in (q, k, v, alpha, b, w, S0, dO, dS_T)],
+                              *[_ptr(x) for x in grads], _ptr(dS0), B, T, H, dk, dv, _ptr(cu_seqlens),
+                              _DTYPES[q.dtype], _stream(stream))
+    if st != GDN2_OK:
+        raise Gdn2Error(st, "gdn2_chunk_bwd")
+    dq, dk_, dv_, dalpha, db, dw = grads
+    return dq, dk_, dv_, dalpha, db, dw, dS0
+
+
+def chunk_bwd_workspace_bytes(B, T, H, d_k, d_v, packed=False):
+    """Device bytes ``chunk_bwd`` takes from the library's pool for this shape."""
+    return int(lib().gdn2_chunk_bwd_workspace_bytes(B, T, H, d_k, d_v, int(bool(packed))))
 
 
 def block_prologue(xq, xk, xv, xa, xb, xw, conv_q, conv_k, conv_v, cu_seqlens=None, stream=None):

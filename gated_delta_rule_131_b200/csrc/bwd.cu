@@ -1,0 +1,327 @@
+// Backward of the Gated Delta Rule-2 recurrence (erase reading R1): gradients with respect to q,
+// k, v, alpha, b, w and S0, given dL/do and dL/dS_T.  The recurrence is the one of
+// "[논문] 게이트형 DeltaNet-2" (euno.news), section "방법론", and
+// "NVIDIA AIがGated DeltaNet-2を発表" (ai.warp-studio.com), section "Gated DeltaNet-2の核心":
+//
+//   S'_t = Diag(alpha_t) S_{t-1},  d_t = w_t (.) v_t - S'_t^T (b_t (.) k_t),
+//   S_t = S'_t + k_t d_t^T,        o_t = S_t^T q_t,
+//
+// and the chain rule taken backwards through it, with G = dL/dS_t:
+//
+//   G += q_t dO_t^T;  dq_t = S_t dO_t;  dd = G^T k_t;  dk_t = G d_t;
+//   dv_t = dd (.) w_t;  dw_t = dd (.) v_t;  da = -S'_t dd;  dS' = G - a_t dd^T;
+//   dalpha_t = rowsum(dS' (.) S_{t-1});  G = Diag(alpha_t) dS';  db_t = da (.) k_t;  dk_t += da (.) b_t.
+//
+// Every value column of the state evolves on its own (the key-side vectors are shared), so one
+// CTA takes one (sequence, head, tile of NJ value columns), one thread per key row i: it holds row
+// i of its tile of S and of G in registers.  Sums over the key rows (the erase read S'^T a and
+// dd = G^T k) are block reductions; sums over the value columns (dq, dk, dalpha, da) are formed in
+// each thread over its tile and added across tiles with fp32 reductions in L2, into a buffer that
+// a second kernel converts to the output type.
+//
+// States are not kept for every token: a first forward pass stores the tile's state every CK
+// tokens (checkpoints in the workspace); the backward pass rebuilds each segment's CK states in
+// shared memory from its checkpoint, then walks the segment backwards.
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace gdn2 {
+namespace {
+
+constexpr int NJ = 16;  // value columns per CTA
+constexpr int CK = 8;   // tokens per checkpoint segment
+
+struct BwdParams {
+  const void *q, *k, *v, *alpha, *b, *w, *dO;
+  const float *S0, *dST;
+  float *acc;        // [tokens, H, 4, d_k] fp32: dq, dk, dalpha, db summed over the tiles (zeroed)
+  float4 *ck;        // checkpoints [slots, H, tiles, NJ / 4, d_k] float4
+  void *dv, *dw;     // [tokens, H, d_v]
+  float *dS0;        // [N, H, d_k, d_v] or nullptr
+  const int32_t *cu;  // packed offsets [N+1] or nullptr
+  int N, T, H, dv_;
+};
+
+template <typename T>
+__device__ __forceinline__ float ld(const void *p, size_t i) {
+  return to_f32(static_cast<const T *>(p)[i]);
+}
+
+// Sum of p[0..15] over the 32 lanes of a warp, transposed: lane l ends with the sum of index l >> 1
+// (lanes 2m and 2m+1 both hold index m).  16 shuffles instead of 80.
+__device__ __forceinline__ float warp_reduce16(float (&p)[NJ], int lane) {
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const bool up = lane & 16;
+    const float send = up ? p[m] : p[m + 8], keep = up ? p[m + 8] : p[m];
+    p[m] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const bool up = lane & 8;
+    const float send = up ? p[m] : p[m + 4], keep = up ? p[m + 4] : p[m];
+    p[m] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+#pragma unroll
+  for (int m = 0; m < 2; ++m) {
+    const bool up = lane & 4;
+    const float send = up ? p[m] : p[m + 2], keep = up ? p[m + 2] : p[m];
+    p[m] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+  }
+  {
+    const bool up = lane & 2;
+    const float send = up ? p[0] : p[1], keep = up ? p[1] : p[0];
+    p[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+  }
+  return p[0] + __shfl_xor_sync(0xffffffffu, p[0], 1);
+}
+
+template <typename T, int DK>
+struct __align__(16) BwdSmem {
+  float4 seg[CK][NJ / 4][DK];  // the tile's state before each token of the segment, row-interleaved
+  float u[CK][NJ];             // w (.) v of the segment's tokens
+  float dO[CK][NJ];            // dL/do of the segment's tokens
+  float dl[CK][NJ];            // d_t of the segment's tokens (from the rebuild)
+  float red[DK / 32][NJ];      // warp partials of a block reduction
+  float bc[NJ];                // the reduced vector, broadcast
+};
+
+// One (sequence, head, NJ-column tile).  blockDim = DK.
+template <typename T, int DK>
+__global__ void __launch_bounds__(DK) chunk_bwd_kernel(const BwdParams p) {
+  extern __shared__ __align__(16) uint8_t dsm[];
+  BwdSmem<T, DK> &sm = *reinterpret_cast<BwdSmem<T, DK> *>(dsm);
+  const int tile = blockIdx.x, h = blockIdx.y, n = blockIdx.z, i = threadIdx.x;
+  const int lane = i & 31, warp = i >> 5;
+  const int tiles = p.dv_ / NJ, j0 = tile * NJ, H = p.H, DV = p.dv_;
+  long long bos, len;
+  if (p.cu) {  // offsets clamped to [0, T_total], so that bad offsets cannot index out of bounds
+    bos = min(max(p.cu[n], 0), p.T);
+    len = min(max(p.cu[n + 1], (int)bos), p.T) - bos;
+  } else {
+    bos = (long long)n * p.T;
+    len = p.T;
+  }
+  const int nseg = (int)((len + CK - 1) / CK);
+  const long long slot0 = bos / CK + n;  // distinct slots for every segment of every sequence
+  auto ck_at = [&](int m) { return p.ck + ((((slot0 + m) * H + h) * tiles + tile) * (NJ / 4)) * DK + i; };
+  auto krow = [&](long long t) { return ((size_t)t * H + h) * DK + i; };
+  auto vcol = [&](long long t, int j) { return ((size_t)t * H + h) * DV + j0 + j; };
+
+  float s[NJ];
+  {
+    const size_t off = (((size_t)n * H + h) * DK + i) * DV + j0;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) s[j] = p.S0 ? p.S0[off + j] : 0.f;
+  }
+  // Block reduction of p16 over the key rows; threads j < NJ get sum_j and run `use(j, sum_j)`,
+  // whose result is broadcast in sm.bc.
+  auto reduce = [&](float (&v)[NJ], auto use) {
+    const float r = warp_reduce16(v, lane);
+    if ((lane & 1) == 0) sm.red[warp][lane >> 1] = r;
+    __syncthreads();
+    if (i < NJ) {
+      float t = 0.f;
+#pragma unroll
+      for (int w = 0; w < DK / 32; ++w) t += sm.red[w][i];
+      sm.bc[i] = use(i, t);
+    }
+    __syncthreads();
+  };
+  // Load the segment's w (.) v (and dL/do) into shared memory.
+  auto load_cols = [&](long long t0, int nt, bool with_do) {
+    for (int e = i; e < CK * NJ; e += DK) {
+      const int u = e / NJ, j = e % NJ;
+      float uu = 0.f, dd = 0.f;
+      if (u < nt) {
+        uu = ld<T>(p.w, vcol(t0 + u, j)) * ld<T>(p.v, vcol(t0 + u, j));
+        if (with_do) dd = ld<T>(p.dO, vcol(t0 + u, j));
+      }
+      sm.u[u][j] = uu;
+      sm.dO[u][j] = dd;
+    }
+  };
+  // One forward token: s <- alpha s; d = u - s^T a; s += k d^T.  d is left in sm.dl[u].
+  auto forward = [&](int u, float al, float kk, float bb) {
+    float v[NJ];
+    const float ai = bb * kk;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      s[j] *= al;
+      v[j] = ai * s[j];
+    }
+    reduce(v, [&](int j, float r) {
+      const float d = sm.u[u][j] - r;
+      sm.dl[u][j] = d;
+      return d;
+    });
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) s[j] = fmaf(kk, sm.bc[j], s[j]);
+  };
+
+  // Pass 1: forward over the sequence, storing the state before every segment.
+  for (int m = 0; m < nseg; ++m) {
+    const long long t0 = bos + (long long)m * CK;
+    const int nt = (int)min((long long)CK, len - (long long)m * CK);
+    float4 *c = ck_at(m);
+#pragma unroll
+    for (int q4 = 0; q4 < NJ / 4; ++q4) c[q4 * DK] = make_float4(s[4 * q4], s[4 * q4 + 1], s[4 * q4 + 2], s[4 * q4 + 3]);
+    load_cols(t0, nt, false);
+    for (int u = 0; u < nt; ++u)
+      forward(u, ld<T>(p.alpha, krow(t0 + u)), ld<T>(p.k, krow(t0 + u)), ld<T>(p.b, krow(t0 + u)));
+  }
+
+  // Pass 2: backwards, one segment at a time.
+  float g[NJ];
+  {
+    const size_t off = (((size_t)n * H + h) * DK + i) * DV + j0;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) g[j] = p.dST ? p.dST[off + j] : 0.f;
+  }
+  for (int m = nseg - 1; m >= 0; --m) {
+    const long long t0 = bos + (long long)m * CK;
+    const int nt = (int)min((long long)CK, len - (long long)m * CK);
+    const float4 *c = ck_at(m);
+#pragma unroll
+    for (int q4 = 0; q4 < NJ / 4; ++q4) {
+      const float4 x = c[q4 * DK];
+      s[4 * q4] = x.x;
+      s[4 * q4 + 1] = x.y;
+      s[4 * q4 + 2] = x.z;
+      s[4 * q4 + 3] = x.w;
+    }
+    load_cols(t0, nt, true);
+    float ral[CK], rk[CK], rb[CK], rq[CK];
+#pragma unroll
+    for (int u = 0; u < CK; ++u) {
+      const bool in = u < nt;
+      ral[u] = in ? ld<T>(p.alpha, krow(t0 + u)) : 0.f;
+      rk[u] = in ? ld<T>(p.k, krow(t0 + u)) : 0.f;
+      rb[u] = in ? ld<T>(p.b, krow(t0 + u)) : 0.f;
+      rq[u] = in ? ld<T>(p.q, krow(t0 + u)) : 0.f;
+    }
+    // rebuild: the state before each token of the segment, and d_t
+#pragma unroll
+    for (int u = 0; u < CK; ++u) {
+      if (u >= nt) break;
+#pragma unroll
+      for (int q4 = 0; q4 < NJ / 4; ++q4)
+        sm.seg[u][q4][i] = make_float4(s[4 * q4], s[4 * q4 + 1], s[4 * q4 + 2], s[4 * q4 + 3]);
+      forward(u, ral[u], rk[u], rb[u]);
+    }
+    // backwards through the segment
+#pragma unroll
+    for (int u = CK - 1; u >= 0; --u) {
+      if (u >= nt) continue;
+      const long long t = t0 + u;
+      const float al = ral[u], kk = rk[u], bb = rb[u], qq = rq[u], ai = bb * kk;
+      float sp[NJ];
+#pragma unroll
+      for (int q4 = 0; q4 < NJ / 4; ++q4) {
+        const float4 x = sm.seg[u][q4][i];
+        sp[4 * q4] = x.x;
+        sp[4 * q4 + 1] = x.y;
+        sp[4 * q4 + 2] = x.z;
+        sp[4 * q4 + 3] = x.w;
+      }
+      float dq = 0.f, dk = 0.f, v[NJ];
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const float doj = sm.dO[u][j], dlj = sm.dl[u][j];
+        g[j] = fmaf(qq, doj, g[j]);
+        const float st = fmaf(kk, dlj, al * sp[j]);  // S_t, as the forward formed it
+        dq = fmaf(st, doj, dq);
+        dk = fmaf(g[j], dlj, dk);
+        v[j] = g[j] * kk;
+      }
+      reduce(v, [&](int j, float dd) {
+        const size_t o = vcol(t, j);
+        const float vv = ld<T>(p.v, o), ww = ld<T>(p.w, o);
+        static_cast<T *>(p.dv)[o] = from_f32<T>(dd * ww);
+        static_cast<T *>(p.dw)[o] = from_f32<T>(dd * vv);
+        return dd;
+      });
+      float da = 0.f, dal = 0.f;
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const float dd = sm.bc[j], spj = al * sp[j];
+        da = fmaf(-spj, dd, da);
+        const float dsp = fmaf(-ai, dd, g[j]);
+        dal = fmaf(dsp, sp[j], dal);
+        g[j] = al * dsp;
+      }
+      dk = fmaf(da, bb, dk);
+      float *acc = p.acc + ((size_t)t * H + h) * 4 * DK + i;
+      atomicAdd(acc, dq);
+      atomicAdd(acc + DK, dk);
+      atomicAdd(acc + 2 * DK, dal);
+      atomicAdd(acc + 3 * DK, da * kk);
+    }
+  }
+  if (p.dS0) {
+    const size_t off = (((size_t)n * H + h) * DK + i) * DV + j0;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) p.dS0[off + j] = g[j];
+  }
+}
+
+// acc [rows, 4, d_k] fp32 -> dq, dk, dalpha, db [rows, d_k] in the output type.
+template <typename T>
+__global__ void __launch_bounds__(256) bwd_finish_kernel(const float *acc, T *dq, T *dk, T *dal, T *db, size_t rows,
+                                                        int DK) {
+  const size_t n = rows * DK;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
+    const size_t r = e / DK, c = e - r * DK;
+    const float *a = acc + r * 4 * DK + c;
+    dq[e] = from_f32<T>(a[0]);
+    dk[e] = from_f32<T>(a[DK]);
+    dal[e] = from_f32<T>(a[2 * DK]);
+    db[e] = from_f32<T>(a[3 * DK]);
+  }
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+template <typename T, int DK>
+cudaError_t bwd_t(const BwdArgs &a, void *ws, cudaStream_t stream) {
+  const long long tokens = a.cu ? (long long)a.T : (long long)a.B * a.T;
+  BwdParams p{};
+  p.q = a.q; p.k = a.k; p.v = a.v; p.alpha = a.alpha; p.b = a.b; p.w = a.w; p.dO = a.dO;
+  p.S0 = a.S0; p.dST = a.dST; p.dv = a.dv; p.dw = a.dw; p.dS0 = a.dS0; p.cu = a.cu;
+  p.N = a.B; p.T = a.T; p.H = a.H; p.dv_ = a.Dv;
+  const size_t acc_bytes = align256((size_t)tokens * a.H * 4 * DK * sizeof(float));
+  p.acc = static_cast<float *>(ws);
+  p.ck = reinterpret_cast<float4 *>(static_cast<uint8_t *>(ws) + acc_bytes);
+  cudaError_t err = cudaMemsetAsync(p.acc, 0, (size_t)tokens * a.H * 4 * DK * sizeof(float), stream);
+  if (err != cudaSuccess) return err;
+  const int smem = (int)sizeof(BwdSmem<T, DK>);
+  err = cudaFuncSetAttribute(chunk_bwd_kernel<T, DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return err;
+  note_launch();
+  chunk_bwd_kernel<T, DK><<<dim3(a.Dv / NJ, a.H, a.B), DK, smem, stream>>>(p);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  if (tokens == 0) return cudaSuccess;
+  const size_t rows = (size_t)tokens * a.H;
+  const unsigned blocks = (unsigned)std::min<size_t>((rows * DK + 255) / 256, (size_t)148 * 16);
+  note_launch();
+  bwd_finish_kernel<T><<<blocks, 256, 0, stream>>>(p.acc, static_cast<T *>(a.dq), static_cast<T *>(a.dk),
+                                                  static_cast<T *>(a.dalpha), static_cast<T *>(a.db), rows, DK);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, bool packed) {
+  const long long tokens = packed ? (long long)T : (long long)B * T;
+  const long long slots = tokens / CK + B + 1;
+  return align256((size_t)tokens * H * 4 * dk * sizeof(float)) + (size_t)slots * H * dk * dv * sizeof(float);
+}
+
+cudaError_t launch_chunk_bwd(const BwdArgs &a, bool bf16, void *ws, cudaStream_t stream) {
+  if (a.Dk == 128)
+    return bf16 ? bwd_t<__nv_bfloat16, 128>(a, ws, stream) : bwd_t<float, 128>(a, ws, stream);
+  return bf16 ? bwd_t<__nv_bfloat16, 64>(a, ws, stream) : bwd_t<float, 64>(a, ws, stream);
+}
+
+}  // namespace gdn2

@@ -68,6 +68,16 @@ struct BlockEpilogueArgs {
   int H, dv;
 };
 
+// Arguments of one gdn2_chunk_bwd call (validated by the API layer).
+struct BwdArgs {
+  const void *q, *k, *v, *alpha, *b, *w, *dO;  // forward inputs and dL/do, [tokens, H, d]
+  const float *S0, *dST;                       // [B, H, d_k, d_v] or nullptr (zeros)
+  void *dq, *dk, *dv, *dalpha, *db, *dw;        // gradients, layouts of their inputs
+  float *dS0;                                  // [B, H, d_k, d_v] or nullptr
+  const int32_t *cu;                           // packed offsets [B+1] or nullptr
+  int B, T, H, Dk, Dv;
+};
+
 // Host side: every kernel launch of the library is counted here.
 void note_launch();
 
@@ -78,6 +88,10 @@ cudaError_t launch_chunk_simt(const ChunkArgs &a, bool bf16, cudaStream_t stream
 // The workspace depends only on the batch shape (B sequences, T tokens each or in total, H heads, d_v).
 bool chunk_wy_supported(int B, int T, int H, int dk, int dv, bool packed, bool bf16);
 size_t chunk_wy_workspace_bytes(int B, int T, int H, int dv, bool packed);
+// Backward of the recurrence over a workspace of chunk_bwd_workspace_bytes(...) bytes, 256-byte
+// aligned (a gradient accumulator it clears, and state checkpoints it writes before reading).
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, bool packed);
+cudaError_t launch_chunk_bwd(const BwdArgs &a, bool bf16, void *ws, cudaStream_t stream);
 cudaError_t launch_chunk_wy(const ChunkArgs &a, void *workspace, cudaStream_t stream);
 cudaError_t launch_bounded_wait_probe(uint64_t limit_ns, cudaStream_t stream);
 // Reads (and optionally clears) the device-side status word that bounded waits set.

@@ -77,6 +77,19 @@ cudaError_t run_chunk_wy(const gdn2::ChunkArgs &a, cudaStream_t stream) {
   return err;
 }
 
+// The backward with a workspace taken from the pool and returned to it on `stream`.
+cudaError_t run_chunk_bwd(const gdn2::BwdArgs &a, bool bf16, cudaStream_t stream) {
+  const size_t bytes = gdn2::chunk_bwd_workspace_bytes(a.B, a.T, a.H, a.Dk, a.Dv, a.cu != nullptr);
+  cudaMemPool_t pool;
+  void *ws = nullptr;
+  cudaError_t err;
+  if ((err = workspace_pool(&pool)) != cudaSuccess) return err;
+  if ((err = cudaMallocFromPoolAsync(&ws, bytes, pool, stream)) != cudaSuccess) return err;
+  err = gdn2::launch_chunk_bwd(a, bf16, ws, stream);
+  const cudaError_t ferr = cudaFreeAsync(ws, stream);
+  return err == cudaSuccess ? ferr : err;
+}
+
 // The fixed workspace of gdn2_chunk_fwd_noalloc: a file-scope device array, so that entry point
 // allocates nothing.  Its device address is looked up once per device, with that device current.
 constexpr size_t kNoallocBytes = (size_t)GDN2_NOALLOC_WORKSPACE_BYTES;
@@ -193,6 +206,35 @@ gdn2_status gdn2_chunk_fwd_noalloc(const void *q, const void *k, const void *v, 
   cudaError_t err = noalloc_workspace(&ws);
   if (err == cudaSuccess) err = gdn2::launch_chunk_wy(a, ws, (cudaStream_t)stream);
   return err == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+}
+
+gdn2_status gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *alpha, const void *b,
+                           const void *w, const float *S0, const void *dO, const float *dS_T, void *dq, void *dk,
+                           void *dv, void *dalpha, void *db, void *dw, float *dS0, int B, int T, int H, int d_k,
+                           int d_v, const int32_t *cu_seqlens, gdn2_dtype dtype, gdn2_stream_t stream) {
+  if (B < 0 || T < 0 || H <= 0) return GDN2_ERR_INVALID_ARG;
+  if (dtype != GDN2_F32 && dtype != GDN2_BF16) return GDN2_ERR_INVALID_ARG;
+  if (!supported_dk(d_k) || !supported_dv(d_v)) return GDN2_ERR_UNSUPPORTED;
+  const long long tokens = cu_seqlens ? (long long)T : (long long)B * T;
+  if (!fits(tokens, H, 4 * (d_v > d_k ? d_v : d_k), 1) || !fits(B, H, d_k, d_v)) return GDN2_ERR_INVALID_ARG;
+  if (!fits(tokens / 8 + B + 1, H, d_k, d_v) || (long long)B * H > INT_MAX / 64) return GDN2_ERR_INVALID_ARG;
+  if (tokens > 0)
+    for (const void *p : {q, k, v, alpha, b, w, dO, (const void *)dq, (const void *)dk, (const void *)dv,
+                          (const void *)dalpha, (const void *)db, (const void *)dw})
+      if (!p || !aligned16(p)) return GDN2_ERR_INVALID_ARG;
+  for (const void *p : {(const void *)S0, (const void *)dS_T, (const void *)dS0})
+    if (p && !aligned16(p)) return GDN2_ERR_INVALID_ARG;
+  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return GDN2_ERR_INVALID_ARG;
+  if (B == 0) return GDN2_OK;
+  const gdn2::BwdArgs a{q, k, v, alpha, b, w, dO, S0, dS_T, dq, dk, dv, dalpha, db, dw, dS0, cu_seqlens,
+                        B, T, H, d_k, d_v};
+  const cudaError_t err = run_chunk_bwd(a, dtype == GDN2_BF16, (cudaStream_t)stream);
+  return err == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+}
+
+size_t gdn2_chunk_bwd_workspace_bytes(int B, int T, int H, int d_k, int d_v, int packed) {
+  if (B <= 0 || T < 0 || H <= 0 || !supported_dk(d_k) || !supported_dv(d_v)) return 0;
+  return gdn2::chunk_bwd_workspace_bytes(B, T, H, d_k, d_v, packed != 0);
 }
 
 size_t gdn2_chunk_fwd_workspace_bytes(int B, int T, int H, int d_k, int d_v, int chunk, int packed,

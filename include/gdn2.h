@@ -31,8 +31,8 @@
  *     takes a workspace of gdn2_chunk_fwd_workspace_bytes() bytes from a
  *     stream-ordered memory pool that the library creates once per device, and
  *     gives it back on `stream` after its kernels; the pool keeps memory given
- *     back to it for later calls until the process exits.  No other call
- *     allocates device memory.
+ *     back to it for later calls until the process exits.  gdn2_chunk_bwd takes
+ *     its workspace from the same pool.  No other call allocates device memory.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and never synchronise.  A validation failure returns before any
  *     launch and writes nothing.  A launch failure returns GDN2_ERR_CUDA.  No
@@ -134,6 +134,43 @@ GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const void *q, const void *k, const 
  */
 GDN2_API size_t gdn2_chunk_fwd_workspace_bytes(int B, int T, int H, int d_k, int d_v, int chunk, int packed,
                                                gdn2_dtype dtype);
+
+/*
+ * gdn2_chunk_bwd -- gradients of a loss L through gdn2_chunk_fwd (erase reading R1).
+ *
+ * Passage: the recurrence of "[논문] 게이트형 DeltaNet-2" (euno.news), section "방법론",
+ * and "NVIDIA AIがGated DeltaNet-2を発表" (ai.warp-studio.com), section
+ * "Gated DeltaNet-2の核心"; the pages name a gate-aware backward of the chunked
+ * form as a contribution but print no formula, so this is the chain rule taken
+ * backwards through the token loop that gdn2_chunk_fwd computes:
+ *     G += q_t dO_t^T,  dq_t = S_t dO_t,  dd = G^T k_t,  dk_t = G d_t + da (.) b_t,
+ *     dv_t = dd (.) w_t,  dw_t = dd (.) v_t,  da = -(Diag(alpha_t) S_{t-1}) dd,
+ *     db_t = da (.) k_t,  dS' = G - (b_t (.) k_t) dd^T,
+ *     dalpha_t = rowsum(dS' (.) S_{t-1}),  G <- Diag(alpha_t) dS',
+ * with G = dL/dS_t starting from dL/dS_T, d_t = w_t (.) v_t - (Diag(alpha_t) S_{t-1})^T (b_t (.) k_t),
+ * and dS0 = G after the first token.
+ *
+ *   q, k, v, alpha, b, w, S0, B, T, H, d_k, d_v, cu_seqlens, dtype: as for gdn2_chunk_fwd (the same
+ *           forward inputs; S0 may be NULL = zeros).
+ *   dO      [.., H, d_v] in dtype: dL/do (layout of o).
+ *   dS_T    [B, H, d_k, d_v] fp32: dL/dS_T, or NULL (zero).
+ *   dq, dk, dalpha, db   [.., H, d_k] in dtype (out), dv, dw [.., H, d_v] in dtype (out).
+ *   dS0     [B, H, d_k, d_v] fp32 (out), or NULL (not returned).  dS0 may alias dS_T.
+ * Arithmetic is fp32; the gradients are rounded to dtype once.  The call takes a workspace of
+ * gdn2_chunk_bwd_workspace_bytes() bytes from the library's pool (a gradient accumulator and
+ * state checkpoints every 8 tokens) and gives it back on `stream`.  Errors as for gdn2_chunk_fwd.
+ */
+GDN2_API gdn2_status gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *alpha,
+                                    const void *b, const void *w, const float *S0, const void *dO,
+                                    const float *dS_T, void *dq, void *dk, void *dv, void *dalpha, void *db,
+                                    void *dw, float *dS0, int B, int T, int H, int d_k, int d_v,
+                                    const int32_t *cu_seqlens, gdn2_dtype dtype, gdn2_stream_t stream);
+
+/*
+ * gdn2_chunk_bwd_workspace_bytes -- device bytes gdn2_chunk_bwd takes from its pool for a call of
+ * this shape (packed != 0: B sequences, T tokens in total); 0 for an unsupported shape.  Host only.
+ */
+GDN2_API size_t gdn2_chunk_bwd_workspace_bytes(int B, int T, int H, int d_k, int d_v, int packed);
 
 /*
  * gdn2_decode_step -- one recurrent step for a batch of single tokens.
