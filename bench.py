@@ -8,7 +8,8 @@ H=16, d_k=d_v=128, chunk 64, bf16 inputs, fp32 state, seeded synthetic data).
 collective on the data path: weak scaling).  The same JSON line carries the
 decode measurement (256 x 16 heads, 1024 single-token steps replayed from one
 CUDA graph) as ``decode_step``, the block prologue and epilogue around the mixer
-(``block_prologue``, ``block_epilogue``), the roofline of the dominant kernel, the CPU
+(``block_prologue``, ``block_epilogue``), the backward on the same workload
+(``chunk_bwd``), the roofline of the dominant kernel, the CPU
 oracle baseline, the end-to-end number through host buffers, and clocks.
 
 ``--impl reference`` times the fp64 CPU oracle (the only reference that
@@ -234,7 +235,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-block", action="store_true", help="skip the block prologue/epilogue measurement")
-    ap.add_argument("--profile-case", choices=["chunk", "decode", "block"],
+    ap.add_argument("--no-bwd", action="store_true", help="skip the backward measurement")
+    ap.add_argument("--profile-case", choices=["chunk", "decode", "block", "bwd", "bwd_small"],
                     help="run one warm-up and one measured launch of that kernel on its full workload, for ncu")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -324,6 +326,8 @@ def main():
     # ------------------------------------------------------------ block prologue / epilogue around the mixer
     if not args.no_block:
         line.update(bench_block(gdn2, dev, stream, pk, pk_kind))
+    if not args.no_bwd:
+        line["chunk_bwd"] = bench_bwd(gdn2, dev, stream, pk, pk_kind)
 
     # ------------------------------------------------------------ end to end through host buffers
     line["e2e"] = bench_e2e(gdn2, wl, sets[0], dev, stream, ws, tokens)
@@ -351,6 +355,16 @@ def profile_case(which):
         d = W.chunk_inputs(wl, device=dev, seed=0)
         for _ in range(2):
             gdn2.chunk_fwd(*[d[n] for n in TOK], S0=d["S0"])
+    elif which in ("bwd", "bwd_small"):
+        wl = W.WORKLOADS["layer_1p3b"]
+        if which == "bwd_small":  # one sequence of 512 tokens: 128 CTAs, a few hundred MB on the device
+            wl = W.Workload("bwd_small", B=1, T=512, H=16, dk=128, dv=128)
+        d = W.chunk_inputs(wl, device=dev, seed=0)
+        gen = torch.Generator(device="cpu").manual_seed(1000)
+        dO = torch.randn(d["q"].shape[:-1] + (wl.dv,), generator=gen).to(dev, torch.bfloat16)
+        dST = torch.randn(d["S0"].shape, generator=gen).to(dev) * 0.1
+        for _ in range(2):
+            gdn2.chunk_bwd(*[d[n] for n in TOK], dO, S0=d["S0"], dS_T=dST)
     elif which == "block":
         wl = W.WORKLOADS["layer_1p3b"]
         d = W.block_inputs(wl, device=dev, seed=0, conv_len=4)
@@ -452,6 +466,45 @@ def bench_block(gdn2, dev, stream, pk, pk_kind, reps=20):
                                   "traffic": tr["dram_bytes_per_launch"] if tr else None, "peak_source": pk_kind,
                                   "algorithmic_bytes_per_launch": nbytes}}
     return out
+
+
+def bwd_bytes(wl, tokens, nseq):
+    """Algorithmic bytes of one backward call: the six forward inputs and dL/do read, the six
+    gradients written (bf16), and S0, dL/dS_T read and dS0 written (fp32)."""
+    e = 2 if wl.dtype == "bf16" else 4
+    th = tokens * wl.H
+    return th * (2 * (4 * wl.dk + 2 * wl.dv) + wl.dv) * e + 3 * nseq * wl.H * wl.dk * wl.dv * 4
+
+
+def bench_bwd(gdn2, dev, stream, pk, pk_kind, reps=5):
+    """gdn2_chunk_bwd on the 1.3B-layer workload (seeded dL/do and dL/dS_T)."""
+    wl = W.WORKLOADS["layer_1p3b"]
+    tokens = wl.B * wl.T
+    d = W.chunk_inputs(wl, device=dev, seed=0)
+    gen = torch.Generator(device="cpu").manual_seed(1000)
+    dO = torch.randn(d["q"].shape[:-1] + (wl.dv,), generator=gen).to(dev, torch.bfloat16)
+    dST = torch.randn(d["S0"].shape, generator=gen).to(dev) * 0.1
+    fn = lambda: gdn2.chunk_bwd(*[d[n] for n in TOK], dO, S0=d["S0"], dS_T=dST, stream=stream)
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize(dev)
+    c0 = gdn2.launch_count()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in ev:
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    nbytes = bwd_bytes(wl, tokens, wl.B)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    tr = traffic_record("chunk_bwd")
+    return {"value": tokens / (ms / 1e3), "unit": "tokens/s", "workload": "layer_1p3b", "ms_per_call": ms,
+            "launches": gdn2.launch_count() - c0,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "traffic": tr["dram_bytes_per_launch"] if tr else None,
+                         "peak_source": pk_kind, "algorithmic_bytes_per_launch": nbytes,
+                         "note": "issue- and latency-bound SIMT kernel (about 655 instructions per warp and token)"}}
 
 
 def bench_e2e(gdn2, wl, d, dev, stream, ws, tokens, steps=3):

@@ -35,8 +35,9 @@ constexpr int CK = 8;   // tokens per checkpoint segment
 struct BwdParams {
   const void *q, *k, *v, *alpha, *b, *w, *dO;
   const float *S0, *dST;
-  float *acc;        // [tokens, H, 4, d_k] fp32: dq, dk, dalpha, db summed over the tiles (zeroed)
+  float4 *acc;       // [tokens, H, d_k] x (dq, dk, dalpha, db) fp32, summed over the tiles (zeroed)
   float4 *ck;        // checkpoints [slots, H, tiles, NJ / 4, d_k] float4
+  float *dl;         // d_t of every token [tokens, H, d_v] fp32, from the first pass
   void *dv, *dw;     // [tokens, H, d_v]
   float *dS0;        // [N, H, d_k, d_v] or nullptr
   const int32_t *cu;  // packed offsets [N+1] or nullptr
@@ -46,6 +47,12 @@ struct BwdParams {
 template <typename T>
 __device__ __forceinline__ float ld(const void *p, size_t i) {
   return to_f32(static_cast<const T *>(p)[i]);
+}
+
+// Adds four floats to 16 aligned bytes of global memory as one reduction in L2.
+__device__ __forceinline__ void red_add4(float4 *p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
 }
 
 // Sum of p[0..15] over the 32 lanes of a warp, transposed: lane l ends with the sum of index l >> 1
@@ -79,19 +86,23 @@ __device__ __forceinline__ float warp_reduce16(float (&p)[NJ], int lane) {
 
 template <typename T, int DK>
 struct __align__(16) BwdSmem {
+  static constexpr int NW = DK / 32;
   float4 seg[CK][NJ / 4][DK];  // the tile's state before each token of the segment, row-interleaved
   float u[CK][NJ];             // w (.) v of the segment's tokens
+  float vv[CK][NJ];            // v and w of the segment's tokens (for dv, dw)
+  float ww[CK][NJ];
   float dO[CK][NJ];            // dL/do of the segment's tokens
-  float dl[CK][NJ];            // d_t of the segment's tokens (from the rebuild)
-  float red[DK / 32][NJ];      // warp partials of a block reduction
-  float bc[NJ];                // the reduced vector, broadcast
+  float dl[CK][NJ];            // d_t of the segment's tokens
+  float red[2][NJ][NW];        // warp partials of a block reduction, double-buffered
 };
 
-// One (sequence, head, NJ-column tile).  blockDim = DK.
+// One (sequence, head, NJ-column tile).  blockDim = DK; three blocks of 128 rows per SM.
 template <typename T, int DK>
-__global__ void __launch_bounds__(DK) chunk_bwd_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(DK, 384 / DK) chunk_bwd_kernel(const BwdParams p) {
+  using Smem = BwdSmem<T, DK>;
+  constexpr int NW = Smem::NW;
   extern __shared__ __align__(16) uint8_t dsm[];
-  BwdSmem<T, DK> &sm = *reinterpret_cast<BwdSmem<T, DK> *>(dsm);
+  Smem &sm = *reinterpret_cast<Smem *>(dsm);
   const int tile = blockIdx.x, h = blockIdx.y, n = blockIdx.z, i = threadIdx.x;
   const int lane = i & 31, warp = i >> 5;
   const int tiles = p.dv_ / NJ, j0 = tile * NJ, H = p.H, DV = p.dv_;
@@ -115,61 +126,83 @@ __global__ void __launch_bounds__(DK) chunk_bwd_kernel(const BwdParams p) {
 #pragma unroll
     for (int j = 0; j < NJ; ++j) s[j] = p.S0 ? p.S0[off + j] : 0.f;
   }
-  // Block reduction of p16 over the key rows; threads j < NJ get sum_j and run `use(j, sum_j)`,
-  // whose result is broadcast in sm.bc.
-  auto reduce = [&](float (&v)[NJ], auto use) {
-    const float r = warp_reduce16(v, lane);
-    if ((lane & 1) == 0) sm.red[warp][lane >> 1] = r;
-    __syncthreads();
-    if (i < NJ) {
-      float t = 0.f;
-#pragma unroll
-      for (int w = 0; w < DK / 32; ++w) t += sm.red[w][i];
-      sm.bc[i] = use(i, t);
+  // Block reduction of v over the key rows: every thread gets all NJ sums.  One barrier: the
+  // partials alternate between two buffers, and a buffer is written again only after the next
+  // reduction's barrier, which every reader of it has passed.
+  int par = 0;
+  auto red_sum = [&](int buf, int j) {  // the block's sum of index j from the warp partials
+    if constexpr (NW == 4) {
+      const float4 x = *reinterpret_cast<const float4 *>(sm.red[buf][j]);
+      return (x.x + x.y) + (x.z + x.w);
+    } else {
+      const float2 x = *reinterpret_cast<const float2 *>(sm.red[buf][j]);
+      return x.x + x.y;
     }
-    __syncthreads();
   };
-  // Load the segment's w (.) v (and dL/do) into shared memory.
-  auto load_cols = [&](long long t0, int nt, bool with_do) {
+  auto reduce = [&](float (&v)[NJ], float (&tot)[NJ]) {
+    const float r = warp_reduce16(v, lane);
+    if ((lane & 1) == 0) sm.red[par][lane >> 1][warp] = r;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) tot[j] = red_sum(par, j);
+    par ^= 1;
+  };
+  // A segment's inputs, all loads issued together: the value-side ones into shared memory, this
+  // row's alpha, k, b (and q) into registers.
+  float ral[CK], rk[CK], rb[CK], rq[CK];
+  auto load_seg = [&](long long t0, int nt, bool bwd) {
     for (int e = i; e < CK * NJ; e += DK) {
       const int u = e / NJ, j = e % NJ;
-      float uu = 0.f, dd = 0.f;
+      float vv = 0.f, ww = 0.f, dd = 0.f, dl = 0.f;
       if (u < nt) {
-        uu = ld<T>(p.w, vcol(t0 + u, j)) * ld<T>(p.v, vcol(t0 + u, j));
-        if (with_do) dd = ld<T>(p.dO, vcol(t0 + u, j));
+        vv = ld<T>(p.v, vcol(t0 + u, j));
+        ww = ld<T>(p.w, vcol(t0 + u, j));
+        if (bwd) {
+          dd = ld<T>(p.dO, vcol(t0 + u, j));
+          dl = p.dl[vcol(t0 + u, j)];
+        }
       }
-      sm.u[u][j] = uu;
+      sm.u[u][j] = ww * vv;
+      sm.vv[u][j] = vv;
+      sm.ww[u][j] = ww;
       sm.dO[u][j] = dd;
+      sm.dl[u][j] = dl;
     }
-  };
-  // One forward token: s <- alpha s; d = u - s^T a; s += k d^T.  d is left in sm.dl[u].
-  auto forward = [&](int u, float al, float kk, float bb) {
-    float v[NJ];
-    const float ai = bb * kk;
 #pragma unroll
-    for (int j = 0; j < NJ; ++j) {
-      s[j] *= al;
-      v[j] = ai * s[j];
+    for (int u = 0; u < CK; ++u) {
+      const bool in = u < nt;
+      ral[u] = in ? ld<T>(p.alpha, krow(t0 + u)) : 0.f;
+      rk[u] = in ? ld<T>(p.k, krow(t0 + u)) : 0.f;
+      rb[u] = in ? ld<T>(p.b, krow(t0 + u)) : 0.f;
+      rq[u] = in && bwd ? ld<T>(p.q, krow(t0 + u)) : 0.f;
     }
-    reduce(v, [&](int j, float r) {
-      const float d = sm.u[u][j] - r;
-      sm.dl[u][j] = d;
-      return d;
-    });
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) s[j] = fmaf(kk, sm.bc[j], s[j]);
   };
 
-  // Pass 1: forward over the sequence, storing the state before every segment.
+  // Pass 1: forward over the sequence, storing the state before every segment and every d_t.
   for (int m = 0; m < nseg; ++m) {
     const long long t0 = bos + (long long)m * CK;
     const int nt = (int)min((long long)CK, len - (long long)m * CK);
     float4 *c = ck_at(m);
 #pragma unroll
     for (int q4 = 0; q4 < NJ / 4; ++q4) c[q4 * DK] = make_float4(s[4 * q4], s[4 * q4 + 1], s[4 * q4 + 2], s[4 * q4 + 3]);
-    load_cols(t0, nt, false);
-    for (int u = 0; u < nt; ++u)
-      forward(u, ld<T>(p.alpha, krow(t0 + u)), ld<T>(p.k, krow(t0 + u)), ld<T>(p.b, krow(t0 + u)));
+    load_seg(t0, nt, false);
+    __syncthreads();  // the segment's value-side inputs are in shared memory
+#pragma unroll
+    for (int u = 0; u < CK; ++u) {
+      if (u >= nt) break;
+      const float al = ral[u], kk = rk[u], ai = rb[u] * kk;
+      float v[NJ], r[NJ];
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        s[j] *= al;
+        v[j] = ai * s[j];
+      }
+      reduce(v, r);
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) s[j] = fmaf(kk, sm.u[u][j] - r[j], s[j]);
+      if (i < NJ) p.dl[vcol(t0 + u, i)] = sm.u[u][i] - r[i];  // same value as used above
+    }
+    __syncthreads();  // before the next segment overwrites the value-side inputs
   }
 
   // Pass 2: backwards, one segment at a time.
@@ -191,24 +224,18 @@ __global__ void __launch_bounds__(DK) chunk_bwd_kernel(const BwdParams p) {
       s[4 * q4 + 2] = x.z;
       s[4 * q4 + 3] = x.w;
     }
-    load_cols(t0, nt, true);
-    float ral[CK], rk[CK], rb[CK], rq[CK];
-#pragma unroll
-    for (int u = 0; u < CK; ++u) {
-      const bool in = u < nt;
-      ral[u] = in ? ld<T>(p.alpha, krow(t0 + u)) : 0.f;
-      rk[u] = in ? ld<T>(p.k, krow(t0 + u)) : 0.f;
-      rb[u] = in ? ld<T>(p.b, krow(t0 + u)) : 0.f;
-      rq[u] = in ? ld<T>(p.q, krow(t0 + u)) : 0.f;
-    }
-    // rebuild: the state before each token of the segment, and d_t
+    load_seg(t0, nt, true);
+    __syncthreads();
+    // rebuild the state before each token of the segment from the checkpoint and the stored d_t
+    // (the same operations as the first pass, so the same values)
 #pragma unroll
     for (int u = 0; u < CK; ++u) {
       if (u >= nt) break;
 #pragma unroll
       for (int q4 = 0; q4 < NJ / 4; ++q4)
         sm.seg[u][q4][i] = make_float4(s[4 * q4], s[4 * q4 + 1], s[4 * q4 + 2], s[4 * q4 + 3]);
-      forward(u, ral[u], rk[u], rb[u]);
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) s[j] = fmaf(rk[u], sm.dl[u][j], s[j] * ral[u]);
     }
     // backwards through the segment
 #pragma unroll
@@ -225,39 +252,36 @@ __global__ void __launch_bounds__(DK) chunk_bwd_kernel(const BwdParams p) {
         sp[4 * q4 + 2] = x.z;
         sp[4 * q4 + 3] = x.w;
       }
-      float dq = 0.f, dk = 0.f, v[NJ];
+      float dq = 0.f, dk = 0.f, v[NJ], dd[NJ];
 #pragma unroll
       for (int j = 0; j < NJ; ++j) {
         const float doj = sm.dO[u][j], dlj = sm.dl[u][j];
         g[j] = fmaf(qq, doj, g[j]);
-        const float st = fmaf(kk, dlj, al * sp[j]);  // S_t, as the forward formed it
+        const float st = fmaf(kk, dlj, sp[j] * al);  // S_t, as the forward formed it
         dq = fmaf(st, doj, dq);
         dk = fmaf(g[j], dlj, dk);
         v[j] = g[j] * kk;
       }
-      reduce(v, [&](int j, float dd) {
-        const size_t o = vcol(t, j);
-        const float vv = ld<T>(p.v, o), ww = ld<T>(p.w, o);
-        static_cast<T *>(p.dv)[o] = from_f32<T>(dd * ww);
-        static_cast<T *>(p.dw)[o] = from_f32<T>(dd * vv);
-        return dd;
-      });
+      reduce(v, dd);
+      if (i < NJ) {  // this thread's column: dv, dw (dd of column i, re-read from the partials)
+        const float ddi = red_sum(par ^ 1, i);
+        const size_t o = vcol(t, i);
+        static_cast<T *>(p.dv)[o] = from_f32<T>(ddi * sm.ww[u][i]);
+        static_cast<T *>(p.dw)[o] = from_f32<T>(ddi * sm.vv[u][i]);
+      }
       float da = 0.f, dal = 0.f;
 #pragma unroll
       for (int j = 0; j < NJ; ++j) {
-        const float dd = sm.bc[j], spj = al * sp[j];
-        da = fmaf(-spj, dd, da);
-        const float dsp = fmaf(-ai, dd, g[j]);
+        const float spj = sp[j] * al;
+        da = fmaf(-spj, dd[j], da);
+        const float dsp = fmaf(-ai, dd[j], g[j]);
         dal = fmaf(dsp, sp[j], dal);
         g[j] = al * dsp;
       }
       dk = fmaf(da, bb, dk);
-      float *acc = p.acc + ((size_t)t * H + h) * 4 * DK + i;
-      atomicAdd(acc, dq);
-      atomicAdd(acc + DK, dk);
-      atomicAdd(acc + 2 * DK, dal);
-      atomicAdd(acc + 3 * DK, da * kk);
+      red_add4(p.acc + ((size_t)t * H + h) * DK + i, dq, dk, dal, da * kk);
     }
+    __syncthreads();  // before the next segment overwrites the segment's inputs
   }
   if (p.dS0) {
     const size_t off = (((size_t)n * H + h) * DK + i) * DV + j0;
@@ -266,18 +290,15 @@ __global__ void __launch_bounds__(DK) chunk_bwd_kernel(const BwdParams p) {
   }
 }
 
-// acc [rows, 4, d_k] fp32 -> dq, dk, dalpha, db [rows, d_k] in the output type.
+// acc [rows, d_k] x (dq, dk, dalpha, db) fp32 -> the four gradients [rows, d_k] in the output type.
 template <typename T>
-__global__ void __launch_bounds__(256) bwd_finish_kernel(const float *acc, T *dq, T *dk, T *dal, T *db, size_t rows,
-                                                        int DK) {
-  const size_t n = rows * DK;
+__global__ void __launch_bounds__(256) bwd_finish_kernel(const float4 *acc, T *dq, T *dk, T *dal, T *db, size_t n) {
   for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
-    const size_t r = e / DK, c = e - r * DK;
-    const float *a = acc + r * 4 * DK + c;
-    dq[e] = from_f32<T>(a[0]);
-    dk[e] = from_f32<T>(a[DK]);
-    dal[e] = from_f32<T>(a[2 * DK]);
-    db[e] = from_f32<T>(a[3 * DK]);
+    const float4 a = acc[e];
+    dq[e] = from_f32<T>(a.x);
+    dk[e] = from_f32<T>(a.y);
+    dal[e] = from_f32<T>(a.z);
+    db[e] = from_f32<T>(a.w);
   }
 }
 
@@ -290,10 +311,13 @@ cudaError_t bwd_t(const BwdArgs &a, void *ws, cudaStream_t stream) {
   p.q = a.q; p.k = a.k; p.v = a.v; p.alpha = a.alpha; p.b = a.b; p.w = a.w; p.dO = a.dO;
   p.S0 = a.S0; p.dST = a.dST; p.dv = a.dv; p.dw = a.dw; p.dS0 = a.dS0; p.cu = a.cu;
   p.N = a.B; p.T = a.T; p.H = a.H; p.dv_ = a.Dv;
-  const size_t acc_bytes = align256((size_t)tokens * a.H * 4 * DK * sizeof(float));
-  p.acc = static_cast<float *>(ws);
-  p.ck = reinterpret_cast<float4 *>(static_cast<uint8_t *>(ws) + acc_bytes);
-  cudaError_t err = cudaMemsetAsync(p.acc, 0, (size_t)tokens * a.H * 4 * DK * sizeof(float), stream);
+  const size_t acc_elems = (size_t)tokens * a.H * DK;  // float4 each
+  uint8_t *base = static_cast<uint8_t *>(ws);
+  p.acc = reinterpret_cast<float4 *>(base);
+  p.dl = reinterpret_cast<float *>(base + align256(acc_elems * sizeof(float4)));
+  p.ck = reinterpret_cast<float4 *>(base + align256(acc_elems * sizeof(float4)) +
+                                    align256((size_t)tokens * a.H * a.Dv * sizeof(float)));
+  cudaError_t err = cudaMemsetAsync(p.acc, 0, acc_elems * sizeof(float4), stream);
   if (err != cudaSuccess) return err;
   const int smem = (int)sizeof(BwdSmem<T, DK>);
   err = cudaFuncSetAttribute(chunk_bwd_kernel<T, DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -302,11 +326,10 @@ cudaError_t bwd_t(const BwdArgs &a, void *ws, cudaStream_t stream) {
   chunk_bwd_kernel<T, DK><<<dim3(a.Dv / NJ, a.H, a.B), DK, smem, stream>>>(p);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   if (tokens == 0) return cudaSuccess;
-  const size_t rows = (size_t)tokens * a.H;
-  const unsigned blocks = (unsigned)std::min<size_t>((rows * DK + 255) / 256, (size_t)148 * 16);
+  const unsigned blocks = (unsigned)std::min<size_t>((acc_elems + 255) / 256, (size_t)148 * 16);
   note_launch();
   bwd_finish_kernel<T><<<blocks, 256, 0, stream>>>(p.acc, static_cast<T *>(a.dq), static_cast<T *>(a.dk),
-                                                  static_cast<T *>(a.dalpha), static_cast<T *>(a.db), rows, DK);
+                                                  static_cast<T *>(a.dalpha), static_cast<T *>(a.db), acc_elems);
   return cudaGetLastError();
 }
 
@@ -315,7 +338,8 @@ cudaError_t bwd_t(const BwdArgs &a, void *ws, cudaStream_t stream) {
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, bool packed) {
   const long long tokens = packed ? (long long)T : (long long)B * T;
   const long long slots = tokens / CK + B + 1;
-  return align256((size_t)tokens * H * 4 * dk * sizeof(float)) + (size_t)slots * H * dk * dv * sizeof(float);
+  return align256((size_t)tokens * H * dk * sizeof(float4)) + align256((size_t)tokens * H * dv * sizeof(float)) +
+         (size_t)slots * H * dk * dv * sizeof(float);
 }
 
 cudaError_t launch_chunk_bwd(const BwdArgs &a, bool bf16, void *ws, cudaStream_t stream) {
