@@ -126,3 +126,94 @@ def test_python_binding_has_no_cpu_path():
     x = torch.zeros(1, 64, 1, 64)
     with pytest.raises((ValueError, RuntimeError)):
         gdn2.chunk_fwd(x, x, x, x, x, x)
+
+
+def bwd(L, ptrs=None, B=1, T=64, H=1, dk=64, dv=64, cu=None, dtype=gdn2.GDN2_BF16):
+    p = ptrs or [FAKE] * 16
+    return L.gdn2_chunk_bwd(*p, B, T, H, dk, dv, cu, dtype, None)
+
+
+# argument order: q k v alpha b w S0 dO dS_T | dq dk dv dalpha db dw dS0
+BWD_REQUIRED = [0, 1, 2, 3, 4, 5, 7, 9, 10, 11, 12, 13, 14]
+BWD_OPTIONAL = [6, 8, 15]
+
+
+def test_bwd_validation(L):
+    before = L.gdn2_launch_count()
+    for i in BWD_REQUIRED:
+        p = [FAKE] * 16
+        p[i] = None
+        assert bwd(L, p) == gdn2.GDN2_ERR_INVALID_ARG, i
+        p[i] = MIS
+        assert bwd(L, p) == gdn2.GDN2_ERR_INVALID_ARG, i
+    for i in BWD_OPTIONAL:  # S0, dS_T and dS0 may be NULL, but not misaligned
+        p = [FAKE] * 16
+        p[i] = MIS
+        assert bwd(L, p) == gdn2.GDN2_ERR_INVALID_ARG, i
+    assert bwd(L, B=-1) == gdn2.GDN2_ERR_INVALID_ARG
+    assert bwd(L, T=-1) == gdn2.GDN2_ERR_INVALID_ARG
+    assert bwd(L, H=0) == gdn2.GDN2_ERR_INVALID_ARG
+    assert bwd(L, dtype=3) == gdn2.GDN2_ERR_INVALID_ARG
+    assert bwd(L, dk=96) == gdn2.GDN2_ERR_UNSUPPORTED
+    assert bwd(L, dv=32) == gdn2.GDN2_ERR_UNSUPPORTED
+    assert bwd(L, B=1 << 30, T=1 << 30, H=1 << 20) == gdn2.GDN2_ERR_INVALID_ARG
+    assert bwd(L, B=0) == gdn2.GDN2_OK
+    assert L.gdn2_launch_count() == before
+
+
+def test_bwd_workspace_bytes(L):
+    # the key-side accumulator, d_t, and checkpoints of every tile's state every 8 tokens
+    n = L.gdn2_chunk_bwd_workspace_bytes(4, 2048, 16, 128, 128, 0)
+    slots = 4 * 2048 // 8 + 4 + 1
+    assert n >= 4 * 2048 * 16 * 128 * 16 + 4 * 2048 * 16 * 128 * 4 + slots * 16 * 128 * 128 * 4
+    assert L.gdn2_chunk_bwd_workspace_bytes(4, 2048, 16, 96, 128, 0) == 0
+    assert L.gdn2_chunk_bwd_workspace_bytes(0, 2048, 16, 128, 128, 0) == 0
+
+
+def prologue(L, ptrs=None, B=1, T=64, H=1, dk=64, dv=64, K=4, cu=None, dtype=gdn2.GDN2_BF16):
+    p = ptrs or [FAKE] * 15
+    return L.gdn2_block_prologue(*p, B, T, H, dk, dv, K, cu, dtype, None)
+
+
+def test_block_prologue_validation(L):
+    before = L.gdn2_launch_count()
+    for i in range(15):
+        p = [FAKE] * 15
+        p[i] = None
+        assert prologue(L, p) == gdn2.GDN2_ERR_INVALID_ARG, i
+    for i in list(range(6)) + list(range(9, 15)):  # token tensors: 16-byte alignment
+        p = [FAKE] * 15
+        p[i] = MIS
+        assert prologue(L, p) == gdn2.GDN2_ERR_INVALID_ARG, i
+    for i in range(6, 9):  # convolution weights: 4-byte alignment is enough
+        p = [FAKE] * 15
+        p[i] = ctypes.c_void_p(0x10002)
+        assert prologue(L, p) == gdn2.GDN2_ERR_INVALID_ARG, i
+    assert prologue(L, K=0) == gdn2.GDN2_ERR_UNSUPPORTED
+    assert prologue(L, K=5) == gdn2.GDN2_ERR_UNSUPPORTED
+    assert prologue(L, dk=256) == gdn2.GDN2_ERR_UNSUPPORTED
+    assert prologue(L, H=0) == gdn2.GDN2_ERR_INVALID_ARG
+    assert prologue(L, dtype=9) == gdn2.GDN2_ERR_INVALID_ARG
+    assert prologue(L, B=0) == gdn2.GDN2_OK
+    assert L.gdn2_launch_count() == before
+
+
+def epilogue(L, ptrs=None, tokens=64, H=1, dv=64, dtype=gdn2.GDN2_BF16):
+    p = ptrs or [FAKE] * 4
+    return L.gdn2_block_epilogue(*p, tokens, H, dv, dtype, None)
+
+
+def test_block_epilogue_validation(L):
+    before = L.gdn2_launch_count()
+    for i in range(4):
+        p = [FAKE] * 4
+        p[i] = None
+        assert epilogue(L, p) == gdn2.GDN2_ERR_INVALID_ARG, i
+    for i in (0, 1, 3):
+        p = [FAKE] * 4
+        p[i] = MIS
+        assert epilogue(L, p) == gdn2.GDN2_ERR_INVALID_ARG, i
+    assert epilogue(L, tokens=-1) == gdn2.GDN2_ERR_INVALID_ARG
+    assert epilogue(L, dv=32) == gdn2.GDN2_ERR_UNSUPPORTED
+    assert epilogue(L, tokens=0) == gdn2.GDN2_OK
+    assert L.gdn2_launch_count() == before
