@@ -23,7 +23,9 @@ def _worker(rank, world, port, out_dir):
     import bench
     import gdn2_workloads as W
     import oracle
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    # loopback for the rendezvous and for gloo's own connections (the host name may not resolve)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      GLOO_SOCKET_IFNAME="lo")
     dist.init_process_group("gloo", rank=rank, world_size=world)
     wl = W.Workload("mr", B=2, T=70, H=2, dk=16, dv=8, dtype="f32")
     n_global = wl.B * world
