@@ -507,38 +507,64 @@ def bench_bwd(gdn2, dev, stream, pk, pk_kind, reps=5):
                          "note": "issue- and latency-bound SIMT kernel (about 655 instructions per warp and token)"}}
 
 
-def bench_e2e(gdn2, wl, d, dev, stream, ws, tokens, steps=3):
-    """chunk_fwd through the public call with pinned host buffers: H2D of the inputs and S0, the call,
-    D2H of o and S_T, all inside the timed region."""
+def bench_e2e(gdn2, wl, d, dev, stream, ws, tokens, steps=6):
+    """chunk_fwd through the public call with pinned host buffers.  Every step copies its inputs and
+    S0 host -> device, calls chunk_fwd and reads o and S_T back to the host, all inside the timed
+    region.  Steps are pipelined over two device buffer sets and three streams (copy in, the call,
+    copy out): one step's input copy overlaps the previous step's call and readback, as a serving
+    loop would run them.  A buffer set is refilled only after the call that read it has finished,
+    and its outputs are overwritten only after their readback."""
     host = {n: d[n].cpu().pin_memory() for n in TOK}
     host["S0"] = d["S0"].cpu().pin_memory()
-    dv_in = {n: torch.empty_like(d[n]) for n in list(TOK)}
-    dv_in["S0"] = torch.empty_like(d["S0"])
-    o_h = torch.empty(wl.B, wl.T, wl.H, wl.dv, dtype=torch.bfloat16).pin_memory()
-    S_h = torch.empty(wl.B, wl.H, wl.dk, wl.dv, dtype=torch.float32).pin_memory()
+    nbuf = 2
+    dev_in = [{n: torch.empty_like(d[n]) for n in host} for _ in range(nbuf)]
+    dev_out = [(torch.empty(wl.B, wl.T, wl.H, wl.dv, dtype=torch.bfloat16, device=dev),
+                torch.empty(wl.B, wl.H, wl.dk, wl.dv, dtype=torch.float32, device=dev)) for _ in range(nbuf)]
+    host_out = [(torch.empty(wl.B, wl.T, wl.H, wl.dv, dtype=torch.bfloat16).pin_memory(),
+                 torch.empty(wl.B, wl.H, wl.dk, wl.dv, dtype=torch.float32).pin_memory()) for _ in range(nbuf)]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = o_h.numel() * o_h.element_size() + S_h.numel() * S_h.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in host_out[0])
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def one():
-        for n, t in host.items():
-            dv_in[n].copy_(t, non_blocking=True)
-        o, ST = gdn2.chunk_fwd(*[dv_in[n] for n in TOK], S0=dv_in["S0"], stream=stream)
-        o_h.copy_(o, non_blocking=True)
-        S_h.copy_(ST, non_blocking=True)
+    def run(n):
+        ev_call = [torch.cuda.Event() for _ in range(n)]
+        ev_back = [torch.cuda.Event() for _ in range(n)]
+        for k in range(n):
+            b = k % nbuf
+            if k >= nbuf:
+                s_in.wait_event(ev_call[k - nbuf])  # the call that read this buffer set is done
+            with torch.cuda.stream(s_in):
+                for name, t in host.items():
+                    dev_in[b][name].copy_(t, non_blocking=True)
+            ev_copied = torch.cuda.Event()
+            ev_copied.record(s_in)
+            stream.wait_event(ev_copied)
+            if k >= nbuf:
+                stream.wait_event(ev_back[k - nbuf])  # this buffer set's outputs were read back
+            gdn2.chunk_fwd(*[dev_in[b][name] for name in TOK], S0=dev_in[b]["S0"], o=dev_out[b][0],
+                           S_T=dev_out[b][1], stream=stream)
+            ev_call[k].record(stream)
+            s_out.wait_event(ev_call[k])
+            with torch.cuda.stream(s_out):
+                host_out[b][0].copy_(dev_out[b][0], non_blocking=True)
+                host_out[b][1].copy_(dev_out[b][1], non_blocking=True)
+            ev_back[k].record(s_out)
+        return ev_back[-1]
 
-    one()
+    run(2)
     torch.cuda.synchronize(dev)
     barrier(ws)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        one()
-    b.record(stream)
+    a.record(s_in)
+    last = run(steps)
+    s_out.wait_event(last)
+    b.record(s_out)
     torch.cuda.synchronize(dev)
     barrier(ws)
     ms = max_over_ranks(a.elapsed_time(b), ws, dev)
     return {"value": ws * tokens * steps / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": steps}
+            "d2h_bytes_per_step": d2h, "steps": steps,
+            "pipelined": "two device buffer sets; copy-in, call and copy-out streams overlap across steps"}
 
 
 if __name__ == "__main__":
