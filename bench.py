@@ -357,8 +357,8 @@ def profile_case(which):
             gdn2.chunk_fwd(*[d[n] for n in TOK], S0=d["S0"])
     elif which in ("bwd", "bwd_small"):
         wl = W.WORKLOADS["layer_1p3b"]
-        if which == "bwd_small":  # one sequence of 512 tokens: 128 CTAs, a few hundred MB on the device
-            wl = W.Workload("bwd_small", B=1, T=512, H=16, dk=128, dv=128)
+        if which == "bwd_small":  # 4 x 512 tokens: the layer's 512 CTAs and occupancy, about 0.4 GB on the device
+            wl = W.Workload("bwd_small", B=4, T=512, H=16, dk=128, dv=128)
         d = W.chunk_inputs(wl, device=dev, seed=0)
         gen = torch.Generator(device="cpu").manual_seed(1000)
         dO = torch.randn(d["q"].shape[:-1] + (wl.dv,), generator=gen).to(dev, torch.bfloat16)
