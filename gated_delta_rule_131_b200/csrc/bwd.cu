@@ -30,7 +30,7 @@ namespace gdn2 {
 namespace {
 
 constexpr int NJ = 16;  // value columns per CTA
-constexpr int CK = 8;   // tokens per checkpoint segment
+constexpr int CK = 4;   // tokens per checkpoint segment (4 CTAs of 128 rows fit an SM)
 
 struct BwdParams {
   const void *q, *k, *v, *alpha, *b, *w, *dO;
@@ -96,9 +96,9 @@ struct __align__(16) BwdSmem {
   float red[2][NJ][NW];        // warp partials of a block reduction, double-buffered
 };
 
-// One (sequence, head, NJ-column tile).  blockDim = DK; three blocks of 128 rows per SM.
+// One (sequence, head, NJ-column tile).  blockDim = DK; four blocks of 128 rows per SM.
 template <typename T, int DK>
-__global__ void __launch_bounds__(DK, 384 / DK) chunk_bwd_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(DK, 512 / DK) chunk_bwd_kernel(const BwdParams p) {
   using Smem = BwdSmem<T, DK>;
   constexpr int NW = Smem::NW;
   extern __shared__ __align__(16) uint8_t dsm[];

@@ -158,7 +158,7 @@ GDN2_API size_t gdn2_chunk_fwd_workspace_bytes(int B, int T, int H, int d_k, int
  *   dS0     [B, H, d_k, d_v] fp32 (out), or NULL (not returned).  dS0 may alias dS_T.
  * Arithmetic is fp32; the gradients are rounded to dtype once.  The call takes a workspace of
  * gdn2_chunk_bwd_workspace_bytes() bytes from the library's pool (a gradient accumulator and
- * state checkpoints every 8 tokens) and gives it back on `stream`.  Errors as for gdn2_chunk_fwd.
+ * state checkpoints every 4 tokens) and gives it back on `stream`.  Errors as for gdn2_chunk_fwd.
  */
 GDN2_API gdn2_status gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *alpha,
                                     const void *b, const void *w, const float *S0, const void *dO,

@@ -162,9 +162,9 @@ def test_bwd_validation(L):
 
 
 def test_bwd_workspace_bytes(L):
-    # the key-side accumulator, d_t, and checkpoints of every tile's state every 8 tokens
+    # the key-side accumulator, d_t, and checkpoints of every tile's state every 4 tokens
     n = L.gdn2_chunk_bwd_workspace_bytes(4, 2048, 16, 128, 128, 0)
-    slots = 4 * 2048 // 8 + 4 + 1
+    slots = 4 * 2048 // 4 + 4 + 1
     assert n >= 4 * 2048 * 16 * 128 * 16 + 4 * 2048 * 16 * 128 * 4 + slots * 16 * 128 * 128 * 4
     assert L.gdn2_chunk_bwd_workspace_bytes(4, 2048, 16, 96, 128, 0) == 0
     assert L.gdn2_chunk_bwd_workspace_bytes(0, 2048, 16, 128, 128, 0) == 0
