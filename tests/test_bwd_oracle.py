@@ -3,11 +3,13 @@
 The gradient in ``oracle/bwd_oracle.c`` is derived by hand from the recurrence of
 "[논문] 게이트형 DeltaNet-2" (euno.news), section "방법론", and
 "NVIDIA AIがGated DeltaNet-2を発表" (ai.warp-studio.com), section "Gated DeltaNet-2の核心".
-It is pinned against two things that do not share its derivation:
+It is pinned against three things that do not share its derivation:
 
 * central finite differences of the forward oracle, element by element, on tiny
   dense and packed problems (every term of the chain rule moves some element);
-* torch autograd through a token loop written here from the same definition.
+* torch autograd through a token loop written here from the same definition;
+* closed forms at alpha = 1, b = 0 (plain linear attention), where every gradient
+  is a sum over later tokens rather than a reverse recurrence.
 """
 import numpy as np
 import pytest
@@ -118,3 +120,32 @@ def test_linearity_in_the_upstream_gradients():
     only_s = _grads(x, cu)
     for name in NAMES:
         np.testing.assert_allclose(both[name], only_o[name] + only_s[name], rtol=1e-12, atol=1e-13)
+
+
+def test_linear_attention_closed_forms():
+    """alpha = 1, b = 0: S_t = S0 + sum_{s<=t} k_s u_s^T (u = w (.) v) and o_t = S_t^T q_t.  Every
+    gradient is then a sum over later tokens, written here without the reverse recurrence:
+      dq_t = S_t dO_t,   G_s = sum_{t>=s} q_t dO_t^T + dST,   du_s = G_s^T k_s,
+      dk_s = G_s u_s,    dS0 = G_1,   dalpha_s[i] = sum_j G_s[i, j] S_{s-1}[i, j],
+      db_s = -k_s (.) (S_{s-1} (G_s^T k_s))   (the erase probe's derivative at b = 0)."""
+    N, T, H, dk, dv = 1, 9, 1, 4, 3
+    x, cu = _problem(N, T, H, dk, dv)
+    x["alpha"][:] = 1.0
+    x["b"][:] = 0.0
+    g = _grads(x, cu)
+    q, k, v, w, dO = (x[n][0, :, 0] for n in ("q", "k", "v", "w", "dO"))
+    S0, dST = x["S0"][0, 0], x["dST"][0, 0]
+    u = w * v
+    S = [S0]
+    for t in range(T):
+        S.append(S[-1] + np.outer(k[t], u[t]))
+    G = [sum((np.outer(q[t], dO[t]) for t in range(s, T)), np.zeros((dk, dv))) + dST for s in range(T)]
+    for s in range(T):
+        np.testing.assert_allclose(g["q"][0, s, 0], S[s + 1] @ dO[s], rtol=1e-12, atol=1e-12)
+        du = G[s].T @ k[s]
+        np.testing.assert_allclose(g["v"][0, s, 0], du * w[s], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(g["w"][0, s, 0], du * v[s], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(g["k"][0, s, 0], G[s] @ u[s], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(g["alpha"][0, s, 0], (G[s] * S[s]).sum(1), rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(g["b"][0, s, 0], -k[s] * (S[s] @ du), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(g["S0"][0, 0], G[0], rtol=1e-12, atol=1e-12)
