@@ -156,7 +156,9 @@ GDN2_API size_t gdn2_chunk_fwd_workspace_bytes(int B, int T, int H, int d_k, int
  *   dS_T    [B, H, d_k, d_v] fp32: dL/dS_T, or NULL (zero).
  *   dq, dk, dalpha, db   [.., H, d_k] in dtype (out), dv, dw [.., H, d_v] in dtype (out).
  *   dS0     [B, H, d_k, d_v] fp32 (out), or NULL (not returned).  dS0 may alias dS_T.
- * Arithmetic is fp32; the gradients are rounded to dtype once.  The call takes a workspace of
+ * Arithmetic is fp32; the gradients are rounded to dtype once.  dq, dk, dalpha and db are sums
+ * over 16-column tiles of the state formed with fp32 reductions in L2, so their last bits may
+ * differ from run to run; dv, dw and dS0 are reproducible.  The call takes a workspace of
  * gdn2_chunk_bwd_workspace_bytes() bytes from the library's pool (a gradient accumulator and
  * state checkpoints every 4 tokens) and gives it back on `stream`.  Errors as for gdn2_chunk_fwd.
  */
