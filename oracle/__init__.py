@@ -30,6 +30,8 @@ Functions and the passages they follow:
 * :func:`recurrent_bwd` -- the reverse-mode gradient of :func:`recurrent`
   (erase reading R1) with respect to q, k, v, alpha, b, w and S0, taken step by
   step backwards through the same token loop; the code is in ``bwd_oracle.c``.
+* :func:`chunkwise_bwd` -- the same gradient taken through the chunkwise WY form
+  (a companion, in numpy, ``chunk_bwd.py``); pinned against :func:`recurrent_bwd`.
 """
 import ctypes
 import os
@@ -37,6 +39,7 @@ import os
 import numpy as np
 
 from . import build as _build
+from .chunk_bwd import chunkwise_bwd  # noqa: F401
 
 ERASE_R1 = 0  # S_t = (I - k (b*k)^T) Diag(alpha) S + k (w*v)^T   (adopted reading)
 ERASE_R2 = 1  # S_t = (I - (b*k) k^T) Diag(alpha) S + k (w*v)^T
