@@ -424,11 +424,12 @@ def bench_decode(gdn2, dev, stream, pk, pk_kind):
             "launches": per_replay * reps}
 
 
-def block_bytes(wl, tokens):
+def block_bytes(wl, tokens, conv_len=4):
     """Algorithmic bytes of the block prologue and epilogue (every element read and written once)."""
     e = 2 if wl.dtype == "bf16" else 4
     th = tokens * wl.H
-    pro = th * 2 * (4 * wl.dk + 2 * wl.dv) * e + 3 * 4 * wl.H * (2 * wl.dk + wl.dv) * 4  # + conv weights
+    # six pre-activations in, six outputs out; plus the fp32 taps of the three paths, [H*d, K] each
+    pro = th * 2 * (4 * wl.dk + 2 * wl.dv) * e + conv_len * wl.H * (2 * wl.dk + wl.dv) * 4
     epi = th * 3 * wl.dv * e + wl.dv * 4
     return pro, epi
 
