@@ -563,7 +563,7 @@ __global__ void __launch_bounds__(wy::NT, 2)
   fence_proxy_async();
   __syncthreads();
 
-  // ------------------------------------------------------------ round 1: [T; P] [A_m | T] and K_m^T T
+  // ------------------------------------------------------------ product pass 1: [T; P] [A_m | T] and K_m^T T
   // TMEM cols 0..127: rows 0..63 T A_m; cols 128..191: rows 64..127 P T; cols 192..255: K_m^T T
   if (tid == 0) {
     tc_fence_after();
@@ -618,14 +618,14 @@ __global__ void __launch_bounds__(wy::NT, 2)
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
-  if (tid == 0) {  // Nt, Pt and e^{g_C} are final: store them while round 2 runs
+  if (tid == 0) {  // Nt, Pt and e^{g_C} are final: store them while product pass 2 runs
     tma_store_2d(&tm_wn, 0, rec * 128, sb + OFF_TP);
     tma_store_2d(&tm_wp, 0, rec * 64, sb + OFF_TS);
     bulk_store(p.g + (size_t)rec * 128, sb + OFF_SC + 256 * 4, REC_G);
     bulk_commit();
   }
 
-  // ------------------------------------------------------------ round 2: K_m^T W and [Pt; *] A_m
+  // ------------------------------------------------------------ product pass 2: K_m^T W and [Pt; *] A_m
   // TMEM cols 0..127: K_m^T W; cols 128..255: rows 0..63 Pt A_m (rows 64..127 read whatever follows Pt)
   if (tid == 0) {
     tc_fence_after();
