@@ -93,7 +93,7 @@ class ClockSampler:
         0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, device_index, period_s=0.001):
+    def __init__(self, device_index, period_s=0.0002):
         self.samples, self.period, self._stop = [], period_s, threading.Event()
         self.ok = False
         self.max_mhz = None
@@ -236,6 +236,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-block", action="store_true", help="skip the block prologue/epilogue measurement")
     ap.add_argument("--no-bwd", action="store_true", help="skip the backward measurement")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the long-context, sequence-length sweep and packed-varlen measurements")
     ap.add_argument("--profile-case", choices=["chunk", "decode", "block", "bwd", "bwd_small"],
                     help="run one warm-up and one measured launch of that kernel on its full workload, for ncu")
     args = ap.parse_args()
@@ -328,6 +330,11 @@ def main():
         line.update(bench_block(gdn2, dev, stream, pk, pk_kind))
     if not args.no_bwd:
         line["chunk_bwd"] = bench_bwd(gdn2, dev, stream, pk, pk_kind)
+    if not args.no_workloads:
+        line["long_context"] = bench_long_context(gdn2, dev, stream, pk, pk_kind)
+        line["varlen"] = bench_varlen(gdn2, dev, stream, pk, pk_kind)
+    # ------------------------------------------------------------ the headline step, sustained for ~0.5 s
+    line["sustained"] = bench_sustained(step, dev, stream, local, len(ev))
 
     # ------------------------------------------------------------ end to end through host buffers
     line["e2e"] = bench_e2e(gdn2, wl, sets[0], dev, stream, ws, tokens)
@@ -506,6 +513,97 @@ def bench_bwd(gdn2, dev, stream, pk, pk_kind, reps=5):
                          "frac": gbs / pk["hbm_gbs"], "traffic": tr["dram_bytes_per_launch"] if tr else None,
                          "peak_source": pk_kind, "algorithmic_bytes_per_launch": nbytes,
                          "note": "issue- and latency-bound SIMT kernel (about 655 instructions per warp and token)"}}
+
+
+def time_calls(fn, dev, stream, reps):
+    """Median CUDA-event time (ms) of ``reps`` calls of ``fn`` on ``stream``, after three warm-up calls."""
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in ev:
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    return statistics.median(a.elapsed_time(b) for a, b in ev)
+
+
+def chunk_entry(gdn2, wl, d, dev, stream, pk, pk_kind, reps):
+    """tokens/s and HBM roofline of one chunk_fwd call on the inputs ``d`` of workload ``wl``."""
+    lens = d["lengths"]
+    tokens = sum(lens)
+    fn = lambda: gdn2.chunk_fwd(*[d[n] for n in TOK], S0=d["S0"], cu_seqlens=d["cu_seqlens"], stream=stream)
+    c0 = gdn2.launch_count()
+    ms = time_calls(fn, dev, stream, reps)
+    launches = (gdn2.launch_count() - c0) // (reps + 3)
+    nbytes = chunk_bytes(wl, tokens, len(lens))
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"value": tokens / (ms / 1e3), "unit": "tokens/s", "workload": wl.name, "tokens": tokens,
+            "B": len(lens), "H": wl.H, "d_k": wl.dk, "d_v": wl.dv, "us_per_call": ms * 1e3,
+            "launches_per_call": launches,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "traffic": None, "peak_source": pk_kind,
+                         "algorithmic_bytes_per_launch": nbytes}}
+
+
+def bench_long_context(gdn2, dev, stream, pk, pk_kind):
+    """The long-context workload (B=1, H=16, T=65536, retention-biased decay), and the pages' claim of
+    near-flat throughput as sequences grow: tokens/s at a fixed 131,072 tokens x 16 heads per call,
+    split into sequences of 2048 ... 65536 tokens.  ``flat_scaling`` = tokens/s at T = 65536 over
+    tokens/s at T = 2048 (1.0 is perfectly flat)."""
+    wl = W.WORKLOADS["long_context"]
+    d = W.chunk_inputs(wl, device=dev, seed=0)
+    out = chunk_entry(gdn2, wl, d, dev, stream, pk, pk_kind, reps=10)
+    del d
+    sweep = []
+    total = 131072
+    for T in (2048, 8192, 32768, 65536):
+        wls = W.scaled(W.WORKLOADS["layer_1p3b"], name=f"seq_{T}", B=total // T, T=T)
+        ds = W.chunk_inputs(wls, device=dev, seed=0)
+        e = chunk_entry(gdn2, wls, ds, dev, stream, pk, pk_kind, reps=10)
+        sweep.append({"B": wls.B, "T": T, "tokens_per_s": e["value"], "us_per_call": e["us_per_call"],
+                      "roofline_frac": e["roofline"]["frac"]})
+        del ds
+    out["seq_sweep"] = sweep
+    out["flat_scaling"] = sweep[-1]["tokens_per_s"] / sweep[0]["tokens_per_s"]
+    out["flat_scaling_note"] = ("tokens/s at 2 x 65536 tokens over 64 x 2048 tokens, 16 heads, d = 128, bf16; "
+                                "same 131,072 tokens per call")
+    return out
+
+
+def bench_varlen(gdn2, dev, stream, pk, pk_kind):
+    """The packed workload (32 sequences, lengths uniform in [1, 8192], H=32, d_v=256) with its three
+    gate variants: per-channel b and w, the KDA case and the Gated DeltaNet case."""
+    out = {}
+    for name in ("varlen", "varlen_kda", "varlen_gdn"):
+        wl = W.WORKLOADS[name]
+        d = W.chunk_inputs(wl, device=dev, seed=0)
+        out[wl.variant] = chunk_entry(gdn2, wl, d, dev, stream, pk, pk_kind, reps=5)
+        del d
+    return out
+
+
+def bench_sustained(step, dev, stream, device_index, first, seconds=0.5):
+    """The headline step repeated back to back for about ``seconds`` (after the timed steps), with its
+    own clock samples: the clocks the step runs at under sustained load."""
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    step(first)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    n = max(10, int(seconds / max(a.elapsed_time(b) / 1e3, 1e-6)))
+    clocks = ClockSampler(device_index).start()
+    t0 = time.perf_counter()
+    a.record(stream)
+    for i in range(n):
+        step(first + i)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    t1 = time.perf_counter()
+    clocks.stop()
+    ms = a.elapsed_time(b)
+    return {"steps": n, "ms_per_step": ms / n, "seconds": ms / 1e3, "clocks": clocks.summary(t0, t1)}
 
 
 def bench_e2e(gdn2, wl, d, dev, stream, ws, tokens, steps=6):

@@ -101,8 +101,8 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
-    s = torch.cuda.current_stream() if stream is None else stream
+def _stream(stream, device=None):
+    s = torch.cuda.current_stream(device) if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
 
 
@@ -140,8 +140,9 @@ def _chunk(entry, q, k, v, alpha, b, w, S0, cu_seqlens, chunk, o, S_T, output_fi
         raise ValueError("gdn2: S0 must be float32")
     _check_tensors(q, k, v, alpha, b, w, S0, o, S_T, cu_seqlens)
     fn = getattr(lib(), entry)
-    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o), _ptr(S_T),
-            B, T, H, dk, dv, chunk, _ptr(cu_seqlens), _DTYPES[q.dtype], _stream(stream))
+    with torch.cuda.device(q.device):  # the library's pool and fixed workspace follow the current device
+        st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o), _ptr(S_T),
+                B, T, H, dk, dv, chunk, _ptr(cu_seqlens), _DTYPES[q.dtype], _stream(stream, q.device))
     if st != GDN2_OK:
         raise Gdn2Error(st, entry)
     return o, S_T
@@ -163,9 +164,11 @@ def chunk_fwd_noalloc(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, chunk=64, 
                       output_final_state=True, stream=None):
     """``chunk_fwd`` through the library's fixed workspace: the library allocates nothing.
 
-    Shapes whose workspace exceeds ``NOALLOC_WORKSPACE_BYTES`` raise ``Gdn2Error``
-    (``GDN2_ERR_UNSUPPORTED``).  Calls that overlap in time on one device race on the shared
-    workspace; calls on one stream are ordered.
+    For callers that cannot let the library allocate device memory (all memory reserved up front,
+    or owned by the caller's own memory manager).  The first call on a device looks the fixed
+    array's address up; make it before any stream capture.  Shapes whose workspace exceeds
+    ``NOALLOC_WORKSPACE_BYTES`` raise ``Gdn2Error`` (``GDN2_ERR_UNSUPPORTED``).  Calls that overlap
+    in time on one device race on the shared workspace; calls on one stream are ordered.
     """
     return _chunk("gdn2_chunk_fwd_noalloc", q, k, v, alpha, b, w, S0, cu_seqlens, chunk, o, S_T,
                   output_final_state, stream)
@@ -195,9 +198,10 @@ def chunk_bwd(q, k, v, alpha, b, w, dO, S0=None, dS_T=None, cu_seqlens=None, wan
     grads = [torch.empty_like(x) for x in (q, k, v, alpha, b, w)]
     dS0 = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device) if want_dS0 else None
     _check_tensors(q, k, v, alpha, b, w, dO, S0, dS_T, *grads, dS0, cu_seqlens)
-    st = lib().gdn2_chunk_bwd(*[_ptr(x) for x in (q, k, v, alpha, b, w, S0, dO, dS_T)],
-                              *[_ptr(x) for x in grads], _ptr(dS0), B, T, H, dk, dv, _ptr(cu_seqlens),
-                              _DTYPES[q.dtype], _stream(stream))
+    with torch.cuda.device(q.device):
+        st = lib().gdn2_chunk_bwd(*[_ptr(x) for x in (q, k, v, alpha, b, w, S0, dO, dS_T)],
+                                  *[_ptr(x) for x in grads], _ptr(dS0), B, T, H, dk, dv, _ptr(cu_seqlens),
+                                  _DTYPES[q.dtype], _stream(stream, q.device))
     if st != GDN2_OK:
         raise Gdn2Error(st, "gdn2_chunk_bwd")
     dq, dk_, dv_, dalpha, db, dw = grads
@@ -229,9 +233,10 @@ def block_prologue(xq, xk, xv, xa, xb, xw, conv_q, conv_k, conv_v, cu_seqlens=No
         raise ValueError("gdn2: convolution weights must be float32")
     outs = [torch.empty_like(x) for x in (xq, xk, xv, xa, xb, xw)]
     _check_tensors(xq, xk, xv, xa, xb, xw, conv_q, conv_k, conv_v, *outs, cu_seqlens)
-    st = lib().gdn2_block_prologue(*[_ptr(x) for x in (xq, xk, xv, xa, xb, xw, conv_q, conv_k, conv_v)],
-                                   *[_ptr(x) for x in outs], B, T, H, dk, dv, conv_q.shape[1],
-                                   _ptr(cu_seqlens), _DTYPES[xq.dtype], _stream(stream))
+    with torch.cuda.device(xq.device):
+        st = lib().gdn2_block_prologue(*[_ptr(x) for x in (xq, xk, xv, xa, xb, xw, conv_q, conv_k, conv_v)],
+                                       *[_ptr(x) for x in outs], B, T, H, dk, dv, conv_q.shape[1],
+                                       _ptr(cu_seqlens), _DTYPES[xq.dtype], _stream(stream, xq.device))
     if st != GDN2_OK:
         raise Gdn2Error(st, "gdn2_block_prologue")
     return tuple(outs)
@@ -248,8 +253,9 @@ def block_epilogue(o, gate, norm_weight, y=None, stream=None):
     if y is None:
         y = torch.empty_like(o)
     _check_tensors(o, gate, norm_weight, y)
-    st = lib().gdn2_block_epilogue(_ptr(o), _ptr(gate), _ptr(norm_weight), _ptr(y), tokens, H, dv,
-                                   _DTYPES[o.dtype], _stream(stream))
+    with torch.cuda.device(o.device):
+        st = lib().gdn2_block_epilogue(_ptr(o), _ptr(gate), _ptr(norm_weight), _ptr(y), tokens, H, dv,
+                                       _DTYPES[o.dtype], _stream(stream, o.device))
     if st != GDN2_OK:
         raise Gdn2Error(st, "gdn2_block_epilogue")
     return y
@@ -266,8 +272,9 @@ def decode_step(q, k, v, alpha, b, w, S, o=None, stream=None):
     if o is None:
         o = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
     _check_tensors(q, k, v, alpha, b, w, S, o)
-    st = lib().gdn2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S),
-                                _ptr(o), B, H, dk, dv, _DTYPES[q.dtype], _stream(stream))
+    with torch.cuda.device(q.device):
+        st = lib().gdn2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S),
+                                    _ptr(o), B, H, dk, dv, _DTYPES[q.dtype], _stream(stream, q.device))
     if st != GDN2_OK:
         raise Gdn2Error(st, "gdn2_decode_step")
     return o

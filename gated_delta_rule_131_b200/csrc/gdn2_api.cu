@@ -198,7 +198,8 @@ gdn2_status gdn2_chunk_fwd_noalloc(const void *q, const void *k, const void *v, 
     const cudaError_t err = gdn2::launch_chunk_simt(a, dtype == GDN2_BF16, (cudaStream_t)stream);
     return err == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
   }
-  // checked on the host before any CUDA call: the shape must fit the fixed workspace
+  // checked on the host before any launch or allocation: the shape must fit the fixed workspace (its size
+  // depends on the current device's SM count, which chunk_wy_workspace_bytes queries)
   if (gdn2::chunk_wy_workspace_bytes(B, T, H, d_v, cu_seqlens != nullptr) > kNoallocBytes) return GDN2_ERR_UNSUPPORTED;
   // nothing in the workspace has to start at zero: the chunk offsets and every record are written
   // by this call's kernels before they are read

@@ -65,7 +65,7 @@ typedef enum {
   GDN2_ERR_INVALID_ARG = 1, /* null / misaligned pointer, negative or overflowing size */
   GDN2_ERR_UNSUPPORTED = 2, /* valid but not implemented: head size, chunk size, dtype */
   GDN2_ERR_CUDA = 3,        /* a CUDA launch or attribute call failed                 */
-  GDN2_ERR_TIMEOUT = 4      /* reserved: a bounded device-side wait gave up            */
+  GDN2_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up (see gdn2_device_status) */
 } gdn2_status;
 
 typedef enum { GDN2_F32 = 0, GDN2_BF16 = 1 } gdn2_dtype;
@@ -111,15 +111,25 @@ GDN2_API gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v,
 /*
  * gdn2_chunk_fwd_noalloc -- gdn2_chunk_fwd without any device allocation.
  *
- * Same arguments, layouts, results and validation as gdn2_chunk_fwd.  It has no counterpart in the
- * pages: it exists for callers that must not allocate (CUDA-graph capture without memory nodes,
- * allocation-free serving loops).  Instead of the pooled workspace it uses one fixed device array of
- * GDN2_NOALLOC_WORKSPACE_BYTES bytes compiled into the library (its address is looked up once per
- * device, with that device current).  A tensor-core call (bf16, d_k = 128) whose workspace,
- * gdn2_chunk_fwd_workspace_bytes(), exceeds that size returns GDN2_ERR_UNSUPPORTED before any CUDA
- * call; calls that run the SIMT kernel need no workspace and are not limited.  The array is shared:
- * calls that overlap in time on one device (different streams, or different host threads) race on
- * it and must not be issued; calls on one stream are ordered and safe.
+ * It has no counterpart in the pages.  Same arguments, layouts, results and validation as
+ * gdn2_chunk_fwd.  It serves callers that cannot call cudaMalloc or a stream-ordered allocator
+ * once they run: a serving process that reserves all of its device memory at start-up and must not
+ * grow it, or a host program that embeds this library under a memory manager of its own that owns
+ * every allocation on the device.  Instead of the pooled workspace it uses one fixed device array
+ * of GDN2_NOALLOC_WORKSPACE_BYTES bytes compiled into the library; every GPU that loads the library
+ * holds that array until the process exits.
+ *   - Set-up: the first call on a device, with that device current, looks the array's device
+ *     address up (cudaGetSymbolAddress) and keeps it; make that first call before any stream
+ *     capture.  Later calls on the device reuse the address.
+ *   - Limit: a tensor-core call (bf16, d_k = 128) whose workspace, gdn2_chunk_fwd_workspace_bytes()
+ *     for this shape on the current device, exceeds the array returns GDN2_ERR_UNSUPPORTED before
+ *     any launch or allocation.  That size depends on the device's SM count (the number of segments
+ *     of the two-level state scan), so a shape near the limit may fit on one device and not on
+ *     another.  Calls that run the SIMT kernel need no workspace and are not limited.
+ *   - Sharing: every call uses the same array, which keeps what the previous call left in it; the
+ *     kernels write every word they read first, so nothing from an earlier call leaks into a
+ *     result.  Calls that overlap in time on one device (different streams, or different host
+ *     threads) race on the array and must not be issued; calls on one stream are ordered and safe.
  */
 #define GDN2_NOALLOC_WORKSPACE_BYTES (64u << 20) /* 64 MiB */
 GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *alpha,

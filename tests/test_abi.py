@@ -1,7 +1,7 @@
 """The C-ABI library loads and exports every symbol its headers declare (CPU only).
 
 No compute call is made here: only argument combinations that the library
-rejects on the host, before any CUDA call, are passed.
+rejects on the host, before any launch or allocation, are passed.
 """
 import ctypes
 import glob

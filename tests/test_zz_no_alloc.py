@@ -1,4 +1,11 @@
-"""gdn2_chunk_fwd_noalloc: the chunk forward through the library's fixed device workspace.
+"""gdn2_chunk_fwd_noalloc: the chunk forward for callers that cannot allocate device memory.
+
+Some callers reserve all of their device memory up front, or run this library under a memory
+manager of their own, and so cannot let it call cudaMalloc or a stream-ordered allocator.  This
+entry point runs the same kernels over one fixed device array compiled into the library.  The
+tests check, through the C ABI, that it gives bit for bit the output of gdn2_chunk_fwd on two calls
+in a row, for a dense batch, a packed batch and a long sequence that takes the two-level state
+scan (whose segment maps and entry states then also live in the fixed array).
 
 Collected last on purpose: it must pass alone and after every other test (the fixed workspace
 then still holds whatever earlier calls left in it, which must not matter).
@@ -24,7 +31,7 @@ def test_limit_matches_header():
     assert m and int(m.group(1)) << int(m.group(2)) == gdn2.NOALLOC_WORKSPACE_BYTES
 
 
-def test_oversized_shape_is_rejected_before_any_cuda_call():
+def test_oversized_shape_is_rejected_before_any_launch_or_allocation():
     gbuild.build()
     L = gdn2.lib()
     fake = ctypes.c_void_p(0x10000)  # never dereferenced: the size check comes first
@@ -66,3 +73,16 @@ def test_noalloc_matches_pooled_entry_packed(g):
     assert g.chunk_fwd_workspace_bytes(len(lengths), sum(lengths), wl.H, wl.dk, wl.dv,
                                        packed=True) <= g.NOALLOC_WORKSPACE_BYTES
     _both_entries_twice(g, wl, (33, 34), lengths=lengths)
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_pooled_entry_two_level_scan(g):
+    """One long sequence and one head: the state walk is cut into segments (two-level scan)."""
+    wl = W.Workload("noalloc_scan", B=1, T=4096, H=1, dk=128, dv=128)
+    dense = g.chunk_fwd_workspace_bytes(wl.B, wl.T, wl.H, wl.dk, wl.dv)
+    packed = g.chunk_fwd_workspace_bytes(wl.B, wl.T, wl.H, wl.dk, wl.dv, packed=True)
+    # the same chunk records either way; only a dense batch can take the scan, whose segment maps
+    # and entry states (about 0.6 MB here) make its workspace the larger one
+    assert dense > packed + 500_000
+    assert dense <= g.NOALLOC_WORKSPACE_BYTES
+    _both_entries_twice(g, wl, (35, 36))
