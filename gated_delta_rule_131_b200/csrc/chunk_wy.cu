@@ -81,7 +81,12 @@ __device__ __forceinline__ void unpack8(uint4 u, float *e) {
   t = bf2_to_f2(u.z); e[4] = t.x; e[5] = t.y;
   t = bf2_to_f2(u.w); e[6] = t.x; e[7] = t.y;
 }
-__device__ __forceinline__ float fast_rcp(float x) { return __fdividef(1.f, x); }
+// Approximate reciprocal (the hardware's single-instruction estimate; relative error about 2^-23).
+__device__ __forceinline__ float fast_rcp(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
 // Two fp32 products at once (sm_100 packed fp32 pipe; each lane rounds exactly like a scalar product).
 __device__ __forceinline__ void mul2(float *d, const float *a, const float *b) {
   const float2 r = __fmul2_rn(make_float2(a[0], a[1]), make_float2(b[0], b[1]));
@@ -232,33 +237,33 @@ static_assert(OFF_AL % 1024 == 0 && OFF_TS % 1024 == 0, "MMA operand tiles are 1
 
 struct WyParams {
   int *status;     // device status word: GDN2_ERR_TIMEOUT (4) when a bounded wait gave up
-  int prefetch_stride;  // WY CTAs resident at once (two per SM)
   int N;           // sequences
   int nc;          // chunks per sequence of a dense batch
+  int nrec;        // records to walk: dense N * nc * H; packed capacity * H (those past the batch are skipped)
+  int reverse;     // dense batches: records in chunk-major order, the last chunk index first
   int64_t tokens;  // rows of the token tensors
   const int32_t *coff;  // packed batch: chunk offsets [N+1]; dense: nullptr
   float *g;             // workspace e^{g_C} [records][128]
-  __nv_bfloat16 *u;     // workspace U = w (.) v, laid out like v
+  int *next;            // record counter, zero at launch: CTAs claim their records after the first in order
 };
 
-__global__ void __launch_bounds__(wy::NT, 2)
-    wy_factor_kernel(const ChunkArgs a, const WyParams p, const __grid_constant__ CUtensorMap tm_q,
-                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_b,
-                     const __grid_constant__ CUtensorMap tm_al, const __grid_constant__ CUtensorMap tm_wm,
-                     const __grid_constant__ CUtensorMap tm_wn, const __grid_constant__ CUtensorMap tm_wq,
-                     const __grid_constant__ CUtensorMap tm_wp, const __grid_constant__ CUtensorMap tm_v,
-                     const __grid_constant__ CUtensorMap tm_w) {
-  using namespace wy;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  const uint32_t sb = smem_u32(sm);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, quad = warp & 3, khalf = warp >> 2;
+// Workspace record of the i-th record a CTA walks.  Dense batches go chunk-major with the last
+// chunk index first, so the records of the first chunks, which the state pass reads first, are the
+// ones written last (most likely still in L2 when it starts).
+__device__ __forceinline__ int wy_record(const WyParams &p, int H, int i) {
+  if (!p.reverse) return i;
+  const int per_c = p.N * H;
+  const int c = p.nc - 1 - i / per_c, rem = i % per_c;
+  return ((rem / H) * p.nc + c) * H + rem % H;
+}
 
-  const int rec = blockIdx.x;  // global chunk * H + head
-  const int h = rec % a.H, gidx = rec / a.H;
+// Token row of the first token of record `rec` (global chunk * H + head), or -1 when the record lies
+// past the chunks of a packed batch.
+__device__ __forceinline__ int wy_tok0(const ChunkArgs &a, const WyParams &p, int rec, int *n_out, int *c_out) {
+  const int gidx = rec / a.H;
   int n, c;
   if (p.coff) {
-    if (gidx >= p.coff[p.N]) return;  // beyond the chunks of the packed batch (uniform per CTA)
+    if (gidx >= p.coff[p.N]) return -1;
     n = seq_of_chunk(p.coff, p.N, gidx);
     c = gidx - p.coff[n];
   } else {
@@ -268,8 +273,28 @@ __global__ void __launch_bounds__(wy::NT, 2)
   int64_t bos;
   int len;
   seq_span(a, n, bos, len);
-  const int Cc = min(C, len - c * C);
-  const int tok0 = (int)(bos + (int64_t)c * C);
+  *n_out = n;
+  *c_out = c;
+  return (int)(bos + (int64_t)c * C);
+}
+
+// Persistent (two CTAs per SM): CTA i takes record i first, then claims the next unclaimed record
+// from a counter when it starts one, so records finish roughly in their walking order and no CTA
+// is left with a long tail.  The set-up (barriers, tensor memory, descriptor prefetch) happens
+// once; every record's inputs are prefetched into L2 one record ahead, and the stores of a record
+// are waited for (their shared-memory sources read) only when the next record's loads are about to
+// overwrite them.
+__global__ void __launch_bounds__(wy::NT, 2)
+    wy_factor_kernel(const ChunkArgs a, const WyParams p, const __grid_constant__ CUtensorMap tm_q,
+                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_b,
+                     const __grid_constant__ CUtensorMap tm_al, const __grid_constant__ CUtensorMap tm_wm,
+                     const __grid_constant__ CUtensorMap tm_wn, const __grid_constant__ CUtensorMap tm_wq,
+                     const __grid_constant__ CUtensorMap tm_wp) {
+  using namespace wy;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, quad = warp & 3, khalf = warp >> 2;
 
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 16);
   const uint32_t bar_full = sb + OFF_BAR, bar_mma = sb + OFF_BAR + 8;
@@ -283,55 +308,11 @@ __global__ void __launch_bounds__(wy::NT, 2)
     mbar_init(bar_mma, 1);
     fence_mbar_init();
     prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_b); prefetch_tmap(&tm_al);
-    mbar_expect_tx(bar_full, TMA_BYTES);
-#pragma unroll
-    for (int blk = 0; blk < 2; ++blk) {
-      tma_load_3d(sb + OFF_XA + blk * XA_BLK, &tm_b, 64 * blk, h, tok0, bar_full);         // b -> rows 0..63
-      tma_load_3d(sb + OFF_XA + blk * XA_BLK + 8192, &tm_q, 64 * blk, h, tok0, bar_full);  // q -> rows 64..127
-      tma_load_3d(sb + OFF_KT + blk * KT_BLK, &tm_k, 64 * blk, h, tok0, bar_full);
-      tma_load_3d(sb + OFF_AL + blk * 8192, &tm_al, 64 * blk, h, tok0, bar_full);
-    }
-    for (int vb = 0; vb < a.dv / 64; ++vb) {  // v and w of this chunk into L2, for U below
-      tma_prefetch_3d(&tm_v, 64 * vb, h, tok0);
-      tma_prefetch_3d(&tm_w, 64 * vb, h, tok0);
-    }
-    // the record about one wave later (CTAs resident at once = prefetch_stride) into L2
-    const int nrec = rec + p.prefetch_stride;
-    if (nrec < (int)gridDim.x) {
-      const int nh = nrec % a.H, ng = nrec / a.H;
-      int nn = -1, ncc = 0;
-      if (p.coff) {
-        if (ng < p.coff[p.N]) {
-          nn = seq_of_chunk(p.coff, p.N, ng);
-          ncc = ng - p.coff[nn];
-        }
-      } else {
-        nn = ng / p.nc;
-        ncc = ng % p.nc;
-      }
-      if (nn >= 0) {
-        int64_t nbos;
-        int nlen;
-        seq_span(a, nn, nbos, nlen);
-        const int ntok = (int)(nbos + (int64_t)ncc * C);
-#pragma unroll
-        for (int blk = 0; blk < 2; ++blk) {
-          tma_prefetch_3d(&tm_b, 64 * blk, nh, ntok);
-          tma_prefetch_3d(&tm_q, 64 * blk, nh, ntok);
-          tma_prefetch_3d(&tm_k, 64 * blk, nh, ntok);
-          tma_prefetch_3d(&tm_al, 64 * blk, nh, ntok);
-        }
-      }
-    }
+    prefetch_tmap(&tm_wm); prefetch_tmap(&tm_wn); prefetch_tmap(&tm_wq); prefetch_tmap(&tm_wp);
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tmem_relinquish();
-  }
-  // the never-written blocks (0,1) and (2,3) of T, which the 32x32 merges read
-  for (int e = tid; e < 512; e += NT) {
-    const int R = 2 * (e >> 8), r = (e >> 4) & 15, j = e & 15;
-    Ts[(16 * R + r) * LDF + 16 * (R + 1) + j] = 0.f;
   }
   tc_fence_before();
   __syncthreads();
@@ -339,373 +320,396 @@ __global__ void __launch_bounds__(wy::NT, 2)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16);
   bool ok = true;
+  uint32_t nfull = 0, nmma = 0;  // completed phases of the two barriers
+  // the claimed next record, in one of two slots by iteration parity (a slot is rewritten only after
+  // every thread has passed the barrier that follows its read)
+  volatile int *s_next = reinterpret_cast<volatile int *>(sm + OFF_BAR + 20);
 
-  // ------------------------------------------------------------ decay factors, operands in place
-  if (!mbar_wait_bounded(bar_full, 0, WAIT_NS)) ok = false;
-  if (__syncthreads_or(!ok)) goto done;
-  {
-    // thread = 8 key channels (chunk x8 of channel block cb) x 4 tokens (group G = rows 4G..4G+3);
-    // groups 0-7 hold tokens 0..31 (walk back to token 31), groups 8-15 tokens 32..63 (walk forward)
-    const int ch8 = tid & 15, G = tid >> 4, cb = ch8 >> 3, x8 = ch8 & 7;
-    uint4 ra[4], rb[4], rq[4], rk[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t o = sw128(4 * G + i, 8 * x8);
-      ra[i] = ld_s128(sm + OFF_AL + cb * 8192 + o);
-      rb[i] = ld_s128(sm + OFF_XA + cb * XA_BLK + o);
-      rq[i] = ld_s128(sm + OFF_XA + cb * XA_BLK + 8192 + o);
-      rk[i] = ld_s128(sm + OFF_KT + cb * KT_BLK + o);
-    }
-    float gp[8];
-#pragma unroll
-    for (int t = 0; t < 8; ++t) gp[t] = 1.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (4 * G + i < Cc) {
-        float al[8];
-        unpack8(ra[i], al);
-#pragma unroll
-        for (int t = 0; t < 8; ++t) gp[t] *= al[t];
-      }
-    *reinterpret_cast<float4 *>(&scan[G * 128 + 8 * ch8]) = make_float4(gp[0], gp[1], gp[2], gp[3]);
-    *reinterpret_cast<float4 *>(&scan[G * 128 + 8 * ch8 + 4]) = make_float4(gp[4], gp[5], gp[6], gp[7]);
+  for (int it = blockIdx.x, nit = 0, par = 0; it < p.nrec; it = nit, par ^= 1) {
+    const int rec = wy_record(p, a.H, it);
+    const int h = rec % a.H;
+    int n, c;
+    const int tok0 = wy_tok0(a, p, rec, &n, &c);
+    if (tid == 0) s_next[par] = (int)gridDim.x + atomicAdd(p.next, 1);
     __syncthreads();
-    if (tid < 128) {  // per channel: products between each group and token 31, in place of the group products
-      float pg[16];
+    nit = s_next[par];
+    if (tok0 < 0) continue;  // past the chunks of a packed batch (uniform per CTA)
+    int64_t bos;
+    int len;
+    seq_span(a, n, bos, len);
+    const int Cc = min(C, len - c * C);
+
+    if (tid == 0) {
+      bulk_wait_read();  // the previous record's stores have read the tiles these loads overwrite
+      mbar_expect_tx(bar_full, TMA_BYTES);
 #pragma unroll
-      for (int g = 0; g < 16; ++g) pg[g] = scan[g * 128 + tid];
-      float acc = 1.f;
-#pragma unroll
-      for (int g = 7; g >= 0; --g) {
-        scan[g * 128 + tid] = acc;  // prod over groups g+1..7
-        acc *= pg[g];
+      for (int blk = 0; blk < 2; ++blk) {
+        tma_load_3d(sb + OFF_XA + blk * XA_BLK, &tm_b, 64 * blk, h, tok0, bar_full);         // b -> rows 0..63
+        tma_load_3d(sb + OFF_XA + blk * XA_BLK + 8192, &tm_q, 64 * blk, h, tok0, bar_full);  // q -> rows 64..127
+        tma_load_3d(sb + OFF_KT + blk * KT_BLK, &tm_k, 64 * blk, h, tok0, bar_full);
+        tma_load_3d(sb + OFF_AL + blk * 8192, &tm_al, 64 * blk, h, tok0, bar_full);
       }
-      const float em = acc;
-      acc = 1.f;
+      // this CTA's next record into L2, so that its loads come from there
+      if (nit < p.nrec) {
+        const int nrec = wy_record(p, a.H, nit);
+        int nn, ncc;
+        const int ntok = wy_tok0(a, p, nrec, &nn, &ncc);
+        if (ntok >= 0) {
 #pragma unroll
-      for (int g = 8; g < 16; ++g) {
-        scan[g * 128 + tid] = acc;  // prod over groups 8..g-1
-        acc *= pg[g];
+          for (int blk = 0; blk < 2; ++blk) {
+            tma_prefetch_3d(&tm_b, 64 * blk, nrec % a.H, ntok);
+            tma_prefetch_3d(&tm_q, 64 * blk, nrec % a.H, ntok);
+            tma_prefetch_3d(&tm_k, 64 * blk, nrec % a.H, ntok);
+            tma_prefetch_3d(&tm_al, 64 * blk, nrec % a.H, ntok);
+          }
+        }
       }
-      s_em[tid] = em;
-      s_egcm[tid] = acc;
-      s_egc[tid] = em * acc;
     }
-    __syncthreads();
-    float run[8];
+
+    // ------------------------------------------------------------ decay factors, operands in place
+    if (!mbar_wait_bounded(bar_full, nfull & 1, WAIT_NS)) ok = false;
+    ++nfull;
+    // the never-written blocks (0,1) and (2,3) of T, which the 32x32 merges read (the region held the
+    // previous record's Pt, whose store has read it)
+    for (int e = tid; e < 512; e += NT) {
+      const int R = 2 * (e >> 8), r = (e >> 4) & 15, j = e & 15;
+      Ts[(16 * R + r) * LDF + 16 * (R + 1) + j] = 0.f;
+    }
+    if (__syncthreads_or(!ok)) goto done;
     {
-      const float4 p0 = *reinterpret_cast<const float4 *>(&scan[G * 128 + 8 * ch8]);
-      const float4 p1 = *reinterpret_cast<const float4 *>(&scan[G * 128 + 8 * ch8 + 4]);
-      run[0] = p0.x; run[1] = p0.y; run[2] = p0.z; run[3] = p0.w;
-      run[4] = p1.x; run[5] = p1.y; run[6] = p1.z; run[7] = p1.w;
-    }
-    uint8_t *pa0 = sm + OFF_XA + cb * XA_BLK, *pk0 = sm + OFF_KT + cb * KT_BLK;
-    if (G < 8) {
-#pragma unroll
-      for (int i = 3; i >= 0; --i) {  // run = prod_{r < s <= 31} alpha_s
-        const int r = 4 * G + i;
-        float al[8], f[8], fi[8];
-        unpack8(ra[i], al);
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          fi[t] = run[t];
-          f[t] = fast_rcp(run[t]);
-          if (r < Cc) run[t] *= al[t];
-        }
-        row_factors(pa0, pk0, sw128(r, 8 * x8), rb[i], rq[i], rk[i], r < Cc, f, fi);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {  // run = prod_{32 <= s <= r} alpha_s
-        const int r = 4 * G + i;
-        float al[8], f[8], fi[8];
-        unpack8(ra[i], al);
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          if (r < Cc) run[t] *= al[t];
-          f[t] = run[t];
-          fi[t] = fast_rcp(run[t]);
-        }
-        row_factors(pa0, pk0, sw128(r, 8 * x8), rb[i], rq[i], rk[i], r < Cc, f, fi);
-      }
-    }
-  }
-  fence_proxy_async();
-  __syncthreads();
-
-  // ------------------------------------------------------------ M1: [L; P] = [A_m; Q_m] K_m^T (TMEM cols 0..63)
-  if (tid == 0) {
-    tc_fence_after();
-#pragma unroll
-    for (int k = 0; k < DK / 16; ++k) {
-      const uint32_t koff = (uint32_t)(k & 3) * 32u;
-      const uint64_t ad = sdesc_sw128(sb + OFF_XA + (k >> 2) * XA_BLK + koff, 16, 1024);
-      const uint64_t bd = sdesc_sw128(sb + OFF_KT + (k >> 2) * KT_BLK + koff, 16, 1024);
-      mma_bf16(tmem + 0, ad, bd, ID_LP, k > 0 ? 1u : 0u);
-    }
-    mma_commit(bar_mma);
-  }
-  {  // while M1 runs: U = w (.) v of this chunk's valid tokens -> workspace (16 threads per 256 B)
-    const int per_row = a.dv / 8;  // 16-byte pieces per token row
-    const size_t row0 = ((size_t)tok0 * a.H + h) * (size_t)a.dv, stride = (size_t)a.H * a.dv;
-    const uint4 *vg = reinterpret_cast<const uint4 *>(a.v), *wg = reinterpret_cast<const uint4 *>(a.w);
-    uint4 *ug = reinterpret_cast<uint4 *>(p.u);
-    for (int base = 0; base < Cc * per_row; base += 4 * NT) {
-      uint4 vv[4], ww[4];
+      // thread = 8 key channels (chunk x8 of channel block cb) x 4 tokens (group G = rows 4G..4G+3);
+      // groups 0-7 hold tokens 0..31 (walk back to token 31), groups 8-15 tokens 32..63 (walk forward)
+      const int ch8 = tid & 15, G = tid >> 4, cb = ch8 >> 3, x8 = ch8 & 7;
+      uint4 ra[4], rb[4], rq[4], rk[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int e = base + i * NT + tid, r = e / per_row;
-        if (r < Cc) {
-          const size_t off = (row0 + (size_t)r * stride) / 8 + (e % per_row);
-          vv[i] = __ldg(vg + off);
-          ww[i] = __ldg(wg + off);
+        const uint32_t o = sw128(4 * G + i, 8 * x8);
+        ra[i] = ld_s128(sm + OFF_AL + cb * 8192 + o);
+        rb[i] = ld_s128(sm + OFF_XA + cb * XA_BLK + o);
+        rq[i] = ld_s128(sm + OFF_XA + cb * XA_BLK + 8192 + o);
+        rk[i] = ld_s128(sm + OFF_KT + cb * KT_BLK + o);
+      }
+      float gp[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) gp[t] = 1.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (4 * G + i < Cc) {
+          float al[8];
+          unpack8(ra[i], al);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) gp[t] *= al[t];
+        }
+      *reinterpret_cast<float4 *>(&scan[G * 128 + 8 * ch8]) = make_float4(gp[0], gp[1], gp[2], gp[3]);
+      *reinterpret_cast<float4 *>(&scan[G * 128 + 8 * ch8 + 4]) = make_float4(gp[4], gp[5], gp[6], gp[7]);
+      __syncthreads();
+      if (tid < 128) {  // per channel: products between each group and token 31, in place of the group products
+        float pg[16];
+#pragma unroll
+        for (int g = 0; g < 16; ++g) pg[g] = scan[g * 128 + tid];
+        float acc = 1.f;
+#pragma unroll
+        for (int g = 7; g >= 0; --g) {
+          scan[g * 128 + tid] = acc;  // prod over groups g+1..7
+          acc *= pg[g];
+        }
+        const float em = acc;
+        acc = 1.f;
+#pragma unroll
+        for (int g = 8; g < 16; ++g) {
+          scan[g * 128 + tid] = acc;  // prod over groups 8..g-1
+          acc *= pg[g];
+        }
+        s_em[tid] = em;
+        s_egcm[tid] = acc;
+        s_egc[tid] = em * acc;
+      }
+      __syncthreads();
+      float run[8];
+      {
+        const float4 p0 = *reinterpret_cast<const float4 *>(&scan[G * 128 + 8 * ch8]);
+        const float4 p1 = *reinterpret_cast<const float4 *>(&scan[G * 128 + 8 * ch8 + 4]);
+        run[0] = p0.x; run[1] = p0.y; run[2] = p0.z; run[3] = p0.w;
+        run[4] = p1.x; run[5] = p1.y; run[6] = p1.z; run[7] = p1.w;
+      }
+      uint8_t *pa0 = sm + OFF_XA + cb * XA_BLK, *pk0 = sm + OFF_KT + cb * KT_BLK;
+      if (G < 8) {
+#pragma unroll
+        for (int i = 3; i >= 0; --i) {  // run = prod_{r < s <= 31} alpha_s
+          const int r = 4 * G + i;
+          float al[8], f[8], fi[8];
+          unpack8(ra[i], al);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            fi[t] = run[t];
+            f[t] = fast_rcp(run[t]);
+            if (r < Cc) run[t] *= al[t];
+          }
+          row_factors(pa0, pk0, sw128(r, 8 * x8), rb[i], rq[i], rk[i], r < Cc, f, fi);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {  // run = prod_{32 <= s <= r} alpha_s
+          const int r = 4 * G + i;
+          float al[8], f[8], fi[8];
+          unpack8(ra[i], al);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            if (r < Cc) run[t] *= al[t];
+            f[t] = run[t];
+            fi[t] = fast_rcp(run[t]);
+          }
+          row_factors(pa0, pk0, sw128(r, 8 * x8), rb[i], rq[i], rk[i], r < Cc, f, fi);
         }
       }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {  // bf16 x bf16 is exact in fp32: the packed product is the rounded one
-        const int e = base + i * NT + tid, r = e / per_row;
-        if (r < Cc) {
-          uint4 uu;
-          uu.x = bf2_mul(vv[i].x, ww[i].x);
-          uu.y = bf2_mul(vv[i].y, ww[i].y);
-          uu.z = bf2_mul(vv[i].z, ww[i].z);
-          uu.w = bf2_mul(vv[i].w, ww[i].w);
-          ug[(row0 + (size_t)r * stride) / 8 + (e % per_row)] = uu;
-        }
-      }
     }
-  }
-  if (!mbar_wait_bounded(bar_mma, 0, WAIT_NS)) ok = false;
-  if (__syncthreads_or(!ok)) goto done;
-  tc_fence_after();
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
 
-  // ------------------------------------------------------------ T = (I + L)^-1
-  {  // L (strict lower) -> fp32 scratch; P (inclusive lower) -> rows 64..127 of [T ; P]
-    float v[32];
-    tmem_ld32(tl + 32 * khalf, v);
-    tmem_wait_ld();
-    const int row = 32 * quad + lane;
-    if (row < 64) {
+    // ------------------------------------------------------------ M1: [L; P] = [A_m; Q_m] K_m^T (TMEM cols 0..63)
+    if (tid == 0) {
+      tc_fence_after();
 #pragma unroll
-      for (int y = 0; y < 8; ++y) {
-        const int i = 32 * khalf + 4 * y;
-        *reinterpret_cast<float4 *>(&Ls[row * LDF + i]) =
-            make_float4(i < row ? v[4 * y] : 0.f, i + 1 < row ? v[4 * y + 1] : 0.f, i + 2 < row ? v[4 * y + 2] : 0.f,
-                        i + 3 < row ? v[4 * y + 3] : 0.f);
+      for (int k = 0; k < DK / 16; ++k) {
+        const uint32_t koff = (uint32_t)(k & 3) * 32u;
+        const uint64_t ad = sdesc_sw128(sb + OFF_XA + (k >> 2) * XA_BLK + koff, 16, 1024);
+        const uint64_t bd = sdesc_sw128(sb + OFF_KT + (k >> 2) * KT_BLK + koff, 16, 1024);
+        mma_bf16(tmem + 0, ad, bd, ID_LP, k > 0 ? 1u : 0u);
       }
-    } else {
-      const int r = row - 64;
-#pragma unroll
-      for (int y = 0; y < 4; ++y) {
-        const int col = 32 * khalf + 8 * y;
-        float e[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) e[t] = (col + t <= r) ? v[8 * y + t] : 0.f;
-        st_s128(sm + OFF_TP + 8192 + sw128(r, col), pack8(e));
-      }
+      mma_commit(bar_mma);
     }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp < 2) {  // the four 16x16 diagonal blocks, right-looking; lane = column j of block R
-    const int R = 2 * warp + (lane >> 4), j = lane & 15;
-    const float *Lb = Ls + 16 * R * LDF + 16 * R;
-    float xv[16];
-#pragma unroll
-    for (int r = 0; r < 16; ++r) xv[r] = (r == j) ? 1.f : 0.f;
-#pragma unroll
-    for (int i = 0; i < 15; ++i)
-#pragma unroll
-      for (int r = i + 1; r < 16; ++r) xv[r] = fmaf(-Lb[r * LDF + i], xv[i], xv[r]);
-    float *Tb = Ts + 16 * R * LDF + 16 * R;
-#pragma unroll
-    for (int r = 0; r < 16; ++r) Tb[r * LDF + j] = xv[r];
-  }
-  __syncthreads();
-  // merges on the warp-level tensor cores (tf32), with [[A,0],[C,B]]^-1 = [[A^-1,0],[-B^-1 C A^-1, B^-1]]:
-  // 16x16 blocks first; a warp needs only its own column tile of Y, so a warp barrier suffices
-  if (warp < 4) {
-    const int R = (warp < 2) ? 1 : 3, nt = warp & 1;
-    float d[4];
-    // Y_R = L_{R,R-1} T_{R-1,R-1}, parked in the upper block (R-1, R) of L
-    mma_tf32_16x8<16>(Ls + 16 * R * LDF + 16 * (R - 1), Ts + 16 * (R - 1) * LDF + 16 * (R - 1) + 8 * nt, lane, d);
-    store_16x8(Ls + 16 * (R - 1) * LDF + 16 * R + 8 * nt, lane, d, 1.f);
-    __syncwarp();
-    // T_{R,R-1} = -T_RR Y_R
-    mma_tf32_16x8<16>(Ts + 16 * R * LDF + 16 * R, Ls + 16 * (R - 1) * LDF + 16 * R + 8 * nt, lane, d);
-    store_16x8(Ts + 16 * R * LDF + 16 * (R - 1) + 8 * nt, lane, d, -1.f);
-  }
-  __syncthreads();
-  {  // lower-left 32x32 block: T[32:64, 0:32] = -T[32:64, 32:64] Y with Y = L[32:64, 0:32] T[0:32, 0:32];
-     // warp (mt, nt) forms both row halves of Y's column tile nt itself and keeps them in registers
-    const int mt = warp >> 2, nt = warp & 3;
-    float y0[4], y1[4], d[4];
-    mma_tf32_16x8<32>(Ls + 32 * LDF, Ts + 8 * nt, lane, y0);
-    mma_tf32_16x8<32>(Ls + 48 * LDF, Ts + 8 * nt, lane, y1);
-    mma_tf32_16x8_yreg(Ts + (32 + 16 * mt) * LDF + 32, y0, y1, lane, d);
-    store_16x8(Ts + (32 + 16 * mt) * LDF + 8 * nt, lane, d, -1.f);
-  }
-  __syncthreads();
-  {  // T -> rows 0..63 of [T ; P], bf16 (the upper-right 32x32 block is zero)
-    const int r = tid >> 2;
-#pragma unroll
-    for (int y = 0; y < 2; ++y) {
-      const int col = 16 * (tid & 3) + 8 * y;
-      float e[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (r >= 32 || col < 32) {
-        const float4 t0 = *reinterpret_cast<const float4 *>(&Ts[r * LDF + col]);
-        const float4 t1 = *reinterpret_cast<const float4 *>(&Ts[r * LDF + col + 4]);
-        e[0] = t0.x; e[1] = t0.y; e[2] = t0.z; e[3] = t0.w; e[4] = t1.x; e[5] = t1.y; e[6] = t1.z; e[7] = t1.w;
-      }
-      st_s128(sm + OFF_TP + sw128(r, col), pack8(e));
-    }
-  }
-  fence_proxy_async();
-  __syncthreads();
-
-  // ------------------------------------------------------------ product pass 1: [T; P] [A_m | T] and K_m^T T
-  // TMEM cols 0..127: rows 0..63 T A_m; cols 128..191: rows 64..127 P T; cols 192..255: K_m^T T
-  if (tid == 0) {
+    if (!mbar_wait_bounded(bar_mma, nmma & 1, WAIT_NS)) ok = false;
+    ++nmma;
+    if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
+
+    // ------------------------------------------------------------ T = (I + L)^-1
+    {  // L (strict lower) -> fp32 scratch; P (inclusive lower) -> rows 64..127 of [T ; P]
+      float v[32];
+      tmem_ld32(tl + 32 * khalf, v);
+      tmem_wait_ld();
+      const int row = 32 * quad + lane;
+      if (row < 64) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint64_t a_tp = sdesc_sw128(sb + OFF_TP + 32 * k, 16, 1024);
-      const uint64_t b_t = sdesc_sw128(sb + OFF_TP + 2048 * k, 8192, 1024);  // T: rows = K, MN-major
-      mma_bf16(tmem + 0, a_tp, sdesc_sw128(sb + OFF_XA + 2048 * k, XA_BLK, 1024), ID_KM128, k > 0 ? 1u : 0u);
-      mma_bf16(tmem + 128, a_tp, b_t, ID_KM64, k > 0 ? 1u : 0u);
-      mma_bf16(tmem + 192, sdesc_sw128(sb + OFF_KT + 2048 * k, KT_BLK, 1024), b_t, ID_MN64, k > 0 ? 1u : 0u);
-    }
-    mma_commit(bar_mma);
-  }
-  if (!mbar_wait_bounded(bar_mma, 1, WAIT_NS)) ok = false;
-  if (__syncthreads_or(!ok)) goto done;
-  tc_fence_after();
-  {
-    const int row = 32 * quad + lane;
-    if (quad < 2) {  // W = -T A_m -> W tile khalf (64 tokens x 64 channels, MN-major B operand)
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        float v[32];
-        tmem_ld32(tl + 64 * khalf + 32 * part, v);
-        tmem_wait_ld();
+        for (int y = 0; y < 8; ++y) {
+          const int i = 32 * khalf + 4 * y;
+          *reinterpret_cast<float4 *>(&Ls[row * LDF + i]) =
+              make_float4(i < row ? v[4 * y] : 0.f, i + 1 < row ? v[4 * y + 1] : 0.f, i + 2 < row ? v[4 * y + 2] : 0.f,
+                          i + 3 < row ? v[4 * y + 3] : 0.f);
+        }
+      } else {
+        const int r = row - 64;
 #pragma unroll
         for (int y = 0; y < 4; ++y) {
+          const int col = 32 * khalf + 8 * y;
           float e[8];
 #pragma unroll
-          for (int t = 0; t < 8; ++t) e[t] = -v[8 * y + t];
-          st_s128(sm + OFF_AL + khalf * 8192 + sw128(row, 32 * part + 8 * y), pack8(e));
+          for (int t = 0; t < 8; ++t) e[t] = (col + t <= r) ? v[8 * y + t] : 0.f;
+          st_s128(sm + OFF_TP + 8192 + sw128(r, col), pack8(e));
         }
       }
-    } else {  // Pt = P T -> rows 64..127 of the products; warp group khalf takes 32 columns
-      float v[32];
-      tmem_ld32(tl + 128 + 32 * khalf, v);
-      tmem_wait_ld();
-#pragma unroll
-      for (int y = 0; y < 4; ++y) st_s128(sm + OFF_TS + sw128(row - 64, 32 * khalf + 8 * y), pack8(&v[8 * y]));
     }
-    {  // Nt = Diag(e^{g_C-m}) K_m^T T, key channel `row`, tokens 32 khalf .. +31
-      float v[32];
-      tmem_ld32(tl + 192 + 32 * khalf, v);
-      tmem_wait_ld();
-      const float g2 = s_egcm[row];
-      const float g2p[2] = {g2, g2};
+    tc_fence_before();
+    __syncthreads();
+    if (warp < 2) {  // the four 16x16 diagonal blocks, right-looking; lane = column j of block R
+      const int R = 2 * warp + (lane >> 4), j = lane & 15;
+      const float *Lb = Ls + 16 * R * LDF + 16 * R;
+      float xv[16];
 #pragma unroll
-      for (int j = 0; j < 32; j += 2) mul2(&v[j], &v[j], g2p);
+      for (int r = 0; r < 16; ++r) xv[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
-      for (int y = 0; y < 4; ++y) st_s128(sm + OFF_TP + sw128(row, 32 * khalf + 8 * y), pack8(&v[8 * y]));
+      for (int i = 0; i < 15; ++i)
+#pragma unroll
+        for (int r = i + 1; r < 16; ++r) xv[r] = fmaf(-Lb[r * LDF + i], xv[i], xv[r]);
+      float *Tb = Ts + 16 * R * LDF + 16 * R;
+#pragma unroll
+      for (int r = 0; r < 16; ++r) Tb[r * LDF + j] = xv[r];
     }
-  }
-  fence_proxy_async();
-  tc_fence_before();
-  __syncthreads();
-  if (tid == 0) {  // Nt, Pt and e^{g_C} are final: store them while product pass 2 runs
-    tma_store_2d(&tm_wn, 0, rec * 128, sb + OFF_TP);
-    tma_store_2d(&tm_wp, 0, rec * 64, sb + OFF_TS);
-    bulk_store(p.g + (size_t)rec * 128, sb + OFF_SC + 256 * 4, REC_G);
-    bulk_commit();
-  }
+    __syncthreads();
+    // merges on the warp-level tensor cores (tf32), with [[A,0],[C,B]]^-1 = [[A^-1,0],[-B^-1 C A^-1, B^-1]]:
+    // 16x16 blocks first; a warp needs only its own column tile of Y, so a warp barrier suffices
+    if (warp < 4) {
+      const int R = (warp < 2) ? 1 : 3, nt = warp & 1;
+      float d[4];
+      // Y_R = L_{R,R-1} T_{R-1,R-1}, parked in the upper block (R-1, R) of L
+      mma_tf32_16x8<16>(Ls + 16 * R * LDF + 16 * (R - 1), Ts + 16 * (R - 1) * LDF + 16 * (R - 1) + 8 * nt, lane, d);
+      store_16x8(Ls + 16 * (R - 1) * LDF + 16 * R + 8 * nt, lane, d, 1.f);
+      __syncwarp();
+      // T_{R,R-1} = -T_RR Y_R
+      mma_tf32_16x8<16>(Ts + 16 * R * LDF + 16 * R, Ls + 16 * (R - 1) * LDF + 16 * R + 8 * nt, lane, d);
+      store_16x8(Ts + 16 * R * LDF + 16 * (R - 1) + 8 * nt, lane, d, -1.f);
+    }
+    __syncthreads();
+    {  // lower-left 32x32 block: T[32:64, 0:32] = -T[32:64, 32:64] Y with Y = L[32:64, 0:32] T[0:32, 0:32];
+       // warp (mt, nt) forms both row halves of Y's column tile nt itself and keeps them in registers
+      const int mt = warp >> 2, nt = warp & 3;
+      float y0[4], y1[4], d[4];
+      mma_tf32_16x8<32>(Ls + 32 * LDF, Ts + 8 * nt, lane, y0);
+      mma_tf32_16x8<32>(Ls + 48 * LDF, Ts + 8 * nt, lane, y1);
+      mma_tf32_16x8_yreg(Ts + (32 + 16 * mt) * LDF + 32, y0, y1, lane, d);
+      store_16x8(Ts + (32 + 16 * mt) * LDF + 8 * nt, lane, d, -1.f);
+    }
+    __syncthreads();
+    {  // T -> rows 0..63 of [T ; P], bf16 (the upper-right 32x32 block is zero)
+      const int r = tid >> 2;
+#pragma unroll
+      for (int y = 0; y < 2; ++y) {
+        const int col = 16 * (tid & 3) + 8 * y;
+        float e[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (r >= 32 || col < 32) {
+          const float4 t0 = *reinterpret_cast<const float4 *>(&Ts[r * LDF + col]);
+          const float4 t1 = *reinterpret_cast<const float4 *>(&Ts[r * LDF + col + 4]);
+          e[0] = t0.x; e[1] = t0.y; e[2] = t0.z; e[3] = t0.w; e[4] = t1.x; e[5] = t1.y; e[6] = t1.z; e[7] = t1.w;
+        }
+        st_s128(sm + OFF_TP + sw128(r, col), pack8(e));
+      }
+    }
+    fence_proxy_async();
+    __syncthreads();
 
-  // ------------------------------------------------------------ product pass 2: K_m^T W and [Pt; *] A_m
-  // TMEM cols 0..127: K_m^T W; cols 128..255: rows 0..63 Pt A_m (rows 64..127 read whatever follows Pt)
-  if (tid == 0) {
-    tc_fence_after();
+    // ------------------------------------------------------------ product pass 1: [T; P] [A_m | T] and K_m^T T
+    // TMEM cols 0..127: rows 0..63 T A_m; cols 128..191: rows 64..127 P T; cols 192..255: K_m^T T
+    if (tid == 0) {
+      tc_fence_after();
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      mma_bf16(tmem + 0, sdesc_sw128(sb + OFF_KT + 2048 * k, KT_BLK, 1024), sdesc_sw128(sb + OFF_AL + 2048 * k, 8192, 1024),
-               ID_MN128, k > 0 ? 1u : 0u);
-      mma_bf16(tmem + 128, sdesc_sw128(sb + OFF_TS + 32 * k, 16, 1024), sdesc_sw128(sb + OFF_XA + 2048 * k, XA_BLK, 1024),
-               ID_KM128, k > 0 ? 1u : 0u);
+      for (int k = 0; k < 4; ++k) {
+        const uint64_t a_tp = sdesc_sw128(sb + OFF_TP + 32 * k, 16, 1024);
+        const uint64_t b_t = sdesc_sw128(sb + OFF_TP + 2048 * k, 8192, 1024);  // T: rows = K, MN-major
+        mma_bf16(tmem + 0, a_tp, sdesc_sw128(sb + OFF_XA + 2048 * k, XA_BLK, 1024), ID_KM128, k > 0 ? 1u : 0u);
+        mma_bf16(tmem + 128, a_tp, b_t, ID_KM64, k > 0 ? 1u : 0u);
+        mma_bf16(tmem + 192, sdesc_sw128(sb + OFF_KT + 2048 * k, KT_BLK, 1024), b_t, ID_MN64, k > 0 ? 1u : 0u);
+      }
+      mma_commit(bar_mma);
     }
-    mma_commit(bar_mma);
-  }
-  if (!mbar_wait_bounded(bar_mma, 0, WAIT_NS)) ok = false;
-  if (__syncthreads_or(!ok)) goto done;
-  tc_fence_after();
-  {
-    const int row = 32 * quad + lane;
-    {  // Mt = Diag(e^{g_C-m}) K_m^T W Diag(e^m): row = key channel, input channels 64 khalf .. +63
-      const float g2 = s_egcm[row];
-      uint8_t *dst = sm + (khalf ? OFF_AL : OFF_KT);
+    if (!mbar_wait_bounded(bar_mma, nmma & 1, WAIT_NS)) ok = false;
+    ++nmma;
+    if (__syncthreads_or(!ok)) goto done;
+    tc_fence_after();
+    {
+      const int row = 32 * quad + lane;
+      if (quad < 2) {  // W' = -T A_m Diag(e^m) -> W tile khalf (64 tokens x 64 channels, MN-major B operand)
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
+        for (int part = 0; part < 2; ++part) {
+          float v[32];
+          tmem_ld32(tl + 64 * khalf + 32 * part, v);
+          tmem_wait_ld();
+          const float4 *em4 = reinterpret_cast<const float4 *>(s_em + 64 * khalf + 32 * part);
+#pragma unroll
+          for (int y = 0; y < 8; ++y) {  // times -e^m of each channel
+            const float4 e = em4[y];
+            const float ne[4] = {-e.x, -e.y, -e.z, -e.w};
+            mul2(&v[4 * y], &v[4 * y], &ne[0]);
+            mul2(&v[4 * y + 2], &v[4 * y + 2], &ne[2]);
+          }
+#pragma unroll
+          for (int y = 0; y < 4; ++y)
+            st_s128(sm + OFF_AL + khalf * 8192 + sw128(row, 32 * part + 8 * y), pack8(&v[8 * y]));
+        }
+      } else {  // Pt = P T -> rows 64..127 of the products; warp group khalf takes 32 columns
         float v[32];
-        tmem_ld32(tl + 64 * khalf + 32 * part, v);
+        tmem_ld32(tl + 128 + 32 * khalf, v);
         tmem_wait_ld();
-        const float4 *em4 = reinterpret_cast<const float4 *>(s_em + 64 * khalf + 32 * part);
+#pragma unroll
+        for (int y = 0; y < 4; ++y) st_s128(sm + OFF_TS + sw128(row - 64, 32 * khalf + 8 * y), pack8(&v[8 * y]));
+      }
+      {  // Nt = Diag(e^{g_C-m}) K_m^T T, key channel `row`, tokens 32 khalf .. +31
+        float v[32];
+        tmem_ld32(tl + 192 + 32 * khalf, v);
+        tmem_wait_ld();
+        const float g2 = s_egcm[row];
         const float g2p[2] = {g2, g2};
 #pragma unroll
-        for (int y = 0; y < 8; ++y) {  // v (g2 e^m), as in the scalar order
-          const float4 e = em4[y];
-          float sc[4] = {e.x, e.y, e.z, e.w};
-          mul2(&sc[0], g2p, &sc[0]);
-          mul2(&sc[2], g2p, &sc[2]);
-          mul2(&v[4 * y], &v[4 * y], &sc[0]);
-          mul2(&v[4 * y + 2], &v[4 * y + 2], &sc[2]);
-        }
+        for (int j = 0; j < 32; j += 2) mul2(&v[j], &v[j], g2p);
 #pragma unroll
-        for (int y = 0; y < 4; ++y) st_s128(dst + sw128(row, 32 * part + 8 * y), pack8(&v[8 * y]));
+        for (int y = 0; y < 4; ++y) st_s128(sm + OFF_TP + sw128(row, 32 * khalf + 8 * y), pack8(&v[8 * y]));
       }
     }
-    if (quad < 2) {  // Qt = (Q_m - Pt A_m) Diag(e^m) in place of A_m, channel block khalf
-      uint8_t *blk = sm + OFF_XA + khalf * XA_BLK;
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        float v[32];
-        tmem_ld32(tl + 128 + 64 * khalf + 32 * part, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int y = 0; y < 4; ++y) {
-          const int col = 32 * part + 8 * y;
-          float qm[8], e[8];
-          unpack8(ld_s128(blk + 8192 + sw128(row, col)), qm);
-#pragma unroll
-          for (int t = 0; t < 8; t += 2) {
-            const float2 dq = __fadd2_rn(make_float2(qm[t], qm[t + 1]), make_float2(-v[8 * y + t], -v[8 * y + t + 1]));
-            const float2 r = __fmul2_rn(dq, *reinterpret_cast<const float2 *>(&s_em[64 * khalf + col + t]));
-            e[t] = r.x;
-            e[t + 1] = r.y;
-          }
-          st_s128(blk + sw128(row, col), pack8(e));
-        }
-      }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {  // Nt, Pt and e^{g_C} are final: store them while product pass 2 runs
+      tma_store_2d(&tm_wn, 0, rec * 128, sb + OFF_TP);
+      tma_store_2d(&tm_wp, 0, rec * 64, sb + OFF_TS);
+      bulk_store(p.g + (size_t)rec * 128, sb + OFF_SC + 256 * 4, REC_G);
+      bulk_commit();
     }
-  }
-  fence_proxy_async();
-  tc_fence_before();
-  __syncthreads();
 
-  // ------------------------------------------------------------ the record -> workspace
-  if (tid == 0) {
-    tma_store_2d(&tm_wm, 0, rec * 128, sb + OFF_KT);
-    tma_store_2d(&tm_wm, 64, rec * 128, sb + OFF_AL);
-    tma_store_2d(&tm_wq, 0, rec * 64, sb + OFF_XA);
-    tma_store_2d(&tm_wq, 64, rec * 64, sb + OFF_XA + XA_BLK);
-    bulk_commit();
-    bulk_wait_read();
+    // ------------------------------------------------------------ product pass 2: K_m^T W' and [Pt; *] A_m
+    // TMEM cols 0..127: K_m^T W'; cols 128..255: rows 0..63 Pt A_m (rows 64..127 read whatever follows Pt)
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        mma_bf16(tmem + 0, sdesc_sw128(sb + OFF_KT + 2048 * k, KT_BLK, 1024),
+                 sdesc_sw128(sb + OFF_AL + 2048 * k, 8192, 1024), ID_MN128, k > 0 ? 1u : 0u);
+        mma_bf16(tmem + 128, sdesc_sw128(sb + OFF_TS + 32 * k, 16, 1024),
+                 sdesc_sw128(sb + OFF_XA + 2048 * k, XA_BLK, 1024), ID_KM128, k > 0 ? 1u : 0u);
+      }
+      mma_commit(bar_mma);
+    }
+    if (!mbar_wait_bounded(bar_mma, nmma & 1, WAIT_NS)) ok = false;
+    ++nmma;
+    if (__syncthreads_or(!ok)) goto done;
+    tc_fence_after();
+    {
+      const int row = 32 * quad + lane;
+      {  // Mt = Diag(e^{g_C-m}) K_m^T W': row = key channel, input channels 64 khalf .. +63
+        const float g2 = s_egcm[row];
+        const float g2p[2] = {g2, g2};
+        uint8_t *dst = sm + (khalf ? OFF_AL : OFF_KT);
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          float v[32];
+          tmem_ld32(tl + 64 * khalf + 32 * part, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) mul2(&v[j], &v[j], g2p);
+#pragma unroll
+          for (int y = 0; y < 4; ++y) st_s128(dst + sw128(row, 32 * part + 8 * y), pack8(&v[8 * y]));
+        }
+      }
+      if (quad < 2) {  // Qt = (Q_m - Pt A_m) Diag(e^m) in place of A_m, channel block khalf
+        uint8_t *blk = sm + OFF_XA + khalf * XA_BLK;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          float v[32];
+          tmem_ld32(tl + 128 + 64 * khalf + 32 * part, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int y = 0; y < 4; ++y) {
+            const int col = 32 * part + 8 * y;
+            float qm[8], e[8];
+            unpack8(ld_s128(blk + 8192 + sw128(row, col)), qm);
+#pragma unroll
+            for (int t = 0; t < 8; t += 2) {
+              const float2 dq = __fadd2_rn(make_float2(qm[t], qm[t + 1]), make_float2(-v[8 * y + t], -v[8 * y + t + 1]));
+              const float2 r = __fmul2_rn(dq, *reinterpret_cast<const float2 *>(&s_em[64 * khalf + col + t]));
+              e[t] = r.x;
+              e[t + 1] = r.y;
+            }
+            st_s128(blk + sw128(row, col), pack8(e));
+          }
+        }
+      }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+
+    // ------------------------------------------------------------ the record -> workspace (waited for at the next record)
+    if (tid == 0) {
+      tma_store_2d(&tm_wm, 0, rec * 128, sb + OFF_KT);
+      tma_store_2d(&tm_wm, 64, rec * 128, sb + OFF_AL);
+      tma_store_2d(&tm_wq, 0, rec * 64, sb + OFF_XA);
+      tma_store_2d(&tm_wq, 64, rec * 64, sb + OFF_XA + XA_BLK);
+      bulk_commit();
+    }
   }
 
 done:
   if (!ok && tid == 0) atomicExch(p.status, 4);
+  if (tid == 0) bulk_wait_read();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -717,50 +721,58 @@ done:
 // ==================================================================== kernel 2: state pass
 // One CTA per (sequence, head, 128 value columns).  The products run transposed, with the state as
 // the A operand straight from tensor memory (value column = TMEM lane):
-//   D1^T = U^T Nt^T + S^T Mt^T   (128 value columns x 128 key channels)
-//   O^T  = S^T Qt^T + U^T Pt^T   (128 value columns x 64 tokens)
-// Roles: warps 0-7 hold the state (thread = value column v, key-channel half hf: S[64 hf ..][v]);
-// one thread of warp 8 loads chunks (U = w (.) v comes ready-made from the WY kernel); one thread
-// of warp 9 issues the products; one thread of warp 10 stores O.
-// Tensor memory is double-buffered per chunk parity, so the U half of D1 and the output of chunk c
-// overlap the state chain, whose step per chunk is: S^T -> TMEM, S^T Mt^T, S update.
-// The two U products share one MMA of N = 192 (Nt and Pt lie back to back in shared memory).
+//   [D1^T | O^T] = U^T [Nt^T | Pt^T] + S^T [Mt^T | Qt^T]   (128 value columns x (128 keys + 64 tokens))
+// as two MMAs of N = 192 per K step: one over U (K = 64 tokens) and one over S (K = 128 keys), whose
+// B operands are Nt over Pt and Mt over Qt, stacked row-wise in shared memory.
+// Roles:
+//   warps 0-7   the state (thread = value column v, key-channel half hf: S[64 hf ..][v]); they do
+//               nothing but the serial chain per chunk: D1 -> S update -> S^T into tensor memory;
+//   warp 8      lane 0 loads each chunk's Mt, e^{g_C} and Qt, lane 1 its v, w, Nt and Pt;
+//   warp 9      lane 0 issues the products;
+//   warps 10-13 form U = w (.) v in shared memory in place of v (tokens past a sequence's end
+//               zero), and read O^T out of tensor memory and store it (staged, one TMA store).
+// A chunk's buffers come in two parts, each double-buffered by chunk parity and released as soon
+// as the product that reads it completes: {v, w, Nt, Pt} after the U product, {Mt, Qt, e^{g_C}}
+// after the S product (and the state warps' read of e^{g_C}); so the loads of chunk c+2 start
+// while chunk c+1 is still in flight.  Tensor memory is double-buffered per chunk parity.
 namespace sp {
 constexpr int VW = 128;        // value columns per CTA
 constexpr int NSTATE = 256;    // warps 0-7
-constexpr int W_LOAD = 8, W_MMA = 9, W_STORE = 10;
-constexpr int NT = 352;
-constexpr int BAR_STATE = 1;
+constexpr int W_LOAD = 8, W_MMA = 9, W_AUX = 10, NAUX = 128;
+constexpr int NT = 448;
+constexpr int BAR_STATE = 1, BAR_AUX = 2;
 // one stage (chunk buffer); every operand tile 1024-aligned
-constexpr uint32_t S_M = 0;                  // Mt: two tiles (input channel blocks), 128 rows each
-constexpr uint32_t S_Q = S_M + REC_M;        // 32768: Qt: two tiles of 64 rows
-constexpr uint32_t S_N = S_Q + REC_Q;        // 49152: Nt, 128 rows, and right after it
+constexpr uint32_t MQ_BLK = 24576;           // one input channel block: Mt (128 rows) over Qt (64 rows)
+constexpr uint32_t S_MQ = 0;                 // two such blocks
+constexpr uint32_t S_N = S_MQ + 2 * MQ_BLK;  // 49152: Nt, 128 rows, and right after it
 constexpr uint32_t S_P = S_N + REC_N;        // 65536: Pt, 64 rows (together one 192-row operand)
-constexpr uint32_t S_U = S_P + REC_P;        // 73728: U = w (.) v: two 64-column tiles of 64 tokens
-constexpr uint32_t STAGE = S_U + 16384;      // 90112
-constexpr uint32_t OFF_OST = 2 * STAGE;      // 180224: O staging, two 64-column tiles of 64 tokens
-constexpr uint32_t OFF_G = OFF_OST + 16384;  // 196608: e^{g_C} of the two stages
-constexpr uint32_t OFF_BAR = OFF_G + 2 * REC_G;  // 197632
+constexpr uint32_t S_V = S_P + REC_P;        // 73728: v, two 64-column tiles of 64 tokens -> U = w (.) v in place
+constexpr uint32_t S_W = S_V + 16384;        // 90112: w, likewise
+constexpr uint32_t STAGE = S_W + 16384;      // 106496
+constexpr uint32_t OFF_OST = 2 * STAGE;      // 212992: O staging, two 64-column tiles of 64 tokens
+constexpr uint32_t OFF_G = OFF_OST + 16384;  // 229376: e^{g_C} of the two stages
+constexpr uint32_t OFF_BAR = OFF_G + 2 * REC_G;  // 230400
 constexpr uint32_t SMEM_USED = OFF_BAR + 256;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 constexpr uint32_t TMEM_COLS = 512;
 // per buffer b = chunk parity (256 columns at 256 b): S^T (bf16 pairs) 64 cols, then D1^T 128 cols
 // and O^T 64 cols side by side, so one MMA of N = 192 writes U^T [Nt^T | Pt^T] into both
 constexpr uint32_t TM_AS = 0, TM_D1 = 64, TM_D2 = 192;
-constexpr uint32_t ID_D1 = idesc_bf16(128, 128, false, false), ID_D2 = idesc_bf16(128, 64, false, false);
-constexpr uint32_t ID_U = idesc_bf16(128, 192, true, false), ID_U1 = idesc_bf16(128, 128, true, false);
+constexpr uint32_t ID_192 = idesc_bf16(128, 192, false, false), ID_128 = idesc_bf16(128, 128, false, false);
+constexpr uint32_t ID_U192 = idesc_bf16(128, 192, true, false), ID_U128 = idesc_bf16(128, 128, true, false);
 enum {
-  B_FULL0 = 0, B_FULL1,      // stage loaded (TMA bytes)
-  B_UZERO,                   // rows of U past a sequence's end zeroed (its last, partial chunk) (one arrive per U warp)
+  B_FU0 = 0, B_FU1,          // v, w, Nt, Pt of the stage loaded
+  B_FM0, B_FM1,              // Mt, Qt and e^{g_C} loaded
+  B_UREADY0, B_UREADY1,      // U^T of the stage formed by the aux warps
+  B_UFREE0, B_UFREE1,        // the U product of the stage complete: v, w, Nt, Pt free
   B_SREADY,                  // S^T of the next chunk is in tensor memory
-  B_D1FULL0, B_D1FULL1,      // D1 of the buffer complete
-  B_D1FREE0, B_D1FREE1,      // D1 of the buffer read by the state warps
-  B_D2FULL0, B_D2FULL1,      // O^T of the buffer complete
-  B_OSTAGED0, B_OSTAGED1,    // O of the chunk read out (staged, or stored directly); O^T of the buffer free
-  B_OFREE,                   // the O staging buffer has been read by its store
+  B_D1FULL0, B_D1FULL1,      // every product of the buffer's chunk complete: D1 and O^T (Mt, Qt free)
+  B_D1FREE0, B_D1FREE1,      // D1 of the buffer and the stage's e^{g_C} read by the state warps
+  B_OREAD0, B_OREAD1,        // O^T of the buffer read out by the aux warps
   B_COUNT
 };
 static_assert(SMEM_BYTES <= 232448, "one CTA per SM");
+static_assert(8 * B_COUNT + 4 <= 256, "barriers and the tensor-memory slot fit their region");
 }  // namespace sp
 
 // How one state-pass CTA is placed and what it produces.  Mode 0 walks whole sequences.  For long
@@ -778,11 +790,16 @@ struct ScanParams {
   float *s_start;  // [N][H][nseg][128][d_v]: entry state of segment j >= 1 (mode 2)
 };
 
+// Shared-memory matrix descriptor of the tile at byte offset `off` from the one `base` describes
+// (the start address is the descriptor's low field, in 16-byte units; offsets stay inside the CTA's
+// shared memory, so the field never carries).
+__device__ __forceinline__ uint64_t desc_at(uint64_t base, uint32_t off) { return base + (uint64_t)(off >> 4); }
+
 __global__ void __launch_bounds__(sp::NT, 1)
     state_pass_kernel(const ChunkArgs a, const WyParams p, const ScanParams q, const __grid_constant__ CUtensorMap tm_wm,
                       const __grid_constant__ CUtensorMap tm_wn, const __grid_constant__ CUtensorMap tm_wq,
-                      const __grid_constant__ CUtensorMap tm_wp, const __grid_constant__ CUtensorMap tm_u,
-                      const __grid_constant__ CUtensorMap tm_o) {
+                      const __grid_constant__ CUtensorMap tm_wp, const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_o) {
   using namespace sp;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -826,13 +843,12 @@ __global__ void __launch_bounds__(sp::NT, 1)
   const int nk = max(ce - cb, 0);  // chunks of this CTA, local index k -> chunk cb + k
   const int coff = p.coff ? p.coff[n] : n * p.nc;  // global chunk of this sequence's chunk 0
   auto chunk_len = [&](int c) { return min(C, len - c * C); };
-  const uint32_t tx_bytes = REC_M + REC_G + (use_u ? REC_N + 2 * 8192 : 0) + (use_o ? REC_Q + REC_P : 0);
 
   if (tid == 0) {
     for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), 1u);
     fence_mbar_init();
     prefetch_tmap(&tm_wm); prefetch_tmap(&tm_wn); prefetch_tmap(&tm_wq); prefetch_tmap(&tm_wp);
-    prefetch_tmap(&tm_u); prefetch_tmap(&tm_o);
+    prefetch_tmap(&tm_v); prefetch_tmap(&tm_w); prefetch_tmap(&tm_o);
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
@@ -845,67 +861,83 @@ __global__ void __launch_bounds__(sp::NT, 1)
   bool ok = true;
 
   if (warp == W_LOAD) {
-    // ---------------------------------------------------------- loads (one thread)
     if (lane == 0) {
-      auto prefetch = [&](int c) {  // chunk c into L2, so its later load from there is short
-        const int rp = (coff + c) * a.H + h, tp = (int)(bos + (int64_t)c * C);
-        tma_prefetch_2d(&tm_wm, 0, rp * 128);
-        tma_prefetch_2d(&tm_wm, 64, rp * 128);
-        if (use_u) {
-          tma_prefetch_2d(&tm_wn, 0, rp * 128);
-#pragma unroll
-          for (int vb = 0; vb < 2; ++vb)
-            if (j0 + 64 * vb < a.dv) tma_prefetch_3d(&tm_u, j0 + 64 * vb, h, tp);
-        }
-        if (use_o) {
-          tma_prefetch_2d(&tm_wq, 0, rp * 64);
-          tma_prefetch_2d(&tm_wq, 64, rp * 64);
-          tma_prefetch_2d(&tm_wp, 0, rp * 64);
-        }
-        bulk_prefetch(p.g + (size_t)rp * 128, REC_G);
-      };
-      if (nk > 1) prefetch(cb + 1);  // chunk cb is loaded at once; chunk c+2 follows chunk c's load
+      // ---------------------------------------------------------- Mt, Qt, e^{g_C} of each chunk
       for (int k = 0; k < nk; ++k) {
-        const int s = k & 1, c = cb + k;
-        // stage s last held chunk k-2: free once its products are complete and its e^{g_C} is read
-        if (k >= 2 && !(mbar_wait_bounded(bar(B_D2FULL0 + s), ((k - 2) >> 1) & 1, WAIT_NS) &&
-                        mbar_wait_bounded(bar(B_D1FREE0 + s), ((k - 2) >> 1) & 1, WAIT_NS))) {
+        const int s = k & 1, c = cb + k, ph2 = ((k - 2) >> 1) & 1;
+        const uint32_t st = sb + s * STAGE, full = bar(B_FM0 + s);
+        const int rec = (coff + c) * a.H + h;
+        // chunk k-2's: read once its products are complete and the state warps read e^{g_C}
+        if (k >= 2 && !(mbar_wait_bounded(bar(B_D1FULL0 + s), ph2, WAIT_NS) &&
+                        mbar_wait_bounded(bar(B_D1FREE0 + s), ph2, WAIT_NS))) {
           ok = false;
           break;
         }
-        const uint32_t st = sb + s * STAGE, full = bar(B_FULL0 + s);
-        const int rec = (coff + c) * a.H + h;
-        const int tok0 = (int)(bos + (int64_t)c * C);
-        mbar_expect_tx(full, tx_bytes);
-        tma_load_2d(st + S_M, &tm_wm, 0, rec * 128, full);
-        tma_load_2d(st + S_M + 16384, &tm_wm, 64, rec * 128, full);
-        if (use_u) {
-          tma_load_2d(st + S_N, &tm_wn, 0, rec * 128, full);
+        mbar_expect_tx(full, REC_M + REC_G + (use_o ? REC_Q : 0));
 #pragma unroll
-          for (int vb = 0; vb < 2; ++vb)  // columns past d_v (d_v = 64) load as zeros
-            tma_load_3d(st + S_U + vb * 8192, &tm_u, j0 + 64 * vb, h, tok0, full);
-        }
-        if (use_o) {
-          tma_load_2d(st + S_Q, &tm_wq, 0, rec * 64, full);
-          tma_load_2d(st + S_Q + 8192, &tm_wq, 64, rec * 64, full);
-          tma_load_2d(st + S_P, &tm_wp, 0, rec * 64, full);
+        for (int blk = 0; blk < 2; ++blk) {
+          tma_load_2d(st + S_MQ + blk * MQ_BLK, &tm_wm, 64 * blk, rec * 128, full);
+          if (use_o) tma_load_2d(st + S_MQ + blk * MQ_BLK + 16384, &tm_wq, 64 * blk, rec * 64, full);
         }
         bulk_load(sb + OFF_G + s * REC_G, p.g + (size_t)rec * 128, REC_G, full);
-        if (k + 2 < nk) prefetch(c + 2);
+        if (k + 2 < nk) {  // chunk k+2 into L2, so its later load from there is short
+          const int rp = rec + 2 * a.H;
+          tma_prefetch_2d(&tm_wm, 0, rp * 128);
+          tma_prefetch_2d(&tm_wm, 64, rp * 128);
+          if (use_o) {
+            tma_prefetch_2d(&tm_wq, 0, rp * 64);
+            tma_prefetch_2d(&tm_wq, 64, rp * 64);
+          }
+          bulk_prefetch(p.g + (size_t)rp * 128, REC_G);
+        }
+      }
+    } else if (lane == 1 && use_u) {
+      // ---------------------------------------------------------- v, w, Nt, Pt of each chunk
+      const uint32_t bytes = 4 * 8192 + REC_N + (use_o ? REC_P : 0);
+      for (int k = 0; k < nk; ++k) {
+        const int s = k & 1, c = cb + k;
+        const uint32_t st = sb + s * STAGE, full = bar(B_FU0 + s);
+        const int rec = (coff + c) * a.H + h;
+        const int tok0 = (int)(bos + (int64_t)c * C);
+        if (k >= 2 && !mbar_wait_bounded(bar(B_UFREE0 + s), ((k - 2) >> 1) & 1, WAIT_NS)) {
+          ok = false;
+          break;
+        }
+        mbar_expect_tx(full, bytes);
+#pragma unroll
+        for (int vb = 0; vb < 2; ++vb) {  // columns past d_v (d_v = 64) load as zeros
+          tma_load_3d(st + S_V + vb * 8192, &tm_v, j0 + 64 * vb, h, tok0, full);
+          tma_load_3d(st + S_W + vb * 8192, &tm_w, j0 + 64 * vb, h, tok0, full);
+        }
+        tma_load_2d(st + S_N, &tm_wn, 0, rec * 128, full);
+        if (use_o) tma_load_2d(st + S_P, &tm_wp, 0, rec * 64, full);
+        if (k + 2 < nk) {
+          const int rp = rec + 2 * a.H, tp = tok0 + 2 * C;
+#pragma unroll
+          for (int vb = 0; vb < 2; ++vb)
+            if (j0 + 64 * vb < a.dv) {
+              tma_prefetch_3d(&tm_v, j0 + 64 * vb, h, tp);
+              tma_prefetch_3d(&tm_w, j0 + 64 * vb, h, tp);
+            }
+          tma_prefetch_2d(&tm_wn, 0, rp * 128);
+          if (use_o) tma_prefetch_2d(&tm_wp, 0, rp * 64);
+        }
       }
     }
   } else if (warp == W_MMA) {
     // ---------------------------------------------------------- products (one thread)
     if (lane == 0) {
+      const uint64_t dk_base = sdesc_sw128(sb, 16, 1024);    // K-major operand tiles
+      const uint64_t dmn_base = sdesc_sw128(sb, 8192, 1024); // MN-major U (two 64-column tiles 8 KB apart)
       for (int k = 0; k < nk; ++k) {
-        const int s = k & 1, b = k & 1, ph = (k >> 1) & 1, c = cb + k;
-        const uint32_t stg = sb + s * STAGE;
-        const uint32_t as = tmem + 256 * b + TM_AS, d1 = tmem + 256 * b + TM_D1, d2 = tmem + 256 * b + TM_D2;
-        if (!mbar_wait_bounded(bar(B_FULL0 + s), ph, WAIT_NS)) { ok = false; break; }
-        if (use_u && chunk_len(c) < C && !mbar_wait_bounded(bar(B_UZERO), 0, WAIT_NS)) { ok = false; break; }
-        // D1 and O^T of this buffer were last read by chunk k-2
+        const int s = k & 1, b = k & 1, ph = (k >> 1) & 1;
+        const uint32_t stg = s * STAGE;
+        const uint32_t as = tmem + 256 * b + TM_AS, d1 = tmem + 256 * b + TM_D1;
+        const uint32_t id = use_o ? ID_192 : ID_128;  // [D1 | O^T], or D1 alone
+        if (use_u && !mbar_wait_bounded(bar(B_UREADY0 + s), ph, WAIT_NS)) { ok = false; break; }
+        // D1 and O^T of this buffer were last read for chunk k-2
         if (k >= 2 && !(mbar_wait_bounded(bar(B_D1FREE0 + b), ph ^ 1, WAIT_NS) &&
-                        mbar_wait_bounded(bar(B_OSTAGED0 + b), ph ^ 1, WAIT_NS))) {
+                        (!use_o || mbar_wait_bounded(bar(B_OREAD0 + b), ph ^ 1, WAIT_NS)))) {
           ok = false;
           break;
         }
@@ -913,40 +945,94 @@ __global__ void __launch_bounds__(sp::NT, 1)
         if (use_u) {  // U^T Nt^T (and U^T Pt^T for the output), before the state is known
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(d1, sdesc_sw128(stg + S_U + 2048 * kk, 8192, 1024), sdesc_sw128(stg + S_N + 32 * kk, 16, 1024),
-                     use_o ? ID_U : ID_U1, kk > 0 ? 1u : 0u);
+            mma_bf16(d1, desc_at(dmn_base, stg + S_V + 2048 * kk), desc_at(dk_base, stg + S_N + 32 * kk),
+                     use_o ? ID_U192 : ID_U128, kk > 0 ? 1u : 0u);
+          mma_commit(bar(B_UFREE0 + s));
         }
-        if (!mbar_wait_bounded(bar(B_SREADY), k & 1, WAIT_NS)) { ok = false; break; }
+        if (!mbar_wait_bounded(bar(B_FM0 + s), ph, WAIT_NS) || !mbar_wait_bounded(bar(B_SREADY), k & 1, WAIT_NS)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk)
-          mma_bf16_tmem_a(d1, as + 8 * kk, sdesc_sw128(stg + S_M + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), ID_D1,
+          mma_bf16_tmem_a(d1, as + 8 * kk, desc_at(dk_base, stg + S_MQ + (kk >> 2) * MQ_BLK + (kk & 3) * 32), id,
                           (use_u || kk > 0) ? 1u : 0u);
         mma_commit(bar(B_D1FULL0 + b));
-        if (use_o) {
-#pragma unroll
-          for (int kk = 0; kk < DK / 16; ++kk)
-            mma_bf16_tmem_a(d2, as + 8 * kk, sdesc_sw128(stg + S_Q + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), ID_D2,
-                            1u);
-        }
-        mma_commit(bar(B_D2FULL0 + b));  // with no output products this completes with D1
       }
     }
-  } else if (warp == W_STORE) {
-    // ---------------------------------------------------------- O stores (one thread)
-    if (lane == 0 && use_o) {
-      for (int k = 0; k < nk; ++k) {  // O of chunk cb + k, staged by the state warps -> global
-        if (!mbar_wait_bounded(bar(B_OSTAGED0 + (k & 1)), (k >> 1) & 1, WAIT_NS)) { ok = false; break; }
-        if (chunk_len(cb + k) == C) {
-          const int tok0 = (int)(bos + (int64_t)(cb + k) * C);
+  } else if (warp >= W_AUX) {
+    // ---------------------------------------------------------- U formation and O readout (warps 10-13)
+    const int atid = tid - W_AUX * 32, aq = warp & 3;
+    // U = w (.) v of chunk cb + k in place of v (16-byte pieces, each read and written by one thread);
+    // tokens past the sequence (the tile holds the next sequence's tokens there) become zero
+    auto form_u = [&](int k) -> bool {
+      const int s = k & 1;
+      if (!group_wait(BAR_AUX, NAUX, bar(B_FU0 + s), (k >> 1) & 1)) return false;
+      const int Cc = chunk_len(cb + k);
+      uint8_t *vt = sm + s * STAGE + S_V, *wt = sm + s * STAGE + S_W;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {  // pieces: 64 rows x (2 tiles x 8)
+        const int e = atid + NAUX * i, r = e >> 4, x = e & 15;
+        const uint32_t off = (uint32_t)(x >> 3) * 8192u + sw128(r, 8 * (x & 7));
+        uint4 u = make_uint4(0u, 0u, 0u, 0u);
+        if (r < Cc) {  // bf16 x bf16 is exact in fp32: the packed product is the rounded one
+          const uint4 vv = ld_s128(vt + off), ww = ld_s128(wt + off);
+          u.x = bf2_mul(vv.x, ww.x);
+          u.y = bf2_mul(vv.y, ww.y);
+          u.z = bf2_mul(vv.z, ww.z);
+          u.w = bf2_mul(vv.w, ww.w);
+        }
+        st_s128(vt + off, u);
+      }
+      fence_proxy_async();
+      group_sync(BAR_AUX, NAUX);
+      if (atid == 0) mbar_arrive(bar(B_UREADY0 + s));
+      return true;
+    };
+    // O readout: thread = value column v of the tile (TMEM lane), all 64 tokens of the chunk; a full
+    // chunk is staged in the swizzled layout of the output map and stored by TMA, the last partial
+    // chunk of a sequence goes straight to global memory (a box would overrun into the next sequence)
+    const int v = 32 * aq + lane;
+    const uint32_t tl = tmem + ((uint32_t)(32 * aq) << 16);
+    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o);
+    const bool vin = j0 + v < a.dv;
+    uint8_t *ot = sm + OFF_OST + (v >> 6) * 8192;
+    if (use_u && nk > 0 && !form_u(0)) ok = false;
+    for (int k = 0; ok && k < nk; ++k) {
+      if (use_u && k + 1 < nk && !form_u(k + 1)) { ok = false; break; }
+      if (!use_o) continue;
+      const int b = k & 1, c = cb + k, Cc = chunk_len(c);
+      const int tok0 = (int)(bos + (int64_t)c * C);
+      if (!group_wait(BAR_AUX, NAUX, bar(B_D1FULL0 + b), (k >> 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      float d[64];
+      tmem_ld32(tl + 256 * b + TM_D2, *reinterpret_cast<float(*)[32]>(&d[0]));
+      tmem_ld32(tl + 256 * b + TM_D2 + 32, *reinterpret_cast<float(*)[32]>(&d[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      if (atid == 0) bulk_wait_read();  // the previous chunk's store has read the staging tiles
+      group_sync(BAR_AUX, NAUX);
+      if (atid == 0) mbar_arrive(bar(B_OREAD0 + b));  // O^T of the buffer is in registers: free
+      if (Cc == C) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j)
+          *reinterpret_cast<__nv_bfloat16 *>(ot + sw128(j, v & 63)) = __float2bfloat16_rn(d[j]);
+        fence_proxy_async();
+        group_sync(BAR_AUX, NAUX);
+        if (atid == 0) {
           tma_store_3d(&tm_o, j0, h, tok0, sb + OFF_OST);
           if (j0 + 64 < a.dv) tma_store_3d(&tm_o, j0 + 64, h, tok0, sb + OFF_OST + 8192);
           bulk_commit();
-          bulk_wait_read();
         }
-        mbar_arrive(bar(B_OFREE));  // the staging buffer is free again
+      } else if (vin) {
+        __nv_bfloat16 *dst = o + ((size_t)tok0 * a.H + h) * (size_t)a.dv + j0 + v;
+#pragma unroll
+        for (int j = 0; j < 64; ++j)
+          if (j < Cc) dst[(size_t)j * a.H * a.dv] = __float2bfloat16_rn(d[j]);
       }
     }
+    if (atid == 0) bulk_wait_read();
   } else if (warp < NSTATE / 32) {
     // ---------------------------------------------------------- state side
     const int q4 = warp & 3, hf = warp >> 2;
@@ -970,7 +1056,6 @@ __global__ void __launch_bounds__(sp::NT, 1)
       for (int i = 0; i < 64; ++i)
         S[i] = ident ? (64 * hf + i == v ? 1.f : 0.f) : ((src && vin) ? src[base + (size_t)i * ld] : 0.f);
     }
-    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o);
     // S^T of the chunk about to start -> tensor memory buffer b (bf16 pairs); signals the issuer
     auto put_state = [&](int b) {
       uint32_t r[32];
@@ -986,20 +1071,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
       if (tid == 0) mbar_arrive(bar(B_SREADY));
     }
     for (int k = 0; k < nk; ++k) {
-      const int s = k & 1, b = k & 1, ph = (k >> 1) & 1, c = cb + k;
-      const int Cc = chunk_len(c);
-      const int tok0 = (int)(bos + (int64_t)c * C);
-      if (use_u && Cc < C) {  // the last chunk: the tile's rows past the sequence hold the next one's U
-        if (!group_wait(BAR_STATE, NSTATE, bar(B_FULL0 + s), ph)) { ok = false; break; }
-        uint8_t *ut = sm + s * STAGE + S_U;
-        for (int e = tid; e < 64 * 16; e += NSTATE) {
-          const int r = e >> 4, x = e & 15;
-          if (r >= Cc) st_s128(ut + (x >> 3) * 8192 + sw128(r, 8 * (x & 7)), make_uint4(0u, 0u, 0u, 0u));
-        }
-        fence_proxy_async();
-        group_sync(BAR_STATE, NSTATE);
-        if (tid == 0) mbar_arrive(bar(B_UZERO));
-      }
+      const int s = k & 1, b = k & 1, ph = (k >> 1) & 1;
       // ---------------------------------------------------------- S <- Diag(e^{g_C}) S + D1
       if (!group_wait(BAR_STATE, NSTATE, bar(B_D1FULL0 + b), ph)) { ok = false; break; }
       tc_fence_after();
@@ -1028,33 +1100,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
       if (tid == 0) {
         mbar_arrive(bar(B_D1FREE0 + b));
         if (k + 1 < nk) mbar_arrive(bar(B_SREADY));
-        if (!use_o) mbar_arrive(bar(B_OSTAGED0 + s));
       }
-      if (!use_o) continue;
-      // ---------------------------------------------------------- O: tokens 32 hf .. 32 hf + 31 of column v
-      if (!group_wait(BAR_STATE, NSTATE, bar(B_D2FULL0 + b), ph)) { ok = false; break; }
-      tc_fence_after();
-      {
-        float d[32];
-        tmem_ld32(tl + 256 * b + TM_D2 + 32 * hf, d);
-        tmem_wait_ld();
-        if (Cc == C) {  // staged for one TMA store per 64-column tile, once the previous store has read it
-          if (k >= 1 && !group_wait(BAR_STATE, NSTATE, bar(B_OFREE), (k - 1) & 1)) { ok = false; break; }
-          uint8_t *ot = sm + OFF_OST + (v >> 6) * 8192;
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            *reinterpret_cast<__nv_bfloat16 *>(ot + sw128(32 * hf + j, v & 63)) = __float2bfloat16_rn(d[j]);
-          fence_proxy_async();
-        } else if (vin) {
-          __nv_bfloat16 *dst = o + ((size_t)tok0 * a.H + h) * (size_t)a.dv + j0 + v;
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (32 * hf + j < Cc) dst[(size_t)(32 * hf + j) * a.H * a.dv] = __float2bfloat16_rn(d[j]);
-        }
-      }
-      tc_fence_before();
-      group_sync(BAR_STATE, NSTATE);
-      if (tid == 0) mbar_arrive(bar(B_OSTAGED0 + s));
     }
     // ---------------------------------------------------------- the state after this CTA's chunks
     if (ok && vin) {
@@ -1262,12 +1308,12 @@ int scan_segments(int B, int T, int H, int dv, bool packed, int sms, int *seg_le
   return (nch + len - 1) / len;
 }
 
-// Workspace layout: Mt tiles | Nt tiles | Qt tiles | Pt tiles | e^{g_C} | U (like v) | two-level scan
-// maps and entry states (long sequences only) | chunk offsets (packed only); 256-byte aligned arrays
+// Workspace layout: Mt tiles | Nt tiles | Qt tiles | Pt tiles | e^{g_C} | two-level scan maps and entry
+// states (long sequences only) | chunk offsets (packed only) | record counter; 256-byte aligned arrays
 struct WsLayout {
   long long records;
   int nseg, seg_len;
-  size_t m, n, q, p, g, u, sa, sbm, ss, coff, total;
+  size_t m, n, q, p, g, sa, sbm, ss, coff, cnt, total;
 };
 size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 WsLayout ws_layout(int B, int T, int H, int dv, bool packed, int sms) {
@@ -1275,19 +1321,18 @@ WsLayout ws_layout(int B, int T, int H, int dv, bool packed, int sms) {
   L.records = chunk_capacity(B, T, packed) * H;
   L.nseg = scan_segments(B, T, H, dv, packed, sms, &L.seg_len);
   const size_t r = (size_t)L.records;
-  const size_t tokens = packed ? (size_t)T : (size_t)B * T;
   const size_t pairs = (size_t)B * H, ns = L.nseg > 1 ? (size_t)L.nseg : 0;
   L.m = 0;
   L.n = L.m + r * REC_M;
   L.q = L.n + r * REC_N;
   L.p = L.q + r * REC_Q;
   L.g = L.p + r * REC_P;
-  L.u = up256(L.g + r * REC_G);
-  L.sa = up256(L.u + tokens * H * dv * 2);
+  L.sa = up256(L.g + r * REC_G);
   L.sbm = up256(L.sa + (ns ? pairs * (ns - 1) * DK * DK * 4 : 0));
   L.ss = up256(L.sbm + (ns ? pairs * (ns - 1) * DK * dv * 4 : 0));
   L.coff = up256(L.ss + pairs * ns * DK * dv * 4);
-  L.total = L.coff + (packed ? up256((size_t)(B + 1) * 4) : 0);
+  L.cnt = L.coff + (packed ? up256((size_t)(B + 1) * 4) : 0);
+  L.total = L.cnt + 256;
   return L;
 }
 
@@ -1312,20 +1357,21 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   WyParams p;
   cudaError_t err = device_status_word(&p.status);
   if (err != cudaSuccess) return err;
-  p.prefetch_stride = 2 * sms;
   p.N = a.B;
   p.nc = (a.T + C - 1) / C;
   p.tokens = tokens;
   p.coff = a.cu ? reinterpret_cast<const int32_t *>(base + L.coff) : nullptr;
   p.g = reinterpret_cast<float *>(base + L.g);
-  p.u = reinterpret_cast<__nv_bfloat16 *>(base + L.u);
+  p.nrec = (int)L.records;
+  p.reverse = a.cu ? 0 : 1;
+  p.next = reinterpret_cast<int *>(base + L.cnt);
 
-  CUtensorMap mq, mk, mb, mal, mv, mw, mu, mo, mm, mn, mqt, mp;
+  CUtensorMap mq, mk, mb, mal, mv, mw, mo, mm, mn, mqt, mp;
   if (tokens > 0) {
     if (!map_tokens(&mq, a.q, tokens, a.H, DK) || !map_tokens(&mk, a.k, tokens, a.H, DK) ||
         !map_tokens(&mb, a.b, tokens, a.H, DK) || !map_tokens(&mal, a.alpha, tokens, a.H, DK) ||
         !map_tokens(&mv, a.v, tokens, a.H, a.dv) || !map_tokens(&mw, a.w, tokens, a.H, a.dv) ||
-        !map_tokens(&mo, a.o, tokens, a.H, a.dv) || !map_tokens(&mu, base + L.u, tokens, a.H, a.dv) ||
+        !map_tokens(&mo, a.o, tokens, a.H, a.dv) ||
         !map_matrix(&mm, base + L.m, L.records * 128, 128, 128) ||
         !map_matrix(&mn, base + L.n, L.records * 128, 64, 128) ||
         !map_matrix(&mqt, base + L.q, L.records * 64, 128, 64) ||
@@ -1334,7 +1380,7 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   } else {
     // no token and no record: the state pass only copies S0 to S_T; its maps are never read
     memset(&mv, 0, sizeof(mv));
-    mw = mu = mo = mm = mn = mqt = mp = mv;
+    mw = mo = mm = mn = mqt = mp = mv;
   }
   if (a.cu) {
     note_launch();
@@ -1342,11 +1388,12 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   if (L.records > 0 && tokens > 0) {
+    if ((err = cudaMemsetAsync(p.next, 0, sizeof(int), stream)) != cudaSuccess) return err;
     err = cudaFuncSetAttribute(wy_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wy::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     note_launch();
-    wy_factor_kernel<<<(unsigned)L.records, wy::NT, wy::SMEM_BYTES, stream>>>(a, p, mq, mk, mb, mal, mm, mn, mqt, mp, mv,
-                                                                              mw);
+    const long long grid = L.records < 2LL * sms ? L.records : 2LL * sms;  // persistent: two CTAs per SM
+    wy_factor_kernel<<<(unsigned)grid, wy::NT, wy::SMEM_BYTES, stream>>>(a, p, mq, mk, mb, mal, mm, mn, mqt, mp);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   const long long tiles = (a.dv + sp::VW - 1) / sp::VW;
@@ -1355,7 +1402,7 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   ScanParams q{};
   if (L.nseg <= 1) {  // one walk per (sequence, head, value tile)
     note_launch();
-    state_pass_kernel<<<(unsigned)(a.B * a.H * tiles), sp::NT, sp::SMEM_BYTES, stream>>>(a, p, q, mm, mn, mqt, mp, mu, mo);
+    state_pass_kernel<<<(unsigned)(a.B * a.H * tiles), sp::NT, sp::SMEM_BYTES, stream>>>(a, p, q, mm, mn, mqt, mp, mv, mw, mo);
     return cudaGetLastError();
   }
   // two-level scan: segment maps, their chain into entry states, then the segments' walks
@@ -1367,7 +1414,7 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   q.mode = 1;
   note_launch();
   state_pass_kernel<<<(unsigned)(a.B * a.H * (L.nseg - 1) * (1 + tiles)), sp::NT, sp::SMEM_BYTES, stream>>>(
-      a, p, q, mm, mn, mqt, mp, mu, mo);
+      a, p, q, mm, mn, mqt, mp, mv, mw, mo);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const int chain_smem = (128 * 132 + 32 * 132) * 4;
   err = cudaFuncSetAttribute(segment_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, chain_smem);
@@ -1378,7 +1425,7 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   q.mode = 2;
   note_launch();
   state_pass_kernel<<<(unsigned)(a.B * a.H * L.nseg * tiles), sp::NT, sp::SMEM_BYTES, stream>>>(a, p, q, mm, mn, mqt,
-                                                                                                  mp, mu, mo);
+                                                                                                  mp, mv, mw, mo);
   return cudaGetLastError();
 }
 
