@@ -14,6 +14,8 @@ Entry points (same names as the C ABI):
   (``gdn2_chunk_bwd``);
 * :func:`decode_step` -- one recurrent step for a batch of single tokens
   (``gdn2_decode_step``);
+* :func:`recurrent_fwd` -- the token loop over whole sequences in either erase orientation
+  (``gdn2_recurrent_fwd``);
 * :func:`block_prologue`, :func:`block_epilogue` -- the work around the mixer
   in its block (``gdn2_block_prologue``, ``gdn2_block_epilogue``).
 """
@@ -27,6 +29,7 @@ LIB_PATH = os.path.join(_PKG, "_build", "libgdn2.so")
 
 GDN2_OK, GDN2_ERR_INVALID_ARG, GDN2_ERR_UNSUPPORTED, GDN2_ERR_CUDA, GDN2_ERR_TIMEOUT = range(5)
 GDN2_F32, GDN2_BF16 = 0, 1
+GDN2_ERASE_R1, GDN2_ERASE_R2 = 0, 1
 _DTYPES = {torch.float32: GDN2_F32, torch.bfloat16: GDN2_BF16}
 
 _lib = None
@@ -67,6 +70,8 @@ def lib():
         L.gdn2_chunk_fwd_workspace_bytes.argtypes = [ci] * 7 + [ci]
         L.gdn2_chunk_fwd_workspace_bytes.restype = ctypes.c_size_t
         L.gdn2_launch_count.restype = ctypes.c_uint64
+        L.gdn2_recurrent_fwd.argtypes = [vp] * 9 + [ci] * 5 + [vp, ci, ci, vp]
+        L.gdn2_recurrent_fwd.restype = ci
         L.gdn2_chunk_bwd.argtypes = [vp] * 16 + [ci] * 5 + [vp, ci, vp]
         L.gdn2_chunk_bwd.restype = ci
         L.gdn2_chunk_bwd_workspace_bytes.argtypes = [ci] * 6
@@ -175,6 +180,38 @@ def chunk_fwd_noalloc(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, chunk=64, 
 
 
 NOALLOC_WORKSPACE_BYTES = 64 << 20  # GDN2_NOALLOC_WORKSPACE_BYTES in include/gdn2.h
+
+
+def recurrent_fwd(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, erase=GDN2_ERASE_R1, o=None, S_T=None,
+                  output_final_state=True, stream=None):
+    """Token-by-token forward in either erase orientation (``GDN2_ERASE_R1`` or ``GDN2_ERASE_R2``).
+
+    Same layouts and returns as :func:`chunk_fwd`; see ``gdn2_recurrent_fwd`` in ``include/gdn2.h``.
+    """
+    if cu_seqlens is None:
+        B, T, H, dk = q.shape
+    else:
+        if cu_seqlens.dtype != torch.int32:
+            raise ValueError("gdn2: cu_seqlens must be int32")
+        B = cu_seqlens.numel() - 1
+        T, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype not in _DTYPES or any(x.dtype != q.dtype for x in (k, v, alpha, b, w)):
+        raise ValueError("gdn2: q, k, v, alpha, b, w must share dtype float32 or bfloat16")
+    if o is None:
+        o = torch.empty(q.shape[:-1] + (dv,), dtype=q.dtype, device=q.device)
+    if S_T is None and output_final_state:
+        S_T = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    if S0 is not None and S0.dtype != torch.float32:
+        raise ValueError("gdn2: S0 must be float32")
+    _check_tensors(q, k, v, alpha, b, w, S0, o, S_T, cu_seqlens)
+    with torch.cuda.device(q.device):
+        st = lib().gdn2_recurrent_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
+                                      _ptr(S_T), B, T, H, dk, dv, _ptr(cu_seqlens), int(erase), _DTYPES[q.dtype],
+                                      _stream(stream, q.device))
+    if st != GDN2_OK:
+        raise Gdn2Error(st, "gdn2_recurrent_fwd")
+    return o, S_T
 
 
 def chunk_bwd(q, k, v, alpha, b, w, dO, S0=None, dS_T=None, cu_seqlens=None, want_dS0=True, stream=None):

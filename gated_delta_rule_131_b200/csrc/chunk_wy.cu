@@ -325,6 +325,7 @@ __global__ void __launch_bounds__(wy::NT, 2)
   // every thread has passed the barrier that follows its read)
   volatile int *s_next = reinterpret_cast<volatile int *>(sm + OFF_BAR + 20);
 
+  bool pre = false;  // this record's input loads were issued by the previous record's epilogue
   for (int it = blockIdx.x, nit = 0, par = 0; it < p.nrec; it = nit, par ^= 1) {
     const int rec = wy_record(p, a.H, it);
     const int h = rec % a.H;
@@ -339,29 +340,30 @@ __global__ void __launch_bounds__(wy::NT, 2)
     seq_span(a, n, bos, len);
     const int Cc = min(C, len - c * C);
 
+    // the next record of this CTA, whose loads this record's epilogue issues when it is a real one
+    int nn = 0, ncc = 0;
+    const int nrec_ = nit < p.nrec ? wy_record(p, a.H, nit) : 0;
+    const int ntok = nit < p.nrec ? wy_tok0(a, p, nrec_, &nn, &ncc) : -1;
     if (tid == 0) {
-      bulk_wait_read();  // the previous record's stores have read the tiles these loads overwrite
-      mbar_expect_tx(bar_full, TMA_BYTES);
+      bulk_wait_read();  // the previous record's stores have read their tiles (TP and TS are reused below)
+      if (!pre) {
+        mbar_expect_tx(bar_full, TMA_BYTES);
 #pragma unroll
-      for (int blk = 0; blk < 2; ++blk) {
-        tma_load_3d(sb + OFF_XA + blk * XA_BLK, &tm_b, 64 * blk, h, tok0, bar_full);         // b -> rows 0..63
-        tma_load_3d(sb + OFF_XA + blk * XA_BLK + 8192, &tm_q, 64 * blk, h, tok0, bar_full);  // q -> rows 64..127
-        tma_load_3d(sb + OFF_KT + blk * KT_BLK, &tm_k, 64 * blk, h, tok0, bar_full);
-        tma_load_3d(sb + OFF_AL + blk * 8192, &tm_al, 64 * blk, h, tok0, bar_full);
+        for (int blk = 0; blk < 2; ++blk) {
+          tma_load_3d(sb + OFF_XA + blk * XA_BLK, &tm_b, 64 * blk, h, tok0, bar_full);         // b -> rows 0..63
+          tma_load_3d(sb + OFF_XA + blk * XA_BLK + 8192, &tm_q, 64 * blk, h, tok0, bar_full);  // q -> rows 64..127
+          tma_load_3d(sb + OFF_KT + blk * KT_BLK, &tm_k, 64 * blk, h, tok0, bar_full);
+          tma_load_3d(sb + OFF_AL + blk * 8192, &tm_al, 64 * blk, h, tok0, bar_full);
+        }
       }
       // this CTA's next record into L2, so that its loads come from there
-      if (nit < p.nrec) {
-        const int nrec = wy_record(p, a.H, nit);
-        int nn, ncc;
-        const int ntok = wy_tok0(a, p, nrec, &nn, &ncc);
-        if (ntok >= 0) {
+      if (ntok >= 0) {
 #pragma unroll
-          for (int blk = 0; blk < 2; ++blk) {
-            tma_prefetch_3d(&tm_b, 64 * blk, nrec % a.H, ntok);
-            tma_prefetch_3d(&tm_q, 64 * blk, nrec % a.H, ntok);
-            tma_prefetch_3d(&tm_k, 64 * blk, nrec % a.H, ntok);
-            tma_prefetch_3d(&tm_al, 64 * blk, nrec % a.H, ntok);
-          }
+        for (int blk = 0; blk < 2; ++blk) {
+          tma_prefetch_3d(&tm_b, 64 * blk, nrec_ % a.H, ntok);
+          tma_prefetch_3d(&tm_q, 64 * blk, nrec_ % a.H, ntok);
+          tma_prefetch_3d(&tm_k, 64 * blk, nrec_ % a.H, ntok);
+          tma_prefetch_3d(&tm_al, 64 * blk, nrec_ % a.H, ntok);
         }
       }
     }
@@ -369,13 +371,13 @@ __global__ void __launch_bounds__(wy::NT, 2)
     // ------------------------------------------------------------ decay factors, operands in place
     if (!mbar_wait_bounded(bar_full, nfull & 1, WAIT_NS)) ok = false;
     ++nfull;
+    if (__syncthreads_or(!ok)) goto done;
     // the never-written blocks (0,1) and (2,3) of T, which the 32x32 merges read (the region held the
-    // previous record's Pt, whose store has read it)
+    // previous record's Mt tile 1, whose store has read it)
     for (int e = tid; e < 512; e += NT) {
       const int R = 2 * (e >> 8), r = (e >> 4) & 15, j = e & 15;
       Ts[(16 * R + r) * LDF + 16 * (R + 1) + j] = 0.f;
     }
-    if (__syncthreads_or(!ok)) goto done;
     {
       // thread = 8 key channels (chunk x8 of channel block cb) x 4 tokens (group G = rows 4G..4G+3);
       // groups 0-7 hold tokens 0..31 (walk back to token 31), groups 8-15 tokens 32..63 (walk forward)
@@ -385,6 +387,7 @@ __global__ void __launch_bounds__(wy::NT, 2)
       for (int i = 0; i < 4; ++i) {
         const uint32_t o = sw128(4 * G + i, 8 * x8);
         ra[i] = ld_s128(sm + OFF_AL + cb * 8192 + o);
+        if (64 * cb >= a.dk) ra[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);  // bf16 1.0
         rb[i] = ld_s128(sm + OFF_XA + cb * XA_BLK + o);
         rq[i] = ld_s128(sm + OFF_XA + cb * XA_BLK + 8192 + o);
         rk[i] = ld_s128(sm + OFF_KT + cb * KT_BLK + o);
@@ -647,17 +650,34 @@ __global__ void __launch_bounds__(wy::NT, 2)
                  sdesc_sw128(sb + OFF_XA + 2048 * k, XA_BLK, 1024), ID_KM128, k > 0 ? 1u : 0u);
       }
       mma_commit(bar_mma);
+      // Nt and Pt: their stores have read the tiles before any thread passes the barrier below
+      // (the epilogue writes Mt into them)
+      bulk_wait_read();
     }
     if (!mbar_wait_bounded(bar_mma, nmma & 1, WAIT_NS)) ok = false;
     ++nmma;
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
+    // K_m and W' are dead now: the next record's k and alpha go into their tiles while this record's
+    // epilogue runs (its q and b follow once Q_m is read and Qt has been stored)
+    pre = ntok >= 0;
+    if (tid == 0) {
+      if (pre) {
+        mbar_expect_tx(bar_full, TMA_BYTES);
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk) {
+          tma_load_3d(sb + OFF_KT + blk * KT_BLK, &tm_k, 64 * blk, nrec_ % a.H, ntok, bar_full);
+          tma_load_3d(sb + OFF_AL + blk * 8192, &tm_al, 64 * blk, nrec_ % a.H, ntok, bar_full);
+        }
+      }
+    }
     {
       const int row = 32 * quad + lane;
-      {  // Mt = Diag(e^{g_C-m}) K_m^T W': row = key channel, input channels 64 khalf .. +63
+      // Mt = Diag(e^{g_C-m}) K_m^T W': row = key channel, input channels 64 khalf .. +63 -> TP / TS
+      auto mt_epilogue = [&]() {
         const float g2 = s_egcm[row];
         const float g2p[2] = {g2, g2};
-        uint8_t *dst = sm + (khalf ? OFF_AL : OFF_KT);
+        uint8_t *dst = sm + (khalf ? OFF_TS : OFF_TP);
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
           float v[32];
@@ -668,8 +688,8 @@ __global__ void __launch_bounds__(wy::NT, 2)
 #pragma unroll
           for (int y = 0; y < 4; ++y) st_s128(dst + sw128(row, 32 * part + 8 * y), pack8(&v[8 * y]));
         }
-      }
-      if (quad < 2) {  // Qt = (Q_m - Pt A_m) Diag(e^m) in place of A_m, channel block khalf
+      };
+      if (quad < 2) {  // Qt = (Q_m - Pt A_m) Diag(e^m) in place of A_m, channel block khalf (warps 0, 1, 4, 5)
         uint8_t *blk = sm + OFF_XA + khalf * XA_BLK;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
@@ -691,19 +711,36 @@ __global__ void __launch_bounds__(wy::NT, 2)
             st_s128(blk + sw128(row, col), pack8(e));
           }
         }
+        fence_proxy_async();
+        group_sync(1, 128);  // the four Qt warps: every Qt tile written, every Q_m row read
+        if (tid == 0) {      // Qt -> workspace; the next record's q into the dead Q_m rows
+          tma_store_2d(&tm_wq, 0, rec * 64, sb + OFF_XA);
+          tma_store_2d(&tm_wq, 64, rec * 64, sb + OFF_XA + XA_BLK);
+          bulk_commit();
+          if (pre) {
+#pragma unroll
+            for (int blk2 = 0; blk2 < 2; ++blk2)
+              tma_load_3d(sb + OFF_XA + blk2 * XA_BLK + 8192, &tm_q, 64 * blk2, nrec_ % a.H, ntok, bar_full);
+          }
+        }
       }
+      mt_epilogue();
     }
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
 
-    // ------------------------------------------------------------ the record -> workspace (waited for at the next record)
+    // ------------------------------------------------------------ Mt -> workspace (waited for at the next record)
     if (tid == 0) {
-      tma_store_2d(&tm_wm, 0, rec * 128, sb + OFF_KT);
-      tma_store_2d(&tm_wm, 64, rec * 128, sb + OFF_AL);
-      tma_store_2d(&tm_wq, 0, rec * 64, sb + OFF_XA);
-      tma_store_2d(&tm_wq, 64, rec * 64, sb + OFF_XA + XA_BLK);
+      tma_store_2d(&tm_wm, 0, rec * 128, sb + OFF_TP);
+      tma_store_2d(&tm_wm, 64, rec * 128, sb + OFF_TS);
       bulk_commit();
+      if (pre) {  // the next record's b into the rows Qt leaves, once its store has read them
+        asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk)
+          tma_load_3d(sb + OFF_XA + blk * XA_BLK, &tm_b, 64 * blk, nrec_ % a.H, ntok, bar_full);
+      }
     }
   }
 
@@ -972,18 +1009,28 @@ __global__ void __launch_bounds__(sp::NT, 1)
       const int Cc = chunk_len(cb + k);
       uint8_t *vt = sm + s * STAGE + S_V, *wt = sm + s * STAGE + S_W;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {  // pieces: 64 rows x (2 tiles x 8)
-        const int e = atid + NAUX * i, r = e >> 4, x = e & 15;
-        const uint32_t off = (uint32_t)(x >> 3) * 8192u + sw128(r, 8 * (x & 7));
-        uint4 u = make_uint4(0u, 0u, 0u, 0u);
-        if (r < Cc) {  // bf16 x bf16 is exact in fp32: the packed product is the rounded one
-          const uint4 vv = ld_s128(vt + off), ww = ld_s128(wt + off);
-          u.x = bf2_mul(vv.x, ww.x);
-          u.y = bf2_mul(vv.y, ww.y);
-          u.z = bf2_mul(vv.z, ww.z);
-          u.w = bf2_mul(vv.w, ww.w);
+      for (int half = 0; half < 2; ++half) {  // pieces: 64 rows x (2 tiles x 8); four loaded, then four stored
+        uint4 vv[4], ww[4];
+        uint32_t off[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int e = atid + NAUX * (4 * half + i), r = e >> 4, x = e & 15;
+          off[i] = (uint32_t)(x >> 3) * 8192u + sw128(r, 8 * (x & 7));
+          vv[i] = ld_s128(vt + off[i]);
+          ww[i] = ld_s128(wt + off[i]);
         }
-        st_s128(vt + off, u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {  // bf16 x bf16 is exact in fp32: the packed product is the rounded one
+          const int r = (atid + NAUX * (4 * half + i)) >> 4;
+          uint4 u = make_uint4(0u, 0u, 0u, 0u);
+          if (r < Cc) {
+            u.x = bf2_mul(vv[i].x, ww[i].x);
+            u.y = bf2_mul(vv[i].y, ww[i].y);
+            u.z = bf2_mul(vv[i].z, ww[i].z);
+            u.w = bf2_mul(vv[i].w, ww[i].w);
+          }
+          st_s128(vt + off[i], u);
+        }
       }
       fence_proxy_async();
       group_sync(BAR_AUX, NAUX);
@@ -1040,8 +1087,10 @@ __global__ void __launch_bounds__(sp::NT, 1)
     const bool vin = j0 + v < cols;
     const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
     const size_t nh = (size_t)n * a.H + h;
-    // S[64 hf + i][j0 + v] lives at base + i * cols in every [.., 128, cols] state array
-    const size_t s_base = (nh * DK + 64 * hf) * (size_t)a.dv + j0 + v;
+    // S[64 hf + i][j0 + v] lives at base + i * cols in every [.., d_k, cols] state array (the caller's
+    // S0 and S_T have d_k rows; with d_k = 64 the rows 64..127 the kernels carry stay zero)
+    const bool kin = 64 * hf < a.dk;
+    const size_t s_base = (nh * a.dk + 64 * hf) * (size_t)a.dv + j0 + v;
     float S[64];
     {
       const float *src = nullptr;
@@ -1049,7 +1098,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
       if (q.mode == 2) {  // every segment, the first included, starts from its entry state (S_T may alias S0)
         src = q.s_start;
         base = ((nh * q.nseg + seg) * DK + 64 * hf) * (size_t)a.dv + j0 + v;
-      } else if (!ident && seg == 0) {
+      } else if (!ident && seg == 0 && kin) {
         src = a.S0;
       }
 #pragma unroll
@@ -1110,7 +1159,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
         const size_t js = nh * (q.nseg - 1) + seg;
         dst = ident ? q.sum_a : q.sum_b;
         base = (js * DK + 64 * hf) * (size_t)cols + j0 + v;
-      } else if (q.mode == 0 || seg == q.nseg - 1) {
+      } else if ((q.mode == 0 || seg == q.nseg - 1) && kin) {
         dst = a.ST;
       }
       if (dst) {
@@ -1143,7 +1192,8 @@ __global__ void __launch_bounds__(256) segment_chain_kernel(const ChunkArgs a, c
   for (int e = tid; e < 128 * 128; e += 256) {  // E_0 = S0 (zeros without one)
     const int i = e >> 7, v = e & 127;
     if (v < cols)
-      q.s_start[((nh * q.nseg) * DK + i) * (size_t)a.dv + j0 + v] = a.S0 ? a.S0[(nh * DK + i) * (size_t)a.dv + j0 + v] : 0.f;
+      q.s_start[((nh * q.nseg) * DK + i) * (size_t)a.dv + j0 + v] =
+          (a.S0 && i < a.dk) ? a.S0[(nh * a.dk + i) * (size_t)a.dv + j0 + v] : 0.f;
   }
   // E_1 = B_0
   for (int e = tid; e < 128 * 128; e += 256) {
@@ -1339,7 +1389,7 @@ WsLayout ws_layout(int B, int T, int H, int dv, bool packed, int sms) {
 }  // namespace
 
 bool chunk_wy_supported(int B, int T, int H, int dk, int dv, bool packed, bool bf16) {
-  if (!bf16 || dk != DK || dv % NV != 0) return false;
+  if (!bf16 || (dk != 64 && dk != DK) || dv % NV != 0) return false;
   // TMA coordinates are int32: token rows (plus one chunk) and workspace rows (records x 128)
   const long long tokens = packed ? (long long)T : (long long)B * T;
   return tokens + C <= (long long)INT_MAX && chunk_capacity(B, T, packed) * H * 128 <= (long long)INT_MAX;
@@ -1368,8 +1418,10 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
 
   CUtensorMap mq, mk, mb, mal, mv, mw, mo, mm, mn, mqt, mp;
   if (tokens > 0) {
-    if (!map_tokens(&mq, a.q, tokens, a.H, DK) || !map_tokens(&mk, a.k, tokens, a.H, DK) ||
-        !map_tokens(&mb, a.b, tokens, a.H, DK) || !map_tokens(&mal, a.alpha, tokens, a.H, DK) ||
+    // key-side maps have the caller's d_k channels: with d_k = 64 the second 64-channel box is
+    // outside the tensor and arrives as zeros
+    if (!map_tokens(&mq, a.q, tokens, a.H, a.dk) || !map_tokens(&mk, a.k, tokens, a.H, a.dk) ||
+        !map_tokens(&mb, a.b, tokens, a.H, a.dk) || !map_tokens(&mal, a.alpha, tokens, a.H, a.dk) ||
         !map_tokens(&mv, a.v, tokens, a.H, a.dv) || !map_tokens(&mw, a.w, tokens, a.H, a.dv) ||
         !map_tokens(&mo, a.o, tokens, a.H, a.dv) ||
         !map_matrix(&mm, base + L.m, L.records * 128, 128, 128) ||

@@ -17,6 +17,16 @@ struct ChunkArgs {
   int B, T, H, dk, dv;
 };
 
+// Arguments of one gdn2_recurrent_fwd call (validated by the API layer); layouts as ChunkArgs.
+struct RecurrentArgs {
+  const void *q, *k, *v, *alpha, *b, *w;
+  const float *S0;
+  void *o;
+  float *ST;
+  const int32_t *cu;  // device offsets [B+1] or nullptr
+  int B, T, H, dk, dv;
+};
+
 // Arguments of one gdn2_decode_step call.
 struct DecodeArgs {
   const void *q, *k, *v, *alpha, *b, *w;
@@ -99,6 +109,8 @@ cudaError_t read_device_status(int *status, bool reset);
 // Device address of that word, for kernels compiled in other files.
 cudaError_t device_status_word(int **ptr);
 cudaError_t launch_decode(const DecodeArgs &a, bool bf16, cudaStream_t stream);
+// Token-loop forward over whole sequences; r2 selects the second erase orientation.
+cudaError_t launch_recurrent(const RecurrentArgs &a, bool bf16, bool r2, cudaStream_t stream);
 cudaError_t launch_block_prologue(const BlockPrologueArgs &p, bool bf16, cudaStream_t stream);
 cudaError_t launch_block_epilogue(const BlockEpilogueArgs &p, bool bf16, cudaStream_t stream);
 

@@ -163,8 +163,8 @@ gdn2_status check_chunk(const void *q, const void *k, const void *v, const void 
   if (!fits(tokens, H, d_v > d_k ? d_v : d_k, 1) || !fits(B, H, d_k, d_v)) return GDN2_ERR_INVALID_ARG;
   if ((long long)B * H * 8 > INT_MAX) return GDN2_ERR_INVALID_ARG;
   *a = gdn2::ChunkArgs{q, k, v, alpha, b, w, S0, o, S_T, cu_seqlens, B, T, H, d_k, d_v};
-  // bf16 with d_k = 128 runs on the tensor cores; fp32 (whose accuracy bf16 operands cannot
-  // keep) and d_k = 64 run the SIMT kernel
+  // bf16 runs on the tensor cores; fp32 (whose accuracy bf16 operands cannot keep) runs the SIMT
+  // kernel
   *tc = gdn2::chunk_wy_supported(B, T, H, d_k, d_v, cu_seqlens != nullptr, dtype == GDN2_BF16);
   return GDN2_OK;
 }
@@ -230,6 +230,21 @@ gdn2_status gdn2_chunk_bwd(const void *q, const void *k, const void *v, const vo
   const gdn2::BwdArgs a{q, k, v, alpha, b, w, dO, S0, dS_T, dq, dk, dv, dalpha, db, dw, dS0, cu_seqlens,
                         B, T, H, d_k, d_v};
   const cudaError_t err = run_chunk_bwd(a, dtype == GDN2_BF16, (cudaStream_t)stream);
+  return err == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+}
+
+gdn2_status gdn2_recurrent_fwd(const void *q, const void *k, const void *v, const void *alpha, const void *b,
+                               const void *w, const float *S0, void *o, float *S_T, int B, int T, int H, int d_k,
+                               int d_v, const int32_t *cu_seqlens, gdn2_erase erase, gdn2_dtype dtype,
+                               gdn2_stream_t stream) {
+  if (erase != GDN2_ERASE_R1 && erase != GDN2_ERASE_R2) return GDN2_ERR_INVALID_ARG;
+  gdn2::ChunkArgs c;
+  bool tc = false;
+  // the same arguments, layouts and checks as gdn2_chunk_fwd (chunk length 64 stands in: it is unused)
+  const gdn2_status st = check_chunk(q, k, v, alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, 64, cu_seqlens, dtype, &c, &tc);
+  if (st != GDN2_OK || B == 0) return st;
+  const gdn2::RecurrentArgs a{q, k, v, alpha, b, w, S0, o, S_T, cu_seqlens, B, T, H, d_k, d_v};
+  const cudaError_t err = gdn2::launch_recurrent(a, dtype == GDN2_BF16, erase == GDN2_ERASE_R2, (cudaStream_t)stream);
   return err == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
 }
 

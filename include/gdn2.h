@@ -95,11 +95,12 @@ typedef struct CUstream_st *gdn2_stream_t;
  * chunk: 64 (the only supported chunk length).
  * T == 0 (or an empty sequence) is valid: its S_T equals its S0; when the
  * batch holds no token at all, the token pointers (q .. w, o) may be NULL.
- * bf16 with d_k = 128 runs two tensor-core kernels over a workspace: the first
- * forms the chunk's WY factors (T = (I + L)^-1, W = -T A, and the decay-
+ * bf16 (d_k = 64 or 128) runs two tensor-core kernels over a workspace: the
+ * first forms the chunk's WY factors (T = (I + L)^-1, W = -T A, and the decay-
  * absorbed q and k) for every chunk at once, the second carries the state
- * through each sequence's chunks in order; other shapes and fp32 run one SIMT
- * kernel without a workspace.
+ * through each sequence's chunks in order (d_k = 64 is carried as 128 key
+ * channels whose upper half stays zero); fp32 runs one SIMT kernel without a
+ * workspace (bf16 tensor-core operands cannot keep the fp32 tolerance).
  * Returns GDN2_OK, or an error status with nothing launched; GDN2_ERR_CUDA
  * also when the workspace cannot be allocated.
  */
@@ -121,7 +122,7 @@ GDN2_API gdn2_status gdn2_chunk_fwd(const void *q, const void *k, const void *v,
  *   - Set-up: the first call on a device, with that device current, looks the array's device
  *     address up (cudaGetSymbolAddress) and keeps it; make that first call before any stream
  *     capture.  Later calls on the device reuse the address.
- *   - Limit: a tensor-core call (bf16, d_k = 128) whose workspace, gdn2_chunk_fwd_workspace_bytes()
+ *   - Limit: a tensor-core call (bf16) whose workspace, gdn2_chunk_fwd_workspace_bytes()
  *     for this shape on the current device, exceeds the array returns GDN2_ERR_UNSUPPORTED before
  *     any launch or allocation.  That size depends on the device's SM count (the number of segments
  *     of the two-level state scan), so a shape near the limit may fit on one device and not on
@@ -144,6 +145,31 @@ GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const void *q, const void *k, const 
  */
 GDN2_API size_t gdn2_chunk_fwd_workspace_bytes(int B, int T, int H, int d_k, int d_v, int chunk, int packed,
                                                gdn2_dtype dtype);
+
+/*
+ * gdn2_recurrent_fwd -- the token-by-token recurrence over whole sequences, in either reading of
+ * the erase orientation.
+ *
+ * The pages state the erase in words only: b_t gates the erase per key channel ("NVIDIA AIが
+ * Gated DeltaNet-2を発表", ai.warp-studio.com, "Gated DeltaNet-2の核心"; "[논문] 게이트형 DeltaNet-2",
+ * euno.news, "방법론", step 2), which leaves open on which side of the rank-1 erase the gate sits:
+ *   GDN2_ERASE_R1:  S_t = (I - k_t (b_t (.) k_t)^T) Diag(alpha_t) S_{t-1} + k_t (w_t (.) v_t)^T
+ *                   (the reading every other call of this library computes)
+ *   GDN2_ERASE_R2:  S_t = (I - (b_t (.) k_t) k_t^T) Diag(alpha_t) S_{t-1} + k_t (w_t (.) v_t)^T
+ * and o_t = S_t^T q_t in both.  Both reduce to KDA when b_t = w_t = one scalar and to Gated
+ * DeltaNet when alpha_t is a scalar as well.
+ *
+ * Arguments, layouts (dense or packed with cu_seqlens), aliasing, supported head sizes and errors
+ * are those of gdn2_chunk_fwd (without `chunk`); erase is GDN2_ERASE_R1 or GDN2_ERASE_R2, anything
+ * else is GDN2_ERR_INVALID_ARG.  fp32 arithmetic and state; o is rounded to dtype once.  It walks
+ * the tokens of each sequence in order in one kernel (one CTA per sequence, head and 64 value
+ * columns), so it costs time linear in the longest sequence; it allocates nothing.
+ */
+typedef enum { GDN2_ERASE_R1 = 0, GDN2_ERASE_R2 = 1 } gdn2_erase;
+GDN2_API gdn2_status gdn2_recurrent_fwd(const void *q, const void *k, const void *v, const void *alpha,
+                                        const void *b, const void *w, const float *S0, void *o, float *S_T,
+                                        int B, int T, int H, int d_k, int d_v, const int32_t *cu_seqlens,
+                                        gdn2_erase erase, gdn2_dtype dtype, gdn2_stream_t stream);
 
 /*
  * gdn2_chunk_bwd -- gradients of a loss L through gdn2_chunk_fwd (erase reading R1).

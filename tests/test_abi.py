@@ -231,6 +231,32 @@ def test_chunk_workspace_layout(L):
     extra = n - 16384 * record - 256
     assert extra > 0 and extra % (16 * 65536) == 0 and (extra // (16 * 65536) + 2) % 3 == 0
     assert (extra // (16 * 65536) + 2) // 3 >= 2
-    # fp32 and d_k = 64 run the SIMT kernel, which needs no workspace
+    # fp32 runs the SIMT kernel, which needs no workspace; bf16 with d_k = 64 runs the tensor-core
+    # path with the same 128-channel records
     assert L.gdn2_chunk_fwd_workspace_bytes(4, 2048, 16, 128, 128, 64, 0, gdn2.GDN2_F32) == 0
-    assert L.gdn2_chunk_fwd_workspace_bytes(4, 2048, 16, 64, 128, 64, 0, gdn2.GDN2_BF16) == 0
+    assert L.gdn2_chunk_fwd_workspace_bytes(4, 2048, 16, 64, 128, 64, 0, gdn2.GDN2_BF16) == 2048 * record + 256
+
+
+def recurrent(L, ptrs=None, B=1, T=64, H=1, dk=64, dv=64, cu=None, erase=gdn2.GDN2_ERASE_R2, dtype=gdn2.GDN2_BF16):
+    p = ptrs or [FAKE] * 9
+    return L.gdn2_recurrent_fwd(*p, B, T, H, dk, dv, cu, erase, dtype, None)
+
+
+def test_recurrent_validation(L):
+    before = L.gdn2_launch_count()
+    assert recurrent(L, erase=2) == gdn2.GDN2_ERR_INVALID_ARG
+    assert recurrent(L, erase=-1) == gdn2.GDN2_ERR_INVALID_ARG
+    assert recurrent(L, dk=96) == gdn2.GDN2_ERR_UNSUPPORTED
+    assert recurrent(L, dv=32) == gdn2.GDN2_ERR_UNSUPPORTED
+    assert recurrent(L, dtype=7) == gdn2.GDN2_ERR_INVALID_ARG
+    assert recurrent(L, B=-1) == gdn2.GDN2_ERR_INVALID_ARG
+    for i in range(9):
+        if i in (6, 8):  # S0, S_T may be NULL
+            continue
+        p = [FAKE] * 9
+        p[i] = None
+        assert recurrent(L, p) == gdn2.GDN2_ERR_INVALID_ARG, i
+        p[i] = MIS
+        assert recurrent(L, p) == gdn2.GDN2_ERR_INVALID_ARG, i
+    assert recurrent(L, [None] * 9, B=0, T=0) == gdn2.GDN2_OK
+    assert L.gdn2_launch_count() == before

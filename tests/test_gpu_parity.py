@@ -229,3 +229,28 @@ def test_two_level_scan_zero_state_and_aliased_final_state(g):
     o_ref2, S_ref2 = oracle.recurrent(*[np64(d[n]) for n in TOK], S0=np64(d["S0"]))
     check_bf16(np64(o2), o_ref2, "o")
     check_bf16(S.cpu().double().numpy(), S_ref2, "aliased S_T")
+
+
+# ------------------------------------------------------------------ d_k = 64 on the tensor-core path
+# bf16 with d_k = 64 runs the same two tensor-core kernels as d_k = 128 (its second 64-channel block
+# arrives as zeros and the state rows it would carry stay zero); the workspace size and the launch
+# count show that the tensor-core path ran, not the SIMT kernel.
+
+@pytest.mark.parametrize("dv", [64, 128, 256])
+def test_dk64_bf16_tensor_core_path(g, dv):
+    wl = W.Workload("dk64_tc", B=2, T=333, H=3, dk=64, dv=dv)
+    assert g.chunk_fwd_workspace_bytes(wl.B, wl.T, wl.H, wl.dk, wl.dv) > 0
+    c0 = g.launch_count()
+    run_case(g, wl, seed=51)
+    assert g.launch_count() - c0 == 2  # the WY kernel and the state pass
+
+
+def test_dk64_bf16_packed_and_two_level_scan(g):
+    lengths = [1, 63, 64, 65, 0, 128, 129, 200]
+    wl = W.Workload("dk64_packed", B=len(lengths), T=256, H=2, dk=64, dv=128, varlen=True)
+    assert g.chunk_fwd_workspace_bytes(len(lengths), sum(lengths), wl.H, wl.dk, wl.dv, packed=True) > 0
+    run_case(g, wl, seed=52, lengths=lengths)
+    wl = W.Workload("dk64_scan", B=1, T=2600, H=2, dk=64, dv=128)
+    c0 = g.launch_count()
+    run_case(g, wl, seed=53)
+    assert g.launch_count() - c0 == 4  # WY, segment maps, their chain, the segments' walks
