@@ -119,6 +119,11 @@ __device__ __forceinline__ bool group_wait(int id, int count, uint32_t bar, uint
   const bool ok = mbar_wait_bounded(bar, parity, WAIT_NS);
   return !group_or(id, count, fail || !ok);
 }
+// The same, polling without suspending (the state chain's wait on its products).
+__device__ __forceinline__ bool group_wait_spin(int id, int count, uint32_t bar, uint32_t parity) {
+  const bool ok = mbar_wait_spin_bounded(bar, parity, WAIT_NS);
+  return !group_or(id, count, !ok);
+}
 
 // D (16 x 8) = A (16 x K) B (K x 8) on the warp-level tensor-core path (mma.sync, tf32 operands
 // rounded from fp32, fp32 accumulate).  A points at element (0, 0) of a row-major fp32 block with
@@ -762,12 +767,12 @@ done:
 // as two MMAs of N = 192 per K step: one over U (K = 64 tokens) and one over S (K = 128 keys), whose
 // B operands are Nt over Pt and Mt over Qt, stacked row-wise in shared memory.
 // Roles:
-//   warps 0-7   the state (thread = value column v, key-channel half hf: S[64 hf ..][v]); they do
-//               nothing but the serial chain per chunk: D1 -> S update -> S^T into tensor memory;
+//   warps 0-7   the state (thread = value column v, key-channel half hf: S[64 hf ..][v]): the serial
+//               chain per chunk (D1 -> S update -> S^T into tensor memory), then, while the next
+//               chunk's products run, O^T out of tensor memory into o (staged, one TMA store);
 //   warp 8      lane 0 loads each chunk's Mt, e^{g_C} and Qt, lane 1 its v, w, Nt and Pt;
 //   warp 9      lane 0 issues the products;
-//   warps 10-13 form U = w (.) v in shared memory in place of v (tokens past a sequence's end
-//               zero), and read O^T out of tensor memory and store it (staged, one TMA store).
+//   warps 10-13 form U = w (.) v in shared memory in place of v (tokens past a sequence's end zero).
 // A chunk's buffers come in two parts, each double-buffered by chunk parity and released as soon
 // as the product that reads it completes: {v, w, Nt, Pt} after the U product, {Mt, Qt, e^{g_C}}
 // after the S product (and the state warps' read of e^{g_C}); so the loads of chunk c+2 start
@@ -986,7 +991,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
                      use_o ? ID_U192 : ID_U128, kk > 0 ? 1u : 0u);
           mma_commit(bar(B_UFREE0 + s));
         }
-        if (!mbar_wait_bounded(bar(B_FM0 + s), ph, WAIT_NS) || !mbar_wait_bounded(bar(B_SREADY), k & 1, WAIT_NS)) {
+        if (!mbar_wait_bounded(bar(B_FM0 + s), ph, WAIT_NS) || !mbar_wait_spin_bounded(bar(B_SREADY), k & 1, WAIT_NS)) {
           ok = false;
           break;
         }
@@ -1037,49 +1042,8 @@ __global__ void __launch_bounds__(sp::NT, 1)
       if (atid == 0) mbar_arrive(bar(B_UREADY0 + s));
       return true;
     };
-    // O readout: thread = value column v of the tile (TMEM lane), all 64 tokens of the chunk; a full
-    // chunk is staged in the swizzled layout of the output map and stored by TMA, the last partial
-    // chunk of a sequence goes straight to global memory (a box would overrun into the next sequence)
-    const int v = 32 * aq + lane;
-    const uint32_t tl = tmem + ((uint32_t)(32 * aq) << 16);
-    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o);
-    const bool vin = j0 + v < a.dv;
-    uint8_t *ot = sm + OFF_OST + (v >> 6) * 8192;
-    if (use_u && nk > 0 && !form_u(0)) ok = false;
-    for (int k = 0; ok && k < nk; ++k) {
-      if (use_u && k + 1 < nk && !form_u(k + 1)) { ok = false; break; }
-      if (!use_o) continue;
-      const int b = k & 1, c = cb + k, Cc = chunk_len(c);
-      const int tok0 = (int)(bos + (int64_t)c * C);
-      if (!group_wait(BAR_AUX, NAUX, bar(B_D1FULL0 + b), (k >> 1) & 1)) { ok = false; break; }
-      tc_fence_after();
-      float d[64];
-      tmem_ld32(tl + 256 * b + TM_D2, *reinterpret_cast<float(*)[32]>(&d[0]));
-      tmem_ld32(tl + 256 * b + TM_D2 + 32, *reinterpret_cast<float(*)[32]>(&d[32]));
-      tmem_wait_ld();
-      tc_fence_before();
-      if (atid == 0) bulk_wait_read();  // the previous chunk's store has read the staging tiles
-      group_sync(BAR_AUX, NAUX);
-      if (atid == 0) mbar_arrive(bar(B_OREAD0 + b));  // O^T of the buffer is in registers: free
-      if (Cc == C) {
-#pragma unroll
-        for (int j = 0; j < 64; ++j)
-          *reinterpret_cast<__nv_bfloat16 *>(ot + sw128(j, v & 63)) = __float2bfloat16_rn(d[j]);
-        fence_proxy_async();
-        group_sync(BAR_AUX, NAUX);
-        if (atid == 0) {
-          tma_store_3d(&tm_o, j0, h, tok0, sb + OFF_OST);
-          if (j0 + 64 < a.dv) tma_store_3d(&tm_o, j0 + 64, h, tok0, sb + OFF_OST + 8192);
-          bulk_commit();
-        }
-      } else if (vin) {
-        __nv_bfloat16 *dst = o + ((size_t)tok0 * a.H + h) * (size_t)a.dv + j0 + v;
-#pragma unroll
-        for (int j = 0; j < 64; ++j)
-          if (j < Cc) dst[(size_t)j * a.H * a.dv] = __float2bfloat16_rn(d[j]);
-      }
-    }
-    if (atid == 0) bulk_wait_read();
+    for (int k = 0; use_u && k < nk; ++k)
+      if (!form_u(k)) { ok = false; break; }
   } else if (warp < NSTATE / 32) {
     // ---------------------------------------------------------- state side
     const int q4 = warp & 3, hf = warp >> 2;
@@ -1113,6 +1077,50 @@ __global__ void __launch_bounds__(sp::NT, 1)
       tmem_st32(tl + 256 * b + TM_AS + 32 * hf, r);
       tmem_wait_st();
     };
+    // O of chunk cb + k, after the chain's work for the chunk (the state warps are otherwise idle until
+    // the next chunk's products complete): thread (v, hf) takes tokens 32 hf .. +31 of column v out of
+    // tensor memory and rounds them to bf16 into the staging tiles (the swizzled layout of the output
+    // map).  A full chunk leaves by TMA; the last partial chunk of a sequence row by row (a box would
+    // overrun into the next sequence): thread = token rr, a quarter qq of the tile's 128 columns.
+    __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(a.o);
+    const int rr = tid >> 2, qq = tid & 3;
+    uint8_t *orow = sm + OFF_OST + (qq >> 1) * 8192;
+    const int cq = 32 * (qq & 1);  // first column of the quarter inside its 64-column tile
+    const bool qin = j0 + 32 * qq < a.dv;
+    auto read_out = [&](int k) -> bool {
+      const int b = k & 1, c = cb + k, Cc = chunk_len(c);
+      const int tok0 = (int)(bos + (int64_t)c * C);
+      uint32_t dp[16];  // O of tokens 32 hf .. +31, column v, as bf16 pairs
+      {
+        float d[32];
+        tmem_ld32(tl + 256 * b + TM_D2 + 32 * hf, d);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) dp[j] = f2_to_bf2(d[2 * j], d[2 * j + 1]);
+      }
+      tc_fence_before();
+      if (tid == 0) bulk_wait_read();  // the previous chunk's store has read the staging tiles
+      group_sync(BAR_STATE, NSTATE);
+      if (tid == 0) mbar_arrive(bar(B_OREAD0 + b));  // O^T of the buffer is in registers: free
+      uint8_t *ot = sm + OFF_OST + (v >> 6) * 8192;
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        *reinterpret_cast<uint16_t *>(ot + sw128(32 * hf + j, v & 63)) = (uint16_t)(dp[j >> 1] >> (16 * (j & 1)));
+      fence_proxy_async();
+      group_sync(BAR_STATE, NSTATE);
+      if (Cc == C) {
+        if (tid == 0) {
+          tma_store_3d(&tm_o, j0, h, tok0, sb + OFF_OST);
+          if (j0 + 64 < a.dv) tma_store_3d(&tm_o, j0 + 64, h, tok0, sb + OFF_OST + 8192);
+          bulk_commit();
+        }
+      } else if (rr < Cc && qin) {
+        uint4 *dst = reinterpret_cast<uint4 *>(out + ((size_t)(tok0 + rr) * a.H + h) * (size_t)a.dv + j0 + 32 * qq);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) dst[x] = ld_s128(orow + sw128(rr, cq + 8 * x));
+      }
+      return true;
+    };
     if (nk > 0) {
       put_state(0);
       tc_fence_before();
@@ -1122,7 +1130,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
     for (int k = 0; k < nk; ++k) {
       const int s = k & 1, b = k & 1, ph = (k >> 1) & 1;
       // ---------------------------------------------------------- S <- Diag(e^{g_C}) S + D1
-      if (!group_wait(BAR_STATE, NSTATE, bar(B_D1FULL0 + b), ph)) { ok = false; break; }
+      if (!group_wait_spin(BAR_STATE, NSTATE, bar(B_D1FULL0 + b), ph)) { ok = false; break; }
       tc_fence_after();
       {
         const float4 *g1 = reinterpret_cast<const float4 *>(sm + OFF_G + s * REC_G) + 16 * hf;
@@ -1150,7 +1158,9 @@ __global__ void __launch_bounds__(sp::NT, 1)
         mbar_arrive(bar(B_D1FREE0 + b));
         if (k + 1 < nk) mbar_arrive(bar(B_SREADY));
       }
+      if (use_o && !read_out(k)) { ok = false; break; }
     }
+    if (tid == 0) bulk_wait_read();  // the last O store has read the staging tiles
     // ---------------------------------------------------------- the state after this CTA's chunks
     if (ok && vin) {
       float *dst = nullptr;

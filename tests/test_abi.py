@@ -260,3 +260,4 @@ def test_recurrent_validation(L):
         assert recurrent(L, p) == gdn2.GDN2_ERR_INVALID_ARG, i
     assert recurrent(L, [None] * 9, B=0, T=0) == gdn2.GDN2_OK
     assert L.gdn2_launch_count() == before
+
