@@ -163,8 +163,8 @@ gdn2_status check_chunk(const void *q, const void *k, const void *v, const void 
   if (!fits(tokens, H, d_v > d_k ? d_v : d_k, 1) || !fits(B, H, d_k, d_v)) return GDN2_ERR_INVALID_ARG;
   if ((long long)B * H * 8 > INT_MAX) return GDN2_ERR_INVALID_ARG;
   *a = gdn2::ChunkArgs{q, k, v, alpha, b, w, S0, o, S_T, cu_seqlens, B, T, H, d_k, d_v};
-  // bf16 runs on the tensor cores; fp32 (whose accuracy bf16 operands cannot keep) runs the SIMT
-  // kernel
+  // bf16 with d_v a multiple of 128 runs on the tensor cores; fp32 (whose accuracy bf16 operands
+  // cannot keep) and bf16 with d_v = 64 run the SIMT kernel
   *tc = gdn2::chunk_wy_supported(B, T, H, d_k, d_v, cu_seqlens != nullptr, dtype == GDN2_BF16);
   return GDN2_OK;
 }

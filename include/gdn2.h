@@ -95,12 +95,13 @@ typedef struct CUstream_st *gdn2_stream_t;
  * chunk: 64 (the only supported chunk length).
  * T == 0 (or an empty sequence) is valid: its S_T equals its S0; when the
  * batch holds no token at all, the token pointers (q .. w, o) may be NULL.
- * bf16 (d_k = 64 or 128) runs two tensor-core kernels over a workspace: the
+ * bf16 with d_v = 128 or 256 (d_k = 64 or 128) runs two tensor-core kernels over a workspace: the
  * first forms the chunk's WY factors (T = (I + L)^-1, W = -T A, and the decay-
  * absorbed q and k) for every chunk at once, the second carries the state
  * through each sequence's chunks in order (d_k = 64 is carried as 128 key
- * channels whose upper half stays zero); fp32 runs one SIMT kernel without a
- * workspace (bf16 tensor-core operands cannot keep the fp32 tolerance).
+ * channels whose upper half stays zero); fp32, and bf16 with d_v = 64, run one
+ * SIMT kernel without a workspace (bf16 tensor-core operands cannot keep the
+ * fp32 tolerance; the second kernel takes 128 value columns per CTA).
  * Returns GDN2_OK, or an error status with nothing launched; GDN2_ERR_CUDA
  * also when the workspace cannot be allocated.
  */
