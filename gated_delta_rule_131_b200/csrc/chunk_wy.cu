@@ -224,6 +224,10 @@ __device__ __forceinline__ int seq_of_chunk(const int32_t *coff, int N, int gidx
 // ==================================================================== kernel 1: WY factors
 namespace wy {
 constexpr int NT = 256;
+// the thread that issues every bulk store and publishes the records: warp 4 idles during the
+// triangular substitution, where the publish (a wait for the previous record's stores and a release)
+// costs nothing; the loads and the products stay with thread 0
+constexpr int ST_TID = 128;
 // shared memory (two CTAs per SM); regions are reused once their first contents are dead
 constexpr uint32_t OFF_XA = 0;                       // [A_m ; Q_m], two channel blocks -> Qt in rows 0..63
 constexpr uint32_t OFF_KT = OFF_XA + 2 * XA_BLK;     // 32768: K_m, two channel blocks -> Mt tile 0
@@ -245,20 +249,29 @@ struct WyParams {
   int N;           // sequences
   int nc;          // chunks per sequence of a dense batch
   int nrec;        // records to walk: dense N * nc * H; packed capacity * H (those past the batch are skipped)
-  int reverse;     // dense batches: records in chunk-major order, the last chunk index first
+  int order;       // walking order: 0 record order; dense batches 1 chunk-major, last chunk first, 2 chunk-major
+  int sms;         // SMs of the device
+  int reserve;     // CTAs on SMs 0 .. reserve-1 stop claiming records at `stop_at` (0: none do)
+  int stop_at;
   int64_t tokens;  // rows of the token tensors
   const int32_t *coff;  // packed batch: chunk offsets [N+1]; dense: nullptr
   float *g;             // workspace e^{g_C} [records][128]
   int *next;            // record counter, zero at launch: CTAs claim their records after the first in order
+  int *ready;           // per record, zero at launch: 1 once its stores are complete (published only when
+                        // the state pass runs alongside: `publish`; else it waits for every CTA to finish)
+  int publish;
+  int *done;            // factorisation CTAs that have finished (every record published), zero at launch
+  int ctas;             // factorisation CTAs launched
 };
 
-// Workspace record of the i-th record a CTA walks.  Dense batches go chunk-major with the last
-// chunk index first, so the records of the first chunks, which the state pass reads first, are the
-// ones written last (most likely still in L2 when it starts).
+// Workspace record of the i-th record in walking order.  Chunk-major walks take chunk c of every
+// (sequence, head) before chunk c+1.  First chunk first suits a state pass that runs alongside the
+// factorisation; last chunk first suits one that starts after it, because the records of the first
+// chunks, which it reads first, are then the ones written last (most likely still in L2).
 __device__ __forceinline__ int wy_record(const WyParams &p, int H, int i) {
-  if (!p.reverse) return i;
+  if (p.order == 0) return i;
   const int per_c = p.N * H;
-  const int c = p.nc - 1 - i / per_c, rem = i % per_c;
+  const int c = p.order == 1 ? p.nc - 1 - i / per_c : i / per_c, rem = i % per_c;
   return ((rem / H) * p.nc + c) * H + rem % H;
 }
 
@@ -283,12 +296,18 @@ __device__ __forceinline__ int wy_tok0(const ChunkArgs &a, const WyParams &p, in
   return (int)(bos + (int64_t)c * C);
 }
 
-// Persistent (two CTAs per SM): CTA i takes record i first, then claims the next unclaimed record
-// from a counter when it starts one, so records finish roughly in their walking order and no CTA
-// is left with a long tail.  The set-up (barriers, tensor memory, descriptor prefetch) happens
-// once; every record's inputs are prefetched into L2 one record ahead, and the stores of a record
-// are waited for (their shared-memory sources read) only when the next record's loads are about to
-// overwrite them.
+// Persistent (two CTAs per SM): CTA i takes record i first, then claims unclaimed records from a
+// counter one record ahead (the claim's round trip overlaps a whole record), so records finish
+// roughly in their walking order and no CTA is left with a long tail.  The set-up (barriers, tensor
+// memory, descriptor prefetch) happens once; every record's inputs are prefetched into L2 one record
+// ahead, and the stores of a record are waited for (their shared-memory sources read) only when the
+// next record's loads are about to overwrite them.  The state pass may start before this kernel
+// ends.  When it is to run alongside (`publish`), CTAs on the first `reserve` SMs stop claiming at
+// `stop_at`, so that those SMs fall idle early and the state pass runs there while the other SMs
+// factor the rest, and each record's flag is published once its stores are complete (during the
+// next record's substitution, where the wait and the release cost least); the state pass waits on
+// the flags.  Otherwise it waits for the count of finished CTAs, which each CTA raises once its last
+// store is complete.
 __global__ void __launch_bounds__(wy::NT, 2)
     wy_factor_kernel(const ChunkArgs a, const WyParams p, const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_b,
@@ -324,11 +343,17 @@ __global__ void __launch_bounds__(wy::NT, 2)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16);
+  griddep_launch_dependents();  // the state pass may be scheduled onto SMs as they fall idle
   bool ok = true;
   uint32_t nfull = 0, nmma = 0;  // completed phases of the two barriers
-  // the claimed next record, in one of two slots by iteration parity (a slot is rewritten only after
-  // every thread has passed the barrier that follows its read)
+  // the next record, in one of two slots by iteration parity (a slot is rewritten only after every
+  // thread has passed the barrier that follows its read)
   volatile int *s_next = reinterpret_cast<volatile int *>(sm + OFF_BAR + 20);
+  const bool stops = p.reserve > 0 && (int)sm_id_count() == p.sms && (int)sm_id() < p.reserve;
+  // thread 0: the record claimed for after the next one; thread ST_TID: the last record whose flag is
+  // still to be published
+  int claim = 0, prev = -1;
+  if (tid == 0) claim = (int)gridDim.x + atomicAdd(p.next, 1);
 
   bool pre = false;  // this record's input loads were issued by the previous record's epilogue
   for (int it = blockIdx.x, nit = 0, par = 0; it < p.nrec; it = nit, par ^= 1) {
@@ -336,7 +361,10 @@ __global__ void __launch_bounds__(wy::NT, 2)
     const int h = rec % a.H;
     int n, c;
     const int tok0 = wy_tok0(a, p, rec, &n, &c);
-    if (tid == 0) s_next[par] = (int)gridDim.x + atomicAdd(p.next, 1);
+    if (tid == 0) {
+      s_next[par] = claim;
+      claim = (claim >= p.nrec || (stops && claim >= p.stop_at)) ? p.nrec : (int)gridDim.x + atomicAdd(p.next, 1);
+    }
     __syncthreads();
     nit = s_next[par];
     if (tok0 < 0) continue;  // past the chunks of a packed batch (uniform per CTA)
@@ -349,8 +377,8 @@ __global__ void __launch_bounds__(wy::NT, 2)
     int nn = 0, ncc = 0;
     const int nrec_ = nit < p.nrec ? wy_record(p, a.H, nit) : 0;
     const int ntok = nit < p.nrec ? wy_tok0(a, p, nrec_, &nn, &ncc) : -1;
+    if (tid == ST_TID) bulk_wait_read();  // the previous record's stores have read TP and TS (reused below)
     if (tid == 0) {
-      bulk_wait_read();  // the previous record's stores have read their tiles (TP and TS are reused below)
       if (!pre) {
         mbar_expect_tx(bar_full, TMA_BYTES);
 #pragma unroll
@@ -520,6 +548,11 @@ __global__ void __launch_bounds__(wy::NT, 2)
     }
     tc_fence_before();
     __syncthreads();
+    if (tid == ST_TID && p.publish && prev >= 0) {  // the previous record's stores are complete: publish it
+      bulk_wait_done<0>();
+      flag_publish(p.ready + prev);
+      prev = -1;
+    }
     if (warp < 2) {  // the four 16x16 diagonal blocks, right-looking; lane = column j of block R
       const int R = 2 * warp + (lane >> 4), j = lane & 15;
       const float *Lb = Ls + 16 * R * LDF + 16 * R;
@@ -636,7 +669,7 @@ __global__ void __launch_bounds__(wy::NT, 2)
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {  // Nt, Pt and e^{g_C} are final: store them while product pass 2 runs
+    if (tid == ST_TID) {  // Nt, Pt and e^{g_C} are final: store them while product pass 2 runs
       tma_store_2d(&tm_wn, 0, rec * 128, sb + OFF_TP);
       tma_store_2d(&tm_wp, 0, rec * 64, sb + OFF_TS);
       bulk_store(p.g + (size_t)rec * 128, sb + OFF_SC + 256 * 4, REC_G);
@@ -655,10 +688,10 @@ __global__ void __launch_bounds__(wy::NT, 2)
                  sdesc_sw128(sb + OFF_XA + 2048 * k, XA_BLK, 1024), ID_KM128, k > 0 ? 1u : 0u);
       }
       mma_commit(bar_mma);
-      // Nt and Pt: their stores have read the tiles before any thread passes the barrier below
-      // (the epilogue writes Mt into them)
-      bulk_wait_read();
     }
+    // Nt and Pt: their stores have read the tiles before any thread passes the barrier below (the
+    // epilogue writes Mt into them)
+    if (tid == ST_TID) bulk_wait_read();
     if (!mbar_wait_bounded(bar_mma, nmma & 1, WAIT_NS)) ok = false;
     ++nmma;
     if (__syncthreads_or(!ok)) goto done;
@@ -718,7 +751,7 @@ __global__ void __launch_bounds__(wy::NT, 2)
         }
         fence_proxy_async();
         group_sync(1, 128);  // the four Qt warps: every Qt tile written, every Q_m row read
-        if (tid == 0) {      // Qt -> workspace; the next record's q into the dead Q_m rows
+        if (tid == ST_TID) {  // Qt -> workspace; the next record's q into the dead Q_m rows
           tma_store_2d(&tm_wq, 0, rec * 64, sb + OFF_XA);
           tma_store_2d(&tm_wq, 64, rec * 64, sb + OFF_XA + XA_BLK);
           bulk_commit();
@@ -736,10 +769,11 @@ __global__ void __launch_bounds__(wy::NT, 2)
     __syncthreads();
 
     // ------------------------------------------------------------ Mt -> workspace (waited for at the next record)
-    if (tid == 0) {
+    if (tid == ST_TID) {
       tma_store_2d(&tm_wm, 0, rec * 128, sb + OFF_TP);
       tma_store_2d(&tm_wm, 64, rec * 128, sb + OFF_TS);
       bulk_commit();
+      prev = rec;
       if (pre) {  // the next record's b into the rows Qt leaves, once its store has read them
         asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 #pragma unroll
@@ -750,8 +784,12 @@ __global__ void __launch_bounds__(wy::NT, 2)
   }
 
 done:
-  if (!ok && tid == 0) atomicExch(p.status, 4);
-  if (tid == 0) bulk_wait_read();
+  if (tid == 0 && !ok) atomicExch(p.status, 4);
+  if (tid == ST_TID) {
+    bulk_wait_done<0>();
+    if (p.publish && prev >= 0) flag_publish(p.ready + prev);
+    counter_release_add(p.done);  // after this CTA's last store is complete
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -862,7 +900,10 @@ __global__ void __launch_bounds__(sp::NT, 1)
     n = blockIdx.x / (per * (q.nseg - 1) * a.H);
     ident = t == 0;
     tile = ident ? 0 : t - 1;
-    if (ident && seg == 0) return;  // segment 0 starts from S0: its end state is all that is needed
+    if (ident && seg == 0) {  // segment 0 starts from S0: its end state is all that is needed
+      griddep_wait();
+      return;
+    }
   } else if (q.mode == 2) {
     tile = blockIdx.x % tiles;
     seg = (blockIdx.x / tiles) % q.nseg;
@@ -903,15 +944,35 @@ __global__ void __launch_bounds__(sp::NT, 1)
   bool ok = true;
 
   if (warp == W_LOAD) {
+    // A chunk's record may be read once its flag is published, or once every factorisation CTA has
+    // finished (the only signal when the factorisation publishes no flags).  The check comes before
+    // the wait for the stage, so that its round trip overlaps that wait.
+    bool all_done = false;
+    auto record_ready = [&](int rec) -> bool {
+      if (all_done) return true;
+      if (p.publish) {
+        if (counter_acquire(p.done) < p.ctas) return flag_wait_bounded(p.ready + rec, WAIT_NS);
+      } else if (counter_acquire(p.done) < p.ctas) {
+        const uint64_t t0 = globaltimer_ns();
+        do {
+          __nanosleep(256);
+          if (globaltimer_ns() - t0 > WAIT_NS) return false;
+        } while (counter_acquire(p.done) < p.ctas);
+      }
+      all_done = true;
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      return true;
+    };
     if (lane == 0) {
       // ---------------------------------------------------------- Mt, Qt, e^{g_C} of each chunk
       for (int k = 0; k < nk; ++k) {
         const int s = k & 1, c = cb + k, ph2 = ((k - 2) >> 1) & 1;
         const uint32_t st = sb + s * STAGE, full = bar(B_FM0 + s);
         const int rec = (coff + c) * a.H + h;
-        // chunk k-2's: read once its products are complete and the state warps read e^{g_C}
-        if (k >= 2 && !(mbar_wait_bounded(bar(B_D1FULL0 + s), ph2, WAIT_NS) &&
-                        mbar_wait_bounded(bar(B_D1FREE0 + s), ph2, WAIT_NS))) {
+        // the record's stores are complete; chunk k-2's buffers are free once its products are
+        // complete and the state warps read e^{g_C}
+        if (!record_ready(rec) || (k >= 2 && !(mbar_wait_bounded(bar(B_D1FULL0 + s), ph2, WAIT_NS) &&
+                                               mbar_wait_bounded(bar(B_D1FREE0 + s), ph2, WAIT_NS)))) {
           ok = false;
           break;
         }
@@ -941,7 +1002,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
         const uint32_t st = sb + s * STAGE, full = bar(B_FU0 + s);
         const int rec = (coff + c) * a.H + h;
         const int tok0 = (int)(bos + (int64_t)c * C);
-        if (k >= 2 && !mbar_wait_bounded(bar(B_UFREE0 + s), ((k - 2) >> 1) & 1, WAIT_NS)) {
+        if (!record_ready(rec) || (k >= 2 && !mbar_wait_bounded(bar(B_UFREE0 + s), ((k - 2) >> 1) & 1, WAIT_NS))) {
           ok = false;
           break;
         }
@@ -1005,7 +1066,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
     }
   } else if (warp >= W_AUX) {
     // ---------------------------------------------------------- U formation and O readout (warps 10-13)
-    const int atid = tid - W_AUX * 32, aq = warp & 3;
+    const int atid = tid - W_AUX * 32;
     // U = w (.) v of chunk cb + k in place of v (16-byte pieces, each read and written by one thread);
     // tokens past the sequence (the tile holds the next sequence's tokens there) become zero
     auto form_u = [&](int k) -> bool {
@@ -1179,6 +1240,10 @@ __global__ void __launch_bounds__(sp::NT, 1)
     }
   }
   if (!ok) atomicExch(p.status, 4);
+  // the factorisation kernel has ended too, so the stream sees both complete.  One converged warp
+  // that has finished its own work waits: the wait parks the whole warp, and the idle lanes of the
+  // loader and issuer warps would otherwise reach it while their working lanes still run.
+  if (warp == 0) griddep_wait();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -1369,7 +1434,8 @@ int scan_segments(int B, int T, int H, int dv, bool packed, int sms, int *seg_le
 }
 
 // Workspace layout: Mt tiles | Nt tiles | Qt tiles | Pt tiles | e^{g_C} | two-level scan maps and entry
-// states (long sequences only) | chunk offsets (packed only) | record counter; 256-byte aligned arrays
+// states (long sequences only) | chunk offsets (packed only) | record counter (256 bytes) and one ready
+// flag per record (int32), zeroed together before each call; 256-byte aligned arrays
 struct WsLayout {
   long long records;
   int nseg, seg_len;
@@ -1392,8 +1458,21 @@ WsLayout ws_layout(int B, int T, int H, int dv, bool packed, int sms) {
   L.ss = up256(L.sbm + (ns ? pairs * (ns - 1) * DK * dv * 4 : 0));
   L.coff = up256(L.ss + pairs * ns * DK * dv * 4);
   L.cnt = L.coff + (packed ? up256((size_t)(B + 1) * 4) : 0);
-  L.total = L.cnt + 256;
+  L.total = L.cnt + up256(256 + r * 4);
   return L;
+}
+
+// Where the factorisation hands SMs to a state pass of `walks` CTAs (one per SM) before it ends.  Run
+// beside the factorisation, the state pass takes about 1.9 us per chunk, and a factorisation CTA
+// about 9 us per record (two per SM; measured on B200, 1.3B layer).  The CTAs on `walks` SMs stop
+// claiming once `stop_at` records are claimed, chosen so that the other SMs factor the remaining
+// records in about the state pass's time: the two then end together.  Returns -1 (no SM handed over)
+// when the walks do not leave room.
+int handover_stop(long long records, long long walks, int nc, int sms) {
+  if (walks <= 0 || walks > sms - 16) return -1;
+  const double rest = 2.0 * (double)(sms - walks) * (double)nc * 1.9 / 9.0;
+  const long long stop = records - (long long)rest;
+  return stop > 0 ? (int)stop : 0;
 }
 
 }  // namespace
@@ -1423,8 +1502,25 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   p.coff = a.cu ? reinterpret_cast<const int32_t *>(base + L.coff) : nullptr;
   p.g = reinterpret_cast<float *>(base + L.g);
   p.nrec = (int)L.records;
-  p.reverse = a.cu ? 0 : 1;
   p.next = reinterpret_cast<int *>(base + L.cnt);
+  p.ready = reinterpret_cast<int *>(base + L.cnt + 256);
+  p.done = p.next + 1;
+  p.ctas = 0;
+  p.publish = 0;
+  p.sms = sms;
+  p.reserve = 0;
+  p.stop_at = p.nrec;
+  p.order = a.cu ? 0 : 1;
+  const long long tiles = (a.dv + sp::VW - 1) / sp::VW;
+  if (!a.cu && L.nseg <= 1) {  // whole-sequence walks that leave SMs free: hand SMs over early
+    const int stop = handover_stop(L.records, (long long)a.B * a.H * tiles, p.nc, sms);
+    if (stop >= 0) {
+      p.order = 2;
+      p.publish = 1;
+      p.reserve = (int)((long long)a.B * a.H * tiles);
+      p.stop_at = stop;
+    }
+  }
 
   CUtensorMap mq, mk, mb, mal, mv, mw, mo, mm, mn, mqt, mp;
   if (tokens > 0) {
@@ -1449,24 +1545,38 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
     chunk_offsets_kernel<<<1, 1024, 0, stream>>>(a.cu, a.B, const_cast<int32_t *>(p.coff));
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
-  if (L.records > 0 && tokens > 0) {
-    if ((err = cudaMemsetAsync(p.next, 0, sizeof(int), stream)) != cudaSuccess) return err;
+  const bool wy_runs = L.records > 0 && tokens > 0;
+  if (wy_runs) {
+    if ((err = cudaMemsetAsync(p.next, 0, 256 + (size_t)L.records * 4, stream)) != cudaSuccess) return err;
     err = cudaFuncSetAttribute(wy_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wy::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     note_launch();
     const long long grid = L.records < 2LL * sms ? L.records : 2LL * sms;  // persistent: two CTAs per SM
+    p.ctas = (int)grid;
     wy_factor_kernel<<<(unsigned)grid, wy::NT, wy::SMEM_BYTES, stream>>>(a, p, mq, mk, mb, mal, mm, mn, mqt, mp);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
-  const long long tiles = (a.dv + sp::VW - 1) / sp::VW;
   err = cudaFuncSetAttribute(state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp::SMEM_BYTES);
   if (err != cudaSuccess) return err;
-  ScanParams q{};
-  if (L.nseg <= 1) {  // one walk per (sequence, head, value tile)
+  // The state pass right after the factorisation is a programmatic dependent launch: its CTAs are
+  // scheduled onto SMs as the factorisation leaves them, and it waits on each record's flag.
+  auto state_pass = [&](long long grid, const ScanParams &sq, bool dependent) -> cudaError_t {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(sp::NT);
+    cfg.dynamicSmemBytes = sp::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = dependent ? 1 : 0;
     note_launch();
-    state_pass_kernel<<<(unsigned)(a.B * a.H * tiles), sp::NT, sp::SMEM_BYTES, stream>>>(a, p, q, mm, mn, mqt, mp, mv, mw, mo);
-    return cudaGetLastError();
-  }
+    return cudaLaunchKernelEx(&cfg, state_pass_kernel, a, p, sq, mm, mn, mqt, mp, mv, mw, mo);
+  };
+  ScanParams q{};
+  if (L.nseg <= 1)  // one walk per (sequence, head, value tile)
+    return state_pass(a.B * a.H * tiles, q, wy_runs);
   // two-level scan: segment maps, their chain into entry states, then the segments' walks
   q.seg_len = L.seg_len;
   q.nseg = L.nseg;
@@ -1474,10 +1584,7 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   q.sum_b = reinterpret_cast<float *>(base + L.sbm);
   q.s_start = reinterpret_cast<float *>(base + L.ss);
   q.mode = 1;
-  note_launch();
-  state_pass_kernel<<<(unsigned)(a.B * a.H * (L.nseg - 1) * (1 + tiles)), sp::NT, sp::SMEM_BYTES, stream>>>(
-      a, p, q, mm, mn, mqt, mp, mv, mw, mo);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  if ((err = state_pass((long long)a.B * a.H * (L.nseg - 1) * (1 + tiles), q, wy_runs)) != cudaSuccess) return err;
   const int chain_smem = (128 * 132 + 32 * 132) * 4;
   err = cudaFuncSetAttribute(segment_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, chain_smem);
   if (err != cudaSuccess) return err;
@@ -1485,10 +1592,7 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   segment_chain_kernel<<<(unsigned)(a.B * a.H * tiles), 256, chain_smem, stream>>>(a, q);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   q.mode = 2;
-  note_launch();
-  state_pass_kernel<<<(unsigned)(a.B * a.H * L.nseg * tiles), sp::NT, sp::SMEM_BYTES, stream>>>(a, p, q, mm, mn, mqt,
-                                                                                                  mp, mv, mw, mo);
-  return cudaGetLastError();
+  return state_pass((long long)a.B * a.H * L.nseg * tiles, q, false);
 }
 
 }  // namespace gdn2

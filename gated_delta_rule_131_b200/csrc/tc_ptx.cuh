@@ -134,6 +134,63 @@ __device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t byt
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until every bulk store of this thread has finished reading its shared-memory source.
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Wait until at most N of this thread's most recent bulk groups are still pending: every older
+// group's writes are complete.
+template <int N>
+__device__ __forceinline__ void bulk_wait_done() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// ------------------------------------------------------------------ flags between kernels
+// A record written by bulk stores is published with a release store of its flag, once the stores are
+// complete; a reader acquires the flag before its own bulk (async-proxy) loads of the record.  The
+// proxy fences order the async-proxy writes and reads against the generic-proxy flag.
+__device__ __forceinline__ void flag_publish(int *flag) {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(1) : "memory");
+}
+__device__ __forceinline__ bool flag_test(const int *flag) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+  return v != 0;
+}
+__device__ __forceinline__ int counter_acquire(const int *c) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(c) : "memory");
+  return v;
+}
+__device__ __forceinline__ void counter_release_add(int *c) {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(c) : "memory");
+}
+// Waits (bounded) for a published flag; false when `limit_ns` passed first.
+__device__ __forceinline__ bool flag_wait_bounded(const int *flag, uint64_t limit_ns) {
+  if (!flag_test(flag)) {
+    const uint64_t t0 = globaltimer_ns();
+    do {
+      __nanosleep(64);
+      if (globaltimer_ns() - t0 > limit_ns) return false;
+    } while (!flag_test(flag));
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return true;
+}
+// Programmatic dependent launch: the next kernel of the stream, launched with programmatic stream
+// serialization, may start once every CTA of this one has called launch_dependents (or exited);
+// griddep_wait returns once the kernel before this one has completed and its writes are visible (at
+// once when this kernel was launched without the attribute).
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ uint32_t sm_id() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t sm_id_count() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nsmid;" : "=r"(r));
+  return r;
+}
 
 // ------------------------------------------------------------------ tcgen05 / TMEM
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_slot, uint32_t ncols) {

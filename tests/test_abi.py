@@ -222,19 +222,23 @@ def test_block_epilogue_validation(L):
 def test_chunk_workspace_layout(L):
     """The tensor-core path's workspace (host arithmetic only; 148 SMs when no GPU is present)."""
     record = 32768 + 16384 + 16384 + 8192 + 512  # M, N, Q, P tiles in bf16 and e^{g_C} in fp32
-    # 1.3B layer: 2048 (chunk, head) records and the 256-byte record counter of the WY kernel; one walk
-    # per head, no scan buffers (the state pass forms U = w * v itself)
-    assert L.gdn2_chunk_fwd_workspace_bytes(4, 2048, 16, 128, 128, 64, 0, gdn2.GDN2_BF16) == 2048 * record + 256
+
+    def counters(records):  # the WY kernel's 256-byte record counter and one int32 ready flag per record
+        return (256 + 4 * records + 255) // 256 * 256
+
+    # 1.3B layer: 2048 (chunk, head) records; one walk per head, no scan buffers (the state pass forms
+    # U = w * v itself)
+    assert L.gdn2_chunk_fwd_workspace_bytes(4, 2048, 16, 128, 128, 64, 0, gdn2.GDN2_BF16) == 2048 * record + counters(2048)
     # long context (1 x 65536 tokens, 16 heads): the two-level scan adds, per head, S - 1 segment maps
     # A_j (128 x 128) and B_j (128 x d_v) and S entry states, all fp32: 64 KiB x (3 S - 2)
     n = L.gdn2_chunk_fwd_workspace_bytes(1, 65536, 16, 128, 128, 64, 0, gdn2.GDN2_BF16)
-    extra = n - 16384 * record - 256
+    extra = n - 16384 * record - counters(16384)
     assert extra > 0 and extra % (16 * 65536) == 0 and (extra // (16 * 65536) + 2) % 3 == 0
     assert (extra // (16 * 65536) + 2) // 3 >= 2
     # fp32 runs the SIMT kernel, which needs no workspace; bf16 with d_k = 64 runs the tensor-core
     # path with the same 128-channel records
     assert L.gdn2_chunk_fwd_workspace_bytes(4, 2048, 16, 128, 128, 64, 0, gdn2.GDN2_F32) == 0
-    assert L.gdn2_chunk_fwd_workspace_bytes(4, 2048, 16, 64, 128, 64, 0, gdn2.GDN2_BF16) == 2048 * record + 256
+    assert L.gdn2_chunk_fwd_workspace_bytes(4, 2048, 16, 64, 128, 64, 0, gdn2.GDN2_BF16) == 2048 * record + counters(2048)
 
 
 def recurrent(L, ptrs=None, B=1, T=64, H=1, dk=64, dv=64, cu=None, erase=gdn2.GDN2_ERASE_R2, dtype=gdn2.GDN2_BF16):
