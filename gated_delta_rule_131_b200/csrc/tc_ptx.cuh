@@ -163,14 +163,23 @@ __device__ __forceinline__ void counter_release_add(int *c) {
   asm volatile("fence.proxy.async.global;" ::: "memory");
   asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(c) : "memory");
 }
-// Waits (bounded) for a published flag; false when `limit_ns` passed first.
+__device__ __forceinline__ bool flag_test_relaxed(const int *flag) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+  return v != 0;
+}
+// Waits (bounded) for a published flag; false when `limit_ns` passed first.  Polls with relaxed loads
+// and a growing pause (many waiters share a few cache lines with the writer), then acquires once.
 __device__ __forceinline__ bool flag_wait_bounded(const int *flag, uint64_t limit_ns) {
   if (!flag_test(flag)) {
     const uint64_t t0 = globaltimer_ns();
+    uint32_t pause = 32;
     do {
-      __nanosleep(64);
+      __nanosleep(pause);
+      pause = pause < 512 ? 2 * pause : 512;
       if (globaltimer_ns() - t0 > limit_ns) return false;
-    } while (!flag_test(flag));
+    } while (!flag_test_relaxed(flag));
+    (void)flag_test(flag);  // acquire: the record's stores happen before what follows
   }
   asm volatile("fence.proxy.async.global;" ::: "memory");
   return true;
