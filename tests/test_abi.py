@@ -223,7 +223,7 @@ def test_chunk_workspace_layout(L):
     """The tensor-core path's workspace (host arithmetic only; 148 SMs when no GPU is present)."""
     record = 32768 + 16384 + 16384 + 8192 + 512  # M, N, Q, P tiles in bf16 and e^{g_C} in fp32
 
-    def counters(records):  # the WY kernel's 256-byte record counter and one int32 ready flag per record
+    def counters(records):  # the WY kernel's 256 bytes of counters and one int32 ready flag per record
         return (256 + 4 * records + 255) // 256 * 256
 
     # 1.3B layer: 2048 (chunk, head) records; one walk per head, no scan buffers (the state pass forms
