@@ -1,13 +1,16 @@
 // Chunkwise WY forward of the Gated Delta Rule-2 as two tensor-core kernels
-// (bf16 inputs, d_k = 128, fp32 state and accumulation), split where the
+// (bf16 inputs, d_k = 64 or 128, fp32 state and accumulation), split where the
 // dependence on the state begins:
 //
-//   wy_factor_kernel   one CTA per (chunk, head), all chunks at once: the
-//                      decay-absorbed erase factors, [L; P], T = (I + L)^-1, and
-//                      from them the chunk's state transition and output maps,
-//                      stored to a workspace record;
-//   state_pass_kernel  one CTA per (sequence, head, 64 value columns): walks the
-//                      chunks of its sequence in order and carries S in fp32.
+//   wy_factor_kernel   persistent, two CTAs per SM, one (chunk, head) record at a
+//                      time, all chunks independently: the decay-absorbed erase
+//                      factors, [L; P], T = (I + L)^-1, and from them the chunk's
+//                      state transition and output maps, stored to a workspace
+//                      record;
+//   state_pass_kernel  one CTA per (sequence, head, 128 value columns): walks the
+//                      chunks of its sequence in order and carries S in fp32.  A
+//                      programmatic dependent launch: it may start on SMs the first
+//                      kernel leaves, and reads each record once it is complete.
 //
 // Per chunk of C = 64 tokens (r, i index tokens, c a key channel, m the running
 // log-decay at token 31 of the chunk, g_r the running log-decay at r):
