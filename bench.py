@@ -512,7 +512,7 @@ def bench_bwd(gdn2, dev, stream, pk, pk_kind, reps=5):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "traffic": tr["dram_bytes_per_launch"] if tr else None,
                          "peak_source": pk_kind, "algorithmic_bytes_per_launch": nbytes,
-                         "note": "issue- and latency-bound SIMT kernel (about 655 instructions per warp and token)"}}
+                         "note": "issue- and latency-bound SIMT kernel (about 860 instructions per warp and token)"}}
 
 
 def time_calls(fn, dev, stream, reps):

@@ -19,9 +19,13 @@
 // each thread over its tile and added across tiles with fp32 reductions in L2, into a buffer that
 // a second kernel converts to the output type.
 //
-// States are not kept for every token: a first forward pass stores the tile's state every CK
-// tokens (checkpoints in the workspace); the backward pass rebuilds each segment's CK states in
-// shared memory from its checkpoint, then walks the segment backwards.
+// States are not kept for every token.  A first forward pass stores the tile's state every GK
+// tokens (one group of GK / CK segments) and every d_t.  The backward pass walks the groups from
+// the last: it first rebuilds the state before each CK-token segment of the group from the group's
+// checkpoint and the stored d_t, into a scratch area of its own in the workspace, then walks the
+// group's segments backwards, rebuilding each segment's CK states in shared memory from the
+// scratch.  Every rebuild repeats the first pass's operations (S = d_t k + alpha S, rounded the
+// same way), so it reproduces its states exactly, and no thread reads what another wrote.
 #include <algorithm>
 
 #include "common.cuh"
@@ -29,14 +33,17 @@
 namespace gdn2 {
 namespace {
 
-constexpr int NJ = 16;  // value columns per CTA
-constexpr int CK = 4;   // tokens per checkpoint segment (4 CTAs of 128 rows fit an SM)
+constexpr int NJ = 16;       // value columns per CTA
+constexpr int CK = 4;        // tokens per segment rebuilt in shared memory (4 CTAs of 128 rows fit an SM)
+constexpr int GK = 64;       // tokens per stored checkpoint
+constexpr int GS = GK / CK;  // segments per checkpoint group
 
 struct BwdParams {
   const void *q, *k, *v, *alpha, *b, *w, *dO;
   const float *S0, *dST;
   float4 *acc;       // [tokens, H, d_k] x (dq, dk, dalpha, db) fp32, summed over the tiles (zeroed)
-  float4 *ck;        // checkpoints [slots, H, tiles, NJ / 4, d_k] float4
+  float4 *ck;        // checkpoints every GK tokens [slots, H, tiles, NJ / 4, d_k] float4
+  float4 *scr;       // per CTA: the states before the segments of one group [CTAs, GS, NJ / 4, d_k] float4
   float *dl;         // d_t of every token [tokens, H, d_v] fp32, from the first pass
   void *dv, *dw;     // [tokens, H, d_v]
   float *dS0;        // [N, H, d_k, d_v] or nullptr
@@ -115,8 +122,10 @@ __global__ void __launch_bounds__(DK, 512 / DK) chunk_bwd_kernel(const BwdParams
     len = p.T;
   }
   const int nseg = (int)((len + CK - 1) / CK);
-  const long long slot0 = bos / CK + n;  // distinct slots for every segment of every sequence
-  auto ck_at = [&](int m) { return p.ck + ((((slot0 + m) * H + h) * tiles + tile) * (NJ / 4)) * DK + i; };
+  const long long slot0 = bos / GK + n;  // distinct slots for every group of every sequence
+  auto ck_at = [&](int grp) { return p.ck + ((((slot0 + grp) * H + h) * tiles + tile) * (NJ / 4)) * DK + i; };
+  const size_t cta = ((size_t)n * H + h) * tiles + tile;
+  auto scr_at = [&](int m) { return p.scr + ((cta * GS + (m % GS)) * (NJ / 4)) * DK + i; };
   auto krow = [&](long long t) { return ((size_t)t * H + h) * DK + i; };
   auto vcol = [&](long long t, int j) { return ((size_t)t * H + h) * DV + j0 + j; };
 
@@ -178,13 +187,15 @@ __global__ void __launch_bounds__(DK, 512 / DK) chunk_bwd_kernel(const BwdParams
     }
   };
 
-  // Pass 1: forward over the sequence, storing the state before every segment and every d_t.
+  // Pass 1: forward over the sequence, storing the state before every group and every d_t.
   for (int m = 0; m < nseg; ++m) {
     const long long t0 = bos + (long long)m * CK;
     const int nt = (int)min((long long)CK, len - (long long)m * CK);
-    float4 *c = ck_at(m);
+    if (m % GS == 0) {
+      float4 *c = ck_at(m / GS);
 #pragma unroll
-    for (int q4 = 0; q4 < NJ / 4; ++q4) c[q4 * DK] = make_float4(s[4 * q4], s[4 * q4 + 1], s[4 * q4 + 2], s[4 * q4 + 3]);
+      for (int q4 = 0; q4 < NJ / 4; ++q4) c[q4 * DK] = make_float4(s[4 * q4], s[4 * q4 + 1], s[4 * q4 + 2], s[4 * q4 + 3]);
+    }
     load_seg(t0, nt, false);
     __syncthreads();  // the segment's value-side inputs are in shared memory
 #pragma unroll
@@ -215,7 +226,43 @@ __global__ void __launch_bounds__(DK, 512 / DK) chunk_bwd_kernel(const BwdParams
   for (int m = nseg - 1; m >= 0; --m) {
     const long long t0 = bos + (long long)m * CK;
     const int nt = (int)min((long long)CK, len - (long long)m * CK);
-    const float4 *c = ck_at(m);
+    if (m == nseg - 1 || m % GS == GS - 1) {
+      // entering group m / GS: the state before each of its segments, from the group's checkpoint
+      // and the stored d_t, into this thread's row of the scratch
+      const int m0 = m - m % GS;
+      {
+        const float4 *c = ck_at(m / GS);
+#pragma unroll
+        for (int q4 = 0; q4 < NJ / 4; ++q4) {
+          const float4 x = c[q4 * DK];
+          s[4 * q4] = x.x;
+          s[4 * q4 + 1] = x.y;
+          s[4 * q4 + 2] = x.z;
+          s[4 * q4 + 3] = x.w;
+        }
+      }
+      for (int mm = m0; mm <= m; ++mm) {
+        float4 *sc = scr_at(mm);
+#pragma unroll
+        for (int q4 = 0; q4 < NJ / 4; ++q4) sc[q4 * DK] = make_float4(s[4 * q4], s[4 * q4 + 1], s[4 * q4 + 2], s[4 * q4 + 3]);
+        if (mm == m) break;  // the state after segment m is not used
+        const long long ta = bos + (long long)mm * CK;  // a full segment: only a sequence's last one can be short
+#pragma unroll
+        for (int u = 0; u < CK; ++u) {
+          const float al = ld<T>(p.alpha, krow(ta + u)), kk = ld<T>(p.k, krow(ta + u));
+          const float4 *dl4 = reinterpret_cast<const float4 *>(p.dl + vcol(ta + u, 0));
+#pragma unroll
+          for (int q4 = 0; q4 < NJ / 4; ++q4) {
+            const float4 d = dl4[q4];
+            s[4 * q4] = fmaf(kk, d.x, s[4 * q4] * al);
+            s[4 * q4 + 1] = fmaf(kk, d.y, s[4 * q4 + 1] * al);
+            s[4 * q4 + 2] = fmaf(kk, d.z, s[4 * q4 + 2] * al);
+            s[4 * q4 + 3] = fmaf(kk, d.w, s[4 * q4 + 3] * al);
+          }
+        }
+      }
+    }
+    const float4 *c = scr_at(m);
 #pragma unroll
     for (int q4 = 0; q4 < NJ / 4; ++q4) {
       const float4 x = c[q4 * DK];
@@ -315,8 +362,10 @@ cudaError_t bwd_t(const BwdArgs &a, void *ws, cudaStream_t stream) {
   uint8_t *base = static_cast<uint8_t *>(ws);
   p.acc = reinterpret_cast<float4 *>(base);
   p.dl = reinterpret_cast<float *>(base + align256(acc_elems * sizeof(float4)));
+  const long long slots = tokens / GK + a.B + 1;
   p.ck = reinterpret_cast<float4 *>(base + align256(acc_elems * sizeof(float4)) +
                                     align256((size_t)tokens * a.H * a.Dv * sizeof(float)));
+  p.scr = reinterpret_cast<float4 *>(reinterpret_cast<uint8_t *>(p.ck) + align256((size_t)slots * a.H * DK * a.Dv * sizeof(float)));
   cudaError_t err = cudaMemsetAsync(p.acc, 0, acc_elems * sizeof(float4), stream);
   if (err != cudaSuccess) return err;
   const int smem = (int)sizeof(BwdSmem<T, DK>);
@@ -337,9 +386,9 @@ cudaError_t bwd_t(const BwdArgs &a, void *ws, cudaStream_t stream) {
 
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, bool packed) {
   const long long tokens = packed ? (long long)T : (long long)B * T;
-  const long long slots = tokens / CK + B + 1;
+  const long long slots = tokens / GK + B + 1;
   return align256((size_t)tokens * H * dk * sizeof(float4)) + align256((size_t)tokens * H * dv * sizeof(float)) +
-         (size_t)slots * H * dk * dv * sizeof(float);
+         align256((size_t)slots * H * dk * dv * sizeof(float)) + (size_t)B * H * GS * dk * dv * sizeof(float);
 }
 
 cudaError_t launch_chunk_bwd(const BwdArgs &a, bool bf16, void *ws, cudaStream_t stream) {

@@ -196,8 +196,9 @@ GDN2_API gdn2_status gdn2_recurrent_fwd(const void *q, const void *k, const void
  * Arithmetic is fp32; the gradients are rounded to dtype once.  dq, dk, dalpha and db are sums
  * over 16-column tiles of the state formed with fp32 reductions in L2, so their last bits may
  * differ from run to run; dv, dw and dS0 are reproducible.  The call takes a workspace of
- * gdn2_chunk_bwd_workspace_bytes() bytes from the library's pool (a gradient accumulator and
- * state checkpoints every 4 tokens) and gives it back on `stream`.  Errors as for gdn2_chunk_fwd.
+ * gdn2_chunk_bwd_workspace_bytes() bytes from the library's pool (a gradient accumulator, the
+ * per-token d_t, state checkpoints every 64 tokens and a per-(sequence, head) scratch of 16 states)
+ * and gives it back on `stream`.  Errors as for gdn2_chunk_fwd.
  */
 GDN2_API gdn2_status gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *alpha,
                                     const void *b, const void *w, const float *S0, const void *dO,
