@@ -650,12 +650,18 @@ __global__ void __launch_bounds__(wy::NT, 2)
           for (int y = 0; y < 4; ++y)
             st_s128(sm + OFF_AL + khalf * 8192 + sw128(row, 32 * part + 8 * y), pack8(&v[8 * y]));
         }
-      } else {  // Pt = P T -> rows 64..127 of the products; warp group khalf takes 32 columns
+      } else {  // Pt = P T -> rows 64..127 of the products; warp group khalf takes 32 columns.  Pt is
+                // written twice, as rows 0..63 and 64..127 of pass 2's A operand, so that Pt A_m
+                // lands in all 128 lanes and every warp can read its share of it
         float v[32];
         tmem_ld32(tl + 128 + 32 * khalf, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int y = 0; y < 4; ++y) st_s128(sm + OFF_TS + sw128(row - 64, 32 * khalf + 8 * y), pack8(&v[8 * y]));
+        for (int y = 0; y < 4; ++y) {
+          const uint4 x = pack8(&v[8 * y]);
+          st_s128(sm + OFF_TS + sw128(row - 64, 32 * khalf + 8 * y), x);
+          st_s128(sm + OFF_TS + 8192 + sw128(row - 64, 32 * khalf + 8 * y), x);
+        }
       }
       {  // Nt = Diag(e^{g_C-m}) K_m^T T, key channel `row`, tokens 32 khalf .. +31
         float v[32];
@@ -680,7 +686,7 @@ __global__ void __launch_bounds__(wy::NT, 2)
     }
 
     // ------------------------------------------------------------ product pass 2: K_m^T W' and [Pt; *] A_m
-    // TMEM cols 0..127: K_m^T W'; cols 128..255: rows 0..63 Pt A_m (rows 64..127 read whatever follows Pt)
+    // TMEM cols 0..127: K_m^T W'; cols 128..255: Pt A_m in rows 0..63 and again in rows 64..127
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
@@ -730,30 +736,30 @@ __global__ void __launch_bounds__(wy::NT, 2)
           for (int y = 0; y < 4; ++y) st_s128(dst + sw128(row, 32 * part + 8 * y), pack8(&v[8 * y]));
         }
       };
-      if (quad < 2) {  // Qt = (Q_m - Pt A_m) Diag(e^m) in place of A_m, channel block khalf (warps 0, 1, 4, 5)
+      {  // Qt = (Q_m - Pt A_m) Diag(e^m) in place of A_m: warp (quad, khalf) takes tokens
+         // 32 (quad & 1) .. +31 of columns 32 (quad >> 1) .. +31 of channel block khalf (quads 2
+         // and 3 read the copy of Pt A_m in lanes 64..127)
+        const int trow = 32 * (quad & 1) + lane, part = quad >> 1;
         uint8_t *blk = sm + OFF_XA + khalf * XA_BLK;
+        float v[32];
+        tmem_ld32(tl + 128 + 64 * khalf + 32 * part, v);
+        tmem_wait_ld();
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          float v[32];
-          tmem_ld32(tl + 128 + 64 * khalf + 32 * part, v);
-          tmem_wait_ld();
+        for (int y = 0; y < 4; ++y) {
+          const int col = 32 * part + 8 * y;
+          float qm[8], e[8];
+          unpack8(ld_s128(blk + 8192 + sw128(trow, col)), qm);
 #pragma unroll
-          for (int y = 0; y < 4; ++y) {
-            const int col = 32 * part + 8 * y;
-            float qm[8], e[8];
-            unpack8(ld_s128(blk + 8192 + sw128(row, col)), qm);
-#pragma unroll
-            for (int t = 0; t < 8; t += 2) {
-              const float2 dq = __fadd2_rn(make_float2(qm[t], qm[t + 1]), make_float2(-v[8 * y + t], -v[8 * y + t + 1]));
-              const float2 r = __fmul2_rn(dq, *reinterpret_cast<const float2 *>(&s_em[64 * khalf + col + t]));
-              e[t] = r.x;
-              e[t + 1] = r.y;
-            }
-            st_s128(blk + sw128(row, col), pack8(e));
+          for (int t = 0; t < 8; t += 2) {
+            const float2 dq = __fadd2_rn(make_float2(qm[t], qm[t + 1]), make_float2(-v[8 * y + t], -v[8 * y + t + 1]));
+            const float2 r = __fmul2_rn(dq, *reinterpret_cast<const float2 *>(&s_em[64 * khalf + col + t]));
+            e[t] = r.x;
+            e[t + 1] = r.y;
           }
+          st_s128(blk + sw128(trow, col), pack8(e));
         }
         fence_proxy_async();
-        group_sync(1, 128);  // the four Qt warps: every Qt tile written, every Q_m row read
+        __syncthreads();  // every Qt tile written, every Q_m row read
         if (tid == ST_TID) {  // Qt -> workspace; the next record's q into the dead Q_m rows
           tma_store_2d(&tm_wq, 0, rec * 64, sb + OFF_XA);
           tma_store_2d(&tm_wq, 64, rec * 64, sb + OFF_XA + XA_BLK);
