@@ -76,8 +76,30 @@ def lib():
         L.gdn2_chunk_bwd.restype = ci
         L.gdn2_chunk_bwd_workspace_bytes.argtypes = [ci] * 6
         L.gdn2_chunk_bwd_workspace_bytes.restype = ctypes.c_size_t
+        L.gdn2_chunk_fwd_plan.argtypes = [ci] * 9 + [ctypes.POINTER(ChunkPlan)]
+        L.gdn2_chunk_fwd_plan.restype = ci
         _lib = L
     return _lib
+
+
+class ChunkPlan(ctypes.Structure):
+    """``gdn2_chunk_plan`` of include/gdn2.h."""
+    _fields_ = [("records", ctypes.c_longlong), ("wy_ctas", ctypes.c_longlong), ("state_ctas", ctypes.c_longlong),
+                ("segments", ctypes.c_int), ("segment_chunks", ctypes.c_int), ("handover_sms", ctypes.c_int),
+                ("handover_at", ctypes.c_longlong), ("order", ctypes.c_int), ("launches", ctypes.c_int),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
+def chunk_fwd_plan(B, T, H, dk, dv, packed=False, sms=0, dtype=torch.bfloat16, chunk=64) -> dict:
+    """What a tensor-core ``chunk_fwd`` call of this shape decides before it launches, for a device
+    of ``sms`` SMs (0: the current one): records, grids, segments, the SM hand-over, the walking
+    order, launches and workspace bytes.  Host only; raises ``Gdn2Error`` when the shape does not
+    take the tensor-core path."""
+    plan = ChunkPlan()
+    st = lib().gdn2_chunk_fwd_plan(B, T, H, dk, dv, chunk, 1 if packed else 0, _DTYPES[dtype], sms, ctypes.byref(plan))
+    if st != GDN2_OK:
+        raise Gdn2Error(st, "chunk_fwd_plan")
+    return {name: int(getattr(plan, name)) for name, _ in ChunkPlan._fields_}
 
 
 def chunk_fwd_workspace_bytes(B, T, H, dk, dv, packed=False, dtype=torch.bfloat16, chunk=64) -> int:

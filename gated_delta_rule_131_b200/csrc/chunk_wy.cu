@@ -44,6 +44,7 @@
 // range); every workload here is far inside it.
 #include <cuda.h>
 
+#include <algorithm>
 #include <climits>
 #include <cstring>
 
@@ -1484,6 +1485,43 @@ int handover_stop(long long records, long long walks, int nc, int sms) {
   return stop > 0 ? (int)stop : 0;
 }
 
+// Everything a call decides before it launches: the workspace layout, the grids, the walking order
+// and the SM hand-over.
+struct Plan {
+  WsLayout L;
+  bool wy_runs;        // a token and a record exist
+  long long wy_ctas;   // persistent WY CTAs (two per SM)
+  long long sp_ctas;   // CTAs of the first state-pass launch
+  long long walks;     // (sequence, head, 128-column) walks
+  int order, reserve, stop_at, publish;
+  int launches;
+};
+Plan make_plan(int B, int T, int H, int dv, bool packed, int sms) {
+  Plan P{};
+  P.L = ws_layout(B, T, H, dv, packed, sms);
+  const long long tokens = packed ? (long long)T : (long long)B * T;
+  const long long tiles = (dv + sp::VW - 1) / sp::VW;
+  P.wy_runs = P.L.records > 0 && tokens > 0;
+  P.wy_ctas = P.wy_runs ? std::min<long long>(P.L.records, 2LL * sms) : 0;
+  P.walks = (long long)B * H * tiles;
+  P.order = packed ? 0 : 1;
+  P.reserve = 0;
+  P.stop_at = (int)P.L.records;
+  P.publish = 0;
+  if (!packed && P.L.nseg <= 1) {  // whole-sequence walks that leave SMs free: hand SMs over early
+    const int stop = handover_stop(P.L.records, P.walks, (T + C - 1) / C, sms);
+    if (stop >= 0) {
+      P.order = 2;
+      P.publish = 1;
+      P.reserve = (int)P.walks;
+      P.stop_at = stop;
+    }
+  }
+  P.sp_ctas = P.L.nseg <= 1 ? P.walks : (long long)B * H * (P.L.nseg - 1) * (1 + tiles);
+  P.launches = (packed ? 1 : 0) + (P.wy_runs ? 1 : 0) + (P.L.nseg <= 1 ? 1 : 3);
+  return P;
+}
+
 }  // namespace
 
 bool chunk_wy_supported(int B, int T, int H, int dk, int dv, bool packed, bool bf16) {
@@ -1497,10 +1535,27 @@ size_t chunk_wy_workspace_bytes(int B, int T, int H, int dv, bool packed) {
   return ws_layout(B, T, H, dv, packed, device_sms()).total;
 }
 
+ChunkWyPlan chunk_wy_plan(int B, int T, int H, int dv, bool packed, int sms) {
+  const Plan P = make_plan(B, T, H, dv, packed, sms > 0 ? sms : device_sms());
+  ChunkWyPlan r{};
+  r.records = P.L.records;
+  r.wy_ctas = P.wy_ctas;
+  r.state_ctas = P.sp_ctas;
+  r.segments = P.L.nseg;
+  r.segment_chunks = P.L.nseg > 1 ? P.L.seg_len : 0;
+  r.handover_sms = P.reserve;
+  r.handover_at = P.reserve > 0 ? P.stop_at : P.L.records;
+  r.order = P.order;
+  r.launches = P.launches;
+  r.workspace_bytes = P.L.total;
+  return r;
+}
+
 cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   const long long tokens = a.cu ? (long long)a.T : (long long)a.B * a.T;
   const int sms = device_sms();
-  const WsLayout L = ws_layout(a.B, a.T, a.H, a.dv, a.cu != nullptr, sms);
+  const Plan P = make_plan(a.B, a.T, a.H, a.dv, a.cu != nullptr, sms);
+  const WsLayout &L = P.L;
   uint8_t *base = static_cast<uint8_t *>(ws);
   WyParams p;
   cudaError_t err = device_status_word(&p.status);
@@ -1514,22 +1569,13 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   p.next = reinterpret_cast<int *>(base + L.cnt);
   p.ready = reinterpret_cast<int *>(base + L.cnt + 256);
   p.done = p.next + 1;
-  p.ctas = 0;
-  p.publish = 0;
+  p.ctas = (int)P.wy_ctas;
+  p.publish = P.publish;
   p.sms = sms;
-  p.reserve = 0;
-  p.stop_at = p.nrec;
-  p.order = a.cu ? 0 : 1;
+  p.reserve = P.reserve;
+  p.stop_at = P.stop_at;
+  p.order = P.order;
   const long long tiles = (a.dv + sp::VW - 1) / sp::VW;
-  if (!a.cu && L.nseg <= 1) {  // whole-sequence walks that leave SMs free: hand SMs over early
-    const int stop = handover_stop(L.records, (long long)a.B * a.H * tiles, p.nc, sms);
-    if (stop >= 0) {
-      p.order = 2;
-      p.publish = 1;
-      p.reserve = (int)((long long)a.B * a.H * tiles);
-      p.stop_at = stop;
-    }
-  }
 
   CUtensorMap mq, mk, mb, mal, mv, mw, mo, mm, mn, mqt, mp;
   if (tokens > 0) {
@@ -1554,15 +1600,13 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
     chunk_offsets_kernel<<<1, 1024, 0, stream>>>(a.cu, a.B, const_cast<int32_t *>(p.coff));
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
-  const bool wy_runs = L.records > 0 && tokens > 0;
+  const bool wy_runs = P.wy_runs;
   if (wy_runs) {
     if ((err = cudaMemsetAsync(p.next, 0, 256 + (size_t)L.records * 4, stream)) != cudaSuccess) return err;
     err = cudaFuncSetAttribute(wy_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wy::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     note_launch();
-    const long long grid = L.records < 2LL * sms ? L.records : 2LL * sms;  // persistent: two CTAs per SM
-    p.ctas = (int)grid;
-    wy_factor_kernel<<<(unsigned)grid, wy::NT, wy::SMEM_BYTES, stream>>>(a, p, mq, mk, mb, mal, mm, mn, mqt, mp);
+    wy_factor_kernel<<<(unsigned)P.wy_ctas, wy::NT, wy::SMEM_BYTES, stream>>>(a, p, mq, mk, mb, mal, mm, mn, mqt, mp);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   err = cudaFuncSetAttribute(state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp::SMEM_BYTES);
@@ -1585,7 +1629,7 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   };
   ScanParams q{};
   if (L.nseg <= 1)  // one walk per (sequence, head, value tile)
-    return state_pass(a.B * a.H * tiles, q, wy_runs);
+    return state_pass(P.sp_ctas, q, wy_runs);
   // two-level scan: segment maps, their chain into entry states, then the segments' walks
   q.seg_len = L.seg_len;
   q.nseg = L.nseg;
@@ -1593,7 +1637,7 @@ cudaError_t launch_chunk_wy(const ChunkArgs &a, void *ws, cudaStream_t stream) {
   q.sum_b = reinterpret_cast<float *>(base + L.sbm);
   q.s_start = reinterpret_cast<float *>(base + L.ss);
   q.mode = 1;
-  if ((err = state_pass((long long)a.B * a.H * (L.nseg - 1) * (1 + tiles), q, wy_runs)) != cudaSuccess) return err;
+  if ((err = state_pass(P.sp_ctas, q, wy_runs)) != cudaSuccess) return err;
   const int chain_smem = (128 * 132 + 32 * 132) * 4;
   err = cudaFuncSetAttribute(segment_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, chain_smem);
   if (err != cudaSuccess) return err;

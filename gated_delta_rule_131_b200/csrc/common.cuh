@@ -98,6 +98,15 @@ cudaError_t launch_chunk_simt(const ChunkArgs &a, bool bf16, cudaStream_t stream
 // The workspace depends only on the batch shape (B sequences, T tokens each or in total, H heads, d_v).
 bool chunk_wy_supported(int B, int T, int H, int dk, int dv, bool packed, bool bf16);
 size_t chunk_wy_workspace_bytes(int B, int T, int H, int dv, bool packed);
+// The launch plan of that path for a device of `sms` SMs (0: the current device); host only.
+struct ChunkWyPlan {
+  long long records, wy_ctas, state_ctas;
+  int segments, segment_chunks, handover_sms;
+  long long handover_at;
+  int order, launches;
+  size_t workspace_bytes;
+};
+ChunkWyPlan chunk_wy_plan(int B, int T, int H, int dv, bool packed, int sms);
 // Backward of the recurrence over a workspace of chunk_bwd_workspace_bytes(...) bytes, 256-byte
 // aligned (a gradient accumulator it clears, and state checkpoints it writes before reading).
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, bool packed);

@@ -163,8 +163,8 @@ gdn2_status check_chunk(const void *q, const void *k, const void *v, const void 
   if (!fits(tokens, H, d_v > d_k ? d_v : d_k, 1) || !fits(B, H, d_k, d_v)) return GDN2_ERR_INVALID_ARG;
   if ((long long)B * H * 8 > INT_MAX) return GDN2_ERR_INVALID_ARG;
   *a = gdn2::ChunkArgs{q, k, v, alpha, b, w, S0, o, S_T, cu_seqlens, B, T, H, d_k, d_v};
-  // bf16 with d_v a multiple of 128 runs on the tensor cores; fp32 (whose accuracy bf16 operands
-  // cannot keep) and bf16 with d_v = 64 run the SIMT kernel
+  // bf16 runs on the tensor cores (unless too large for their 32-bit TMA coordinates); fp32, whose
+  // accuracy bf16 operands cannot keep, runs the SIMT kernel
   *tc = gdn2::chunk_wy_supported(B, T, H, d_k, d_v, cu_seqlens != nullptr, dtype == GDN2_BF16);
   return GDN2_OK;
 }
@@ -251,6 +251,26 @@ gdn2_status gdn2_recurrent_fwd(const void *q, const void *k, const void *v, cons
 size_t gdn2_chunk_bwd_workspace_bytes(int B, int T, int H, int d_k, int d_v, int packed) {
   if (B <= 0 || T < 0 || H <= 0 || !supported_dk(d_k) || !supported_dv(d_v)) return 0;
   return gdn2::chunk_bwd_workspace_bytes(B, T, H, d_k, d_v, packed != 0);
+}
+
+gdn2_status gdn2_chunk_fwd_plan(int B, int T, int H, int d_k, int d_v, int chunk, int packed, gdn2_dtype dtype,
+                                int sms, gdn2_chunk_plan *plan) {
+  if (!plan || B < 0 || T < 0 || H <= 0 || sms < 0) return GDN2_ERR_INVALID_ARG;
+  if (dtype != GDN2_F32 && dtype != GDN2_BF16) return GDN2_ERR_INVALID_ARG;
+  if (!supported_dk(d_k) || !supported_dv(d_v) || chunk != 64) return GDN2_ERR_UNSUPPORTED;
+  if (!gdn2::chunk_wy_supported(B, T, H, d_k, d_v, packed != 0, dtype == GDN2_BF16)) return GDN2_ERR_UNSUPPORTED;
+  const gdn2::ChunkWyPlan r = gdn2::chunk_wy_plan(B, T, H, d_v, packed != 0, sms);
+  plan->records = r.records;
+  plan->wy_ctas = r.wy_ctas;
+  plan->state_ctas = r.state_ctas;
+  plan->segments = r.segments;
+  plan->segment_chunks = r.segment_chunks;
+  plan->handover_sms = r.handover_sms;
+  plan->handover_at = r.handover_at;
+  plan->order = r.order;
+  plan->launches = r.launches;
+  plan->workspace_bytes = r.workspace_bytes;
+  return GDN2_OK;
 }
 
 size_t gdn2_chunk_fwd_workspace_bytes(int B, int T, int H, int d_k, int d_v, int chunk, int packed,

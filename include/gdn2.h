@@ -95,13 +95,14 @@ typedef struct CUstream_st *gdn2_stream_t;
  * chunk: 64 (the only supported chunk length).
  * T == 0 (or an empty sequence) is valid: its S_T equals its S0; when the
  * batch holds no token at all, the token pointers (q .. w, o) may be NULL.
- * bf16 with d_v = 128 or 256 (d_k = 64 or 128) runs two tensor-core kernels over a workspace: the
+ * bf16 (d_k = 64 or 128, d_v = 64, 128 or 256) runs two tensor-core kernels over a workspace: the
  * first forms the chunk's WY factors (T = (I + L)^-1, W = -T A, and the decay-
  * absorbed q and k) for every chunk at once, the second carries the state
  * through each sequence's chunks in order (d_k = 64 is carried as 128 key
- * channels whose upper half stays zero); fp32, and bf16 with d_v = 64, run one
- * SIMT kernel without a workspace (bf16 tensor-core operands cannot keep the
- * fp32 tolerance; the second kernel takes 128 value columns per CTA).
+ * channels whose upper half stays zero, d_v = 64 as a 128-column tile whose
+ * upper half stays zero); fp32 runs one SIMT kernel without a workspace (bf16
+ * tensor-core operands cannot keep the fp32 tolerance), as do bf16 shapes too
+ * large for the kernels' 32-bit TMA coordinates.
  * Returns GDN2_OK, or an error status with nothing launched; GDN2_ERR_CUDA
  * also when the workspace cannot be allocated.
  */
@@ -146,6 +147,37 @@ GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const void *q, const void *k, const 
  */
 GDN2_API size_t gdn2_chunk_fwd_workspace_bytes(int B, int T, int H, int d_k, int d_v, int chunk, int packed,
                                                gdn2_dtype dtype);
+
+/*
+ * gdn2_chunk_plan / gdn2_chunk_fwd_plan -- what a tensor-core gdn2_chunk_fwd call of this shape
+ * decides before it launches, for a device of `sms` SMs (0: the current device, which is then
+ * queried; no other CUDA call is made and nothing is launched or allocated).  It has no
+ * counterpart in the pages: it describes how this library schedules the chunkwise form.
+ *   records          (chunk, head) records the WY kernel writes (a packed batch: its chunk
+ *                    capacity, sum over sequences of ceil(len / 64) at most, times H)
+ *   wy_ctas          persistent WY-kernel CTAs (two per SM, at most one per record)
+ *   state_ctas       CTAs of the first state-pass launch
+ *   segments         segments per (sequence, head, 128-column) walk of the two-level scan, 1 for
+ *                    whole-sequence walks; segment_chunks their length in chunks (0 when 1)
+ *   handover_sms     SMs whose WY CTAs stop claiming records early so that the state pass runs
+ *                    there alongside the rest of the factorisation (0: none)
+ *   handover_at      records claimed before they stop (records when handover_sms is 0)
+ *   order            the WY kernel's walking order: 0 record order (packed batches), 1 chunk-major
+ *                    with the last chunk first, 2 chunk-major with the first chunk first
+ *   launches         kernel launches of the call
+ *   workspace_bytes  as gdn2_chunk_fwd_workspace_bytes() for that SM count
+ * Returns GDN2_OK; GDN2_ERR_INVALID_ARG for a NULL plan or a negative size; GDN2_ERR_UNSUPPORTED
+ * when the shape does not take the tensor-core path (fp32, or sizes outside it).
+ */
+typedef struct gdn2_chunk_plan {
+  long long records, wy_ctas, state_ctas;
+  int segments, segment_chunks, handover_sms;
+  long long handover_at;
+  int order, launches;
+  size_t workspace_bytes;
+} gdn2_chunk_plan;
+GDN2_API gdn2_status gdn2_chunk_fwd_plan(int B, int T, int H, int d_k, int d_v, int chunk, int packed,
+                                         gdn2_dtype dtype, int sms, gdn2_chunk_plan *plan);
 
 /*
  * gdn2_recurrent_fwd -- the token-by-token recurrence over whole sequences, in either reading of

@@ -269,3 +269,57 @@ def test_recurrent_validation(L):
     assert recurrent(L, [None] * 9, B=0, T=0) == gdn2.GDN2_OK
     assert L.gdn2_launch_count() == before
 
+
+
+def plan(L, B, T, H, dk=128, dv=128, packed=0, sms=148, dtype=gdn2.GDN2_BF16):
+    p = gdn2.ChunkPlan()
+    st = L.gdn2_chunk_fwd_plan(B, T, H, dk, dv, 64, packed, dtype, sms, ctypes.byref(p))
+    return st, {name: getattr(p, name) for name, _ in gdn2.ChunkPlan._fields_}
+
+
+def test_chunk_fwd_plan(L):
+    """The launch plan of the tensor-core path (host arithmetic only; nothing is launched)."""
+    before = L.gdn2_launch_count()
+    # 1.3B layer on 148 SMs: 2048 records over 296 persistent WY CTAs; 64 whole-sequence walks leave
+    # 84 SMs, so the CTAs on 64 SMs stop claiming at records - floor(2 (148 - 64) 32 x 1.9 / 9)
+    st, p = plan(L, 4, 2048, 16)
+    assert st == gdn2.GDN2_OK
+    assert (p["records"], p["wy_ctas"], p["state_ctas"], p["segments"], p["launches"]) == (2048, 296, 64, 1, 2)
+    assert p["handover_sms"] == 64 and p["order"] == 2
+    assert p["handover_at"] == 2048 - int(2 * 84 * 32 * 1.9 / 9)
+    assert p["workspace_bytes"] == L.gdn2_chunk_fwd_workspace_bytes(4, 2048, 16, 128, 128, 64, 0, gdn2.GDN2_BF16)
+    # fewer SMs leave fewer for the rest of the factorisation: the hand-over comes later
+    st, p100 = plan(L, 4, 2048, 16, sms=100)
+    assert p100["wy_ctas"] == 200 and p100["handover_at"] == 2048 - int(2 * 36 * 32 * 1.9 / 9)
+    # walks that fill the GPU: no hand-over, last chunk first
+    st, p = plan(L, 64, 2048, 16)
+    assert (p["state_ctas"], p["handover_sms"], p["handover_at"], p["order"]) == (1024, 0, 32768, 1)
+    # d_v = 256: two 128-column walks per (sequence, head)
+    st, p = plan(L, 4, 2048, 16, dv=256)
+    assert p["state_ctas"] == 128 and p["handover_sms"] == 128
+    # one long sequence: the two-level scan (summaries, chain, walks), no hand-over
+    st, p = plan(L, 1, 65536, 16)
+    assert p["segments"] > 1 and p["segments"] * p["segment_chunks"] >= 1024 > (p["segments"] - 1) * p["segment_chunks"]
+    assert p["segment_chunks"] >= 16 and p["launches"] == 4 and p["handover_sms"] == 0 and p["order"] == 1
+    assert p["state_ctas"] == 16 * (p["segments"] - 1) * 2
+    # a packed batch: chunk offsets first, records in record order, no hand-over
+    st, p = plan(L, 32, 156118, 32, dv=256, packed=1)
+    assert (p["launches"], p["order"], p["handover_sms"]) == (3, 0, 0)
+    assert p["records"] == ((156118 + 63 * 32) // 64) * 32 and p["state_ctas"] == 32 * 32 * 2
+    # a single record: a hand-over from the start
+    st, p = plan(L, 1, 64, 1)
+    assert (p["records"], p["wy_ctas"], p["handover_sms"], p["handover_at"]) == (1, 1, 1, 0)
+    # no token: no WY launch
+    st, p = plan(L, 2, 0, 4)
+    assert (p["wy_ctas"], p["launches"]) == (0, 1)
+    # not the tensor-core path, or bad arguments
+    assert plan(L, 4, 2048, 16, dtype=gdn2.GDN2_F32)[0] == gdn2.GDN2_ERR_UNSUPPORTED
+    st, p = plan(L, 4, 2048, 16, dv=64)  # d_v = 64: one 128-column walk per (sequence, head), half of it zero
+    assert st == gdn2.GDN2_OK and p["state_ctas"] == 64
+    assert plan(L, 4, 2048, 16, dk=96)[0] == gdn2.GDN2_ERR_UNSUPPORTED
+    assert plan(L, -1, 2048, 16)[0] == gdn2.GDN2_ERR_INVALID_ARG
+    assert plan(L, 4, 2048, 16, sms=-1)[0] == gdn2.GDN2_ERR_INVALID_ARG
+    assert L.gdn2_chunk_fwd_plan(4, 2048, 16, 128, 128, 64, 0, gdn2.GDN2_BF16, 148, None) == gdn2.GDN2_ERR_INVALID_ARG
+    # the binding returns the same numbers
+    assert gdn2.chunk_fwd_plan(4, 2048, 16, 128, 128, sms=148)["handover_at"] == 2048 - int(2 * 84 * 32 * 1.9 / 9)
+    assert L.gdn2_launch_count() == before
