@@ -9,8 +9,11 @@ collective on the data path: weak scaling).  The same JSON line carries the
 decode measurement (256 x 16 heads, 1024 single-token steps replayed from one
 CUDA graph) as ``decode_step``, the block prologue and epilogue around the mixer
 (``block_prologue``, ``block_epilogue``), the backward on the same workload
-(``chunk_bwd``), the roofline of the dominant kernel, the CPU
-oracle baseline, the end-to-end number through host buffers, and clocks.
+(``chunk_bwd``), the long-context workload with a sequence-length sweep
+(``long_context``), the packed workload with its three gate variants (``varlen``),
+the step sustained for about 0.5 s with its own clock samples (``sustained``), the
+roofline of the chunk forward (its two kernels overlap, so the call is the unit),
+the CPU oracle baseline, the end-to-end number through host buffers, and clocks.
 
 ``--impl reference`` times the fp64 CPU oracle (the only reference that
 exists for this method) on a bounded sample of the same workload.
